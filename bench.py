@@ -1,0 +1,418 @@
+"""Benchmark of the MoE FFN layer (dots.llm1 fine-grained MoE) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload train|layer]
+                    [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch:
+  train (default): T=16384 tokens, d=4096, 128 routed experts top-6 + 2 shared,
+                   I=1408, pad block 128; forward (gate, top-k, permute, grouped
+                   SwiGLU GEMMs, combine) + backward (combine bwd, dX and dW
+                   grouped GEMMs, SwiGLU bwd, un-permute-sum).
+  layer:           T=8192, same layer, forward only.
+Inputs are synthetic (seeded generator), resident in HBM for ``value``; the
+weights alone (4.5 GB) exceed L2, so no flush is needed between steps.
+
+``value`` is whole-job tokens/s (device time, CUDA events, max over ranks);
+``e2e`` is the same metric through the C ABI with the step's inputs copied from
+pinned host memory and its results copied back inside the timed region.
+``--impl reference`` times the FP64 CPU oracle on host cores instead.
+For N > 1 (torchrun) each rank runs an independent replica of the step on its
+own GPU (weak scaling; the single-GPU path has no exchange step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of B200 BF16 peak), 1 GPU"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="train", choices=["train", "layer"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fitted_bias(name):
+    path = os.path.join(ROOT, "tests", "golden", f"{name}_bias.txt")
+    if not os.path.exists(path):
+        return None
+    vals = [float(l) for l in open(path) if l.strip() and not l.startswith("#")]
+    return np.array(vals, dtype=np.float32)
+
+
+def workload(name):
+    import synth
+    wl = synth.WORKLOADS[name]
+    return wl, synth.make_inputs(wl, bias_override=fitted_bias(name))
+
+
+def gemm_flops(dm, backward):
+    """Algorithmic FLOPs of the grouped GEMMs (real rows only: T*k routed + S*T shared)."""
+    R = dm.T * dm.k + dm.S * dm.T
+    fwd1, fwd2 = 2 * R * dm.d * 2 * dm.I, 2 * R * dm.I * dm.d
+    f = {"fwd": fwd1 + fwd2}
+    if backward:
+        f.update(dx2=2 * R * dm.d * dm.I, dw2=2 * R * dm.d * dm.I, dx1=2 * R * 2 * dm.I * dm.d,
+                 dw1=2 * R * 2 * dm.I * dm.d)
+    return f
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=600))
+    elif args.impl == "ours":
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def dist_max(v, world, device=None):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------- CPU (oracle) --
+def oracle_sample_step(wl, inp, ntok):
+    """The oracle on the first ``ntok`` tokens of the workload: gate + route +
+    permute + expert forward (+ backward incl. every group's dW when the
+    workload trains).  Returns seconds."""
+    import oracle
+    dm = wl.dims
+    x = inp["x"][:ntok]
+    t0 = time.perf_counter()
+    lg = oracle.gate_logits(x, inp["wg"])
+    _, idx, w, _ = oracle.route(lg, inp["bias"], dm.k)
+    oracle.permute(idx, dm.E, dm.P, ntok * dm.k + dm.E * (dm.P - 1))
+    oracle.layer_fwd(x, idx, w, inp["w1"], inp["w2"], dm.S)
+    if wl.backward:
+        dout = inp["dout"][:ntok]
+        oracle.layer_bwd(x, idx, w, inp["w1"], inp["w2"], dout, dm.S)
+        used = set(np.unique(idx).tolist()) | set(range(dm.E, dm.E + dm.S))
+        for g in sorted(used):
+            oracle.group_dw(x, idx, w, inp["w1"], inp["w2"], dout, dm.S, g)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, inp, ntok=64):
+    import oracle
+    oracle.build()
+    oracle_sample_step(wl, inp, 2)  # warm the library and the page cache
+    secs = oracle_sample_step(wl, inp, ntok)
+    return {"value": ntok / secs, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {ntok} tokens of the workload, full "
+                      f"{'forward+backward (all dW)' if wl.backward else 'forward'} in FP64, "
+                      f"{secs:.1f} s; tokens/s scales linearly in tokens"}
+
+
+def run_reference(args):
+    # under torchrun only rank 0 runs the oracle; the other ranks have no work
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    wl, inp = workload(args.workload)
+    ntok = 16
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, inp, ntok)
+    total = 0.0
+    for _ in range(args.steps):
+        total += oracle_sample_step(wl, inp, ntok)
+    import oracle
+    val = ntok * args.steps / total
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": describe(wl), "sample_tokens_per_step": ntok},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": f"{ntok} tokens per step, full layer step in FP64"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def describe(wl):
+    dm = wl.dims
+    return (f"{wl.name}: T={dm.T} d={dm.d} E={dm.E} k={dm.k} S={dm.S} I={dm.I} P={dm.P}, "
+            f"{'forward+backward' if wl.backward else 'forward'}")
+
+
+# ---------------------------------------------------------------- GPU (ours) --
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_setup(args)
+    import grouped_gemm_fp32_b200 as moe
+    from grouped_gemm_fp32_b200 import layer
+
+    wl, inp = workload(args.workload)
+    dm = wl.dims
+    dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P)
+    train = wl.backward
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
+    x, w1, w2 = bf(inp["x"]), bf(inp["w1"]), bf(inp["w2"])
+    wg = torch.from_numpy(inp["wg"]).to(dev)
+    bias = torch.from_numpy(inp["bias"]).to(dev)
+    dout = bf(inp["dout"]) if train else None
+    b = layer.MoEBuffers(dims, device=dev, train=train)
+    torch.cuda.synchronize()
+
+    def step(s, xx=x, gg=dout, ev=None):
+        if ev is None:
+            layer.forward(b, xx, wg, bias, w1, w2, stream=s)
+            if train:
+                layer.backward(b, xx, gg, w1, w2, stream=s)
+            return
+        # instrumented: events around each C-ABI call
+        L = moe
+        rec = lambda k: ev[k].append(torch.cuda.Event(enable_timing=True)) or ev[k][-1].record(s)
+        rec("t0")
+        L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, s)
+        rec("gate")
+        L.moe_permute_align(dims, b.topk_idx, xx, b.counts, b.offsets, b.sorted_ids, b.row_of,
+                            b.x_perm, b.ws, s)
+        rec("permute")
+        L.grouped_gemm_fwd(dims, b.ws, b.x_perm, xx, w1, w2, b.h, b.a1, b.y, s)
+        rec("fwd")
+        L.moe_combine(dims, b.y, b.row_of, b.topk_w, b.out, s)
+        rec("combine")
+        if train:
+            L.moe_combine_bwd(dims, b.ws, gg, b.y, b.row_of, b.topk_w, b.dy, b.dw_comb, s)
+            rec("combine_bwd")
+            L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM2, b.dy, gg, w2, b.a1, b.da, s)
+            rec("dx2")
+            L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM2, b.dy, gg, b.h, None, b.dw2, 0, s)
+            rec("dw2")
+            L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, s)
+            rec("dx1")
+            L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, xx, b.dw1, 0, s)
+            rec("dw1")
+            L.moe_combine(dims, b.dxp, b.row_of, None, b.dx, s)
+            rec("unpermute")
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(stream)
+    stream.synchronize()
+    status = moe.moe_get_device_status(b.ws, stream)
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(status)}")
+
+    # ---- timed region: device-resident inputs
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.25)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(stream)
+        e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = dist_max(ms, world, dev)
+    tokens_per_s = world * dm.T / (ms / 1000.0)
+
+    # ---- per-call breakdown (separate instrumented pass; not the headline)
+    names = ["t0", "gate", "permute", "fwd", "combine"] + (
+        ["combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute"] if train else [])
+    ev = {n: [] for n in names}
+    nprof = max(3, min(args.steps, 20))
+    with torch.cuda.stream(stream):
+        for _ in range(nprof):
+            step(stream, ev=ev)
+    stream.synchronize()
+    per = {}
+    for i in range(1, len(names)):
+        a, c = ev[names[i - 1]], ev[names[i]]
+        per[names[i]] = sum(x0.elapsed_time(x1) for x0, x1 in zip(a, c)) / nprof
+    flops = gemm_flops(dm, train)
+    gemm_ms = sum(per[k] for k in flops)
+    gemm_tflops = sum(flops.values()) / (gemm_ms / 1000.0) / 1e12
+    pk, pk_src = peaks()
+    sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    gemm_detail = {k: {"ms": round(per[k], 4), "tflops": round(flops[k] / per[k] / 1e9, 1)}
+                   for k in flops}
+
+    # ---- e2e: pinned host inputs in, results out, through the same C ABI calls
+    hx = torch.from_numpy(inp["x"]).view(torch.bfloat16).pin_memory()
+    hd = torch.from_numpy(inp["dout"]).view(torch.bfloat16).pin_memory() if train else None
+    ho = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory()
+    hdx = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() if train else None
+    dx_in = torch.empty_like(x)
+    dd_in = torch.empty_like(dout) if train else None
+    h2d = hx.numel() * 2 + (hd.numel() * 2 if train else 0)
+    d2h = ho.numel() * 2 + (hdx.numel() * 2 if train else 0)
+
+    def e2e_step():
+        dx_in.copy_(hx, non_blocking=True)
+        if train:
+            dd_in.copy_(hd, non_blocking=True)
+        step(stream, xx=dx_in, gg=dd_in)
+        ho.copy_(b.out, non_blocking=True)
+        if train:
+            hdx.copy_(b.dx, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
+    stream.synchronize()
+    barrier(world)
+    ne2e = max(3, args.steps // 2)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(ne2e):
+            e2e_step()
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = dist_max(f0.elapsed_time(f1) / ne2e, world, dev)
+    status = moe.moe_get_device_status(b.ws, stream)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {moe.moe_status_string(status)}")
+
+    launches_per_step = 1 + 5 + 2 + 1 + ((2 + 4 + 1) if train else 0)
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": describe(wl), "tokens_per_gpu": dm.T,
+                   "global_batch_tokens": world * dm.T,
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "no flush: weights (4.5 GB) and activations exceed the 126 MB L2"},
+        "roofline": {"bound": "tensor", "kernel": "ggemm_kernel (all grouped-GEMM launches)",
+                     "achieved": gemm_tflops, "peak": sustained, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / sustained,
+                     "peak_kind": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
+                     "frac_of_burst_peak": gemm_tflops / pk["bf16_tflops"],
+                     "traffic": None},
+        "grouped_gemm": gemm_detail,
+        "breakdown_ms": {k: round(v, 4) for k, v in per.items()},
+        "e2e": {"value": world * dm.T / (e2e_ms / 1000.0), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, inp)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

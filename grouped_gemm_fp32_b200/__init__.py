@@ -1,0 +1,13 @@
+"""B200 (sm_100a) MoE FFN layer: the dots.llm1 fine-grained MoE hot path.
+
+The compute lives in ``libmoe.so`` (hand-written CUDA, C ABI declared in
+``include/moe.h``).  This package only marshals arguments to it
+(``grouped_gemm_fp32_b200._lib``) and sequences the calls of one layer over
+caller-owned torch buffers (``grouped_gemm_fp32_b200.layer``).  There is no
+CPU or PyTorch fallback: without the built library every call raises.
+"""
+from ._lib import (MOE_GEMM1, MOE_GEMM2, MoeDims, MoeError, grouped_gemm_bwd_dw,  # noqa: F401
+                   grouped_gemm_bwd_dx, grouped_gemm_fwd, grouped_gemm_set_groups, lib_path,
+                   load, moe_combine, moe_combine_bwd, moe_gate_topk, moe_get_device_status,
+                   moe_permute_align, moe_rows_routed, moe_rows_total, moe_status_string,
+                   moe_workspace_size)

@@ -1,0 +1,172 @@
+"""ctypes binding of libmoe.so: one Python function per C entry point, same name.
+
+Arguments are torch CUDA tensors (their ``data_ptr()`` is passed), ``None``
+(NULL) or plain integers.  ``stream`` defaults to torch's current stream.  A
+negative status raises ``MoeError``.  Nothing here computes anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmoe.so")
+_lib = None
+
+MOE_GEMM1, MOE_GEMM2 = 1, 2
+EXPORTS = (
+    "moe_rows_routed", "moe_rows_total", "moe_workspace_size", "moe_gate_topk",
+    "moe_permute_align", "grouped_gemm_set_groups", "grouped_gemm_fwd", "grouped_gemm_bwd_dx",
+    "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd", "moe_get_device_status",
+    "moe_status_string",
+)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {moe_status_string(status)} ({status})")
+        self.status = status
+
+
+class MoeDims(ctypes.Structure):
+    """Mirror of ``struct moe_dims`` in include/moe.h."""
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("S", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("P", ctypes.c_int32), ("rows_cap", ctypes.c_int64)]
+
+    @classmethod
+    def of(cls, T, d, E, k, S, I, P, rows_cap=0):
+        return cls(int(T), int(d), int(E), int(k), int(S), int(I), int(P), int(rows_cap))
+
+    def __repr__(self):
+        return ("MoeDims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libmoe.so (built in-tree by ``grouped_gemm_fp32_b200.build``); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m grouped_gemm_fp32_b200.build` (there is no fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    D = ctypes.POINTER(MoeDims)
+    sig = {
+        "moe_rows_routed": (i64, [D]),
+        "moe_rows_total": (i64, [D]),
+        "moe_workspace_size": (sz, [D]),
+        "moe_gate_topk": (i32, [D, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_permute_align": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "grouped_gemm_set_groups": (i32, [D, vp, vp, vp, sz, vp]),
+        "grouped_gemm_fwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "grouped_gemm_bwd_dx": (i32, [D, vp, i32, vp, vp, vp, vp, vp, vp]),
+        "grouped_gemm_bwd_dw": (i32, [D, vp, i32, vp, vp, vp, vp, vp, i32, vp]),
+        "moe_combine": (i32, [D, vp, vp, vp, vp, vp]),
+        "moe_combine_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_get_device_status": (i32, [vp, vp, vp]),
+        "moe_status_string": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _p(t):
+    """Device pointer of a tensor (or an int address), NULL for None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ck(rc: int, what: str):
+    if rc != 0:
+        raise MoeError(rc, what)
+
+
+def moe_status_string(status: int) -> str:
+    return load().moe_status_string(int(status)).decode()
+
+
+def moe_rows_routed(dims: MoeDims) -> int:
+    return int(load().moe_rows_routed(ctypes.byref(dims)))
+
+
+def moe_rows_total(dims: MoeDims) -> int:
+    return int(load().moe_rows_total(ctypes.byref(dims)))
+
+
+def moe_workspace_size(dims: MoeDims) -> int:
+    return int(load().moe_workspace_size(ctypes.byref(dims)))
+
+
+def moe_gate_topk(dims, x, wg, bias, topk_idx, topk_w, probs=None, stream=None):
+    _ck(load().moe_gate_topk(ctypes.byref(dims), _p(x), _p(wg), _p(bias), _p(topk_idx),
+                             _p(topk_w), _p(probs), _s(stream)), "moe_gate_topk")
+
+
+def moe_permute_align(dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_perm, ws,
+                      stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _ck(load().moe_permute_align(ctypes.byref(dims), _p(topk_idx), _p(x), _p(counts),
+                                 _p(offsets), _p(sorted_ids), _p(row_of), _p(x_perm), _p(ws),
+                                 nbytes, _s(stream)), "moe_permute_align")
+
+
+def grouped_gemm_set_groups(dims, counts, offsets, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _ck(load().grouped_gemm_set_groups(ctypes.byref(dims), _p(counts), _p(offsets), _p(ws),
+                                       nbytes, _s(stream)), "grouped_gemm_set_groups")
+
+
+def grouped_gemm_fwd(dims, ws, x_perm, x, w1, w2, h, a1, y, stream=None):
+    _ck(load().grouped_gemm_fwd(ctypes.byref(dims), _p(ws), _p(x_perm), _p(x), _p(w1), _p(w2),
+                                _p(h), _p(a1), _p(y), _s(stream)), "grouped_gemm_fwd")
+
+
+def grouped_gemm_bwd_dx(dims, ws, which, dy_routed, dy_shared, w, a1, out, stream=None):
+    _ck(load().grouped_gemm_bwd_dx(ctypes.byref(dims), _p(ws), int(which), _p(dy_routed),
+                                   _p(dy_shared), _p(w), _p(a1), _p(out), _s(stream)),
+        "grouped_gemm_bwd_dx")
+
+
+def grouped_gemm_bwd_dw(dims, ws, which, lhs_routed, lhs_shared, rhs_routed, rhs_shared, dw,
+                        accumulate=0, stream=None):
+    _ck(load().grouped_gemm_bwd_dw(ctypes.byref(dims), _p(ws), int(which), _p(lhs_routed),
+                                   _p(lhs_shared), _p(rhs_routed), _p(rhs_shared), _p(dw),
+                                   int(accumulate), _s(stream)), "grouped_gemm_bwd_dw")
+
+
+def moe_combine(dims, y, row_of, topk_w, out, stream=None):
+    _ck(load().moe_combine(ctypes.byref(dims), _p(y), _p(row_of), _p(topk_w), _p(out),
+                           _s(stream)), "moe_combine")
+
+
+def moe_combine_bwd(dims, ws, dout, y, row_of, topk_w, dy_routed, dw, stream=None):
+    _ck(load().moe_combine_bwd(ctypes.byref(dims), _p(ws), _p(dout), _p(y), _p(row_of),
+                               _p(topk_w), _p(dy_routed), _p(dw), _s(stream)), "moe_combine_bwd")
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _ck(load().moe_get_device_status(_p(ws), ctypes.addressof(out), _s(stream)),
+        "moe_get_device_status")
+    return int(out.value)

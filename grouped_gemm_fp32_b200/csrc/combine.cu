@@ -1,0 +1,154 @@
+// combine.cu -- weighted un-permute / combine of the expert outputs, and its
+// backward.
+//
+// Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer":
+// a token's output sums its top-6 routed experts (weighted) and the 2 shared
+// experts that every token uses.
+//
+// HBM-bound; one warp per token, 16-byte vector accesses along the hidden
+// dimension, FP32 accumulation.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ void acc8(float* a, uint4 v, float w) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    a[2 * p] = fmaf(w, __uint_as_float(u[p] << 16), a[2 * p]);
+    a[2 * p + 1] = fmaf(w, __uint_as_float(u[p] & 0xFFFF0000u), a[2 * p + 1]);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* a) {
+  uint4 r;
+  uint32_t* u = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(a[2 * p], a[2 * p + 1]);
+    u[p] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  return r;
+}
+
+// out[t] = sum_j w[t, j] y[row_of[t, j]] + sum_s y[Rr + s T + t]
+template <int KMAX>
+__global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
+                               const float* __restrict__ w, int64_t T, int row_vec, int k, int S,
+                               int64_t Rr, uint4* __restrict__ out) {
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int64_t rows[KMAX];
+  float wt[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k) {
+      rows[j] = (int64_t)row_of[t * k + j] * row_vec;
+      wt[j] = w ? w[t * k + j] : 1.0f;
+    } else if (j < k + S) {
+      rows[j] = (Rr + (int64_t)(j - k) * T + t) * row_vec;
+      wt[j] = 1.0f;
+    }
+  }
+  for (int c = lane; c < row_vec; c += 32) {
+    float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint4 v[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k + S) v[j] = y[rows[j] + c];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k + S) acc8(a, v[j], wt[j]);
+    out[t * row_vec + c] = pack8(a);
+  }
+}
+
+// Generic fallback (any k + S): rows gathered on the fly.
+__global__ void combine_kernel_any(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
+                                   const float* __restrict__ w, int64_t T, int row_vec, int k,
+                                   int S, int64_t Rr, uint4* __restrict__ out) {
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  for (int c = lane; c < row_vec; c += 32) {
+    float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k + S; ++j) {
+      const int64_t r = j < k ? (int64_t)row_of[t * k + j] : Rr + (int64_t)(j - k) * T + t;
+      acc8(a, y[r * row_vec + c], j < k ? (w ? w[t * k + j] : 1.0f) : 1.0f);
+    }
+    out[t * row_vec + c] = pack8(a);
+  }
+}
+
+// dy[row_of[t, j]] = w[t, j] dout[t] (bf16);  dw[t, j] = <dout[t], y[row_of[t, j]]>
+__global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
+                                   const int32_t* __restrict__ row_of, const float* __restrict__ w,
+                                   int64_t T, int row_vec, int k, uint4* __restrict__ dy,
+                                   float* __restrict__ dw) {
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  for (int j = 0; j < k; ++j) {
+    const int64_t r = row_of[t * k + j];
+    const float wj = w[t * k + j];
+    float dot = 0.0f;
+    for (int c = lane; c < row_vec; c += 32) {
+      const uint4 g = dout[t * row_vec + c];
+      const uint4 yv = y[r * row_vec + c];
+      float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      acc8(a, g, wj);
+      dy[r * row_vec + c] = pack8(a);
+      const uint32_t gu[4] = {g.x, g.y, g.z, g.w}, yu[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        dot = fmaf(__uint_as_float(gu[p] << 16), __uint_as_float(yu[p] << 16), dot);
+        dot = fmaf(__uint_as_float(gu[p] & 0xFFFF0000u), __uint_as_float(yu[p] & 0xFFFF0000u), dot);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane == 0) dw[t * k + j] = dot;
+  }
+}
+
+}  // namespace
+
+int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream);
+
+int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, const float* w,
+                   void* out, void* stream) {
+  if (dm.T == 0) return MOE_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int warps = 8;
+  const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);
+  const int row_vec = dm.d / 8;
+  const int64_t Rr = rows_routed(dm);
+  const uint4* yv = reinterpret_cast<const uint4*>(y);
+  uint4* o = reinterpret_cast<uint4*>(out);
+  if (dm.k + dm.S <= 8)
+    combine_kernel<8><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k, dm.S, Rr, o);
+  else
+    combine_kernel_any<<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k, dm.S, Rr,
+                                                      o);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
+                       const int32_t* row_of, const float* w, void* dy, float* dw, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int rc = launch_zero_pad_rows(dm, ws, dy, dm.d, stream);
+  if (rc != MOE_OK || dm.T == 0) return rc;
+  const int warps = 8;
+  const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);
+  combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(
+      reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), row_of, w, dm.T,
+      dm.d / 8, dm.k, reinterpret_cast<uint4*>(dy), dw);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

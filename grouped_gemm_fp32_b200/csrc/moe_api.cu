@@ -1,0 +1,186 @@
+// moe_api.cu -- the extern "C" entry points of libmoe.so: argument and shape
+// validation, then the launches.  No allocation, no host synchronisation
+// (except moe_get_device_status), nothing but plain pointers and sizes.
+#include <cuda_runtime.h>
+
+#include "moe_internal.cuh"
+
+using namespace moe;
+
+namespace {
+
+bool dims_ok(const moe_dims* dm) {
+  if (!dm) return false;
+  if (dm->T < 0 || dm->d <= 0 || dm->E <= 0 || dm->k <= 0 || dm->S < 0 || dm->I <= 0 ||
+      dm->P <= 0)
+    return false;
+  return true;
+}
+
+// Shapes the kernels support (see include/moe.h).
+int check_shape(const moe_dims* dm, bool need_bwd) {
+  if (!dims_ok(dm)) return MOE_ERR_INVALID_ARG;
+  if (dm->d % 64 || dm->I % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dm->E > 256 || dm->k > dm->E || dm->S > 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dm->P % 8 || dm->P < 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (need_bwd && dm->P % 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // rows and (t, j) indices are int32 on the device
+  if (rows_total(*dm) >= (int64_t(1) << 31) || dm->T * dm->k >= (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows_routed(*dm) < 0) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+bool ws_ok(const moe_dims* dm, const void* ws, size_t bytes) {
+  return ws != nullptr && bytes >= ws_layout(*dm).bytes;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_rows_routed(const moe_dims* dims) { return dims_ok(dims) ? rows_routed(*dims) : -1; }
+int64_t moe_rows_total(const moe_dims* dims) { return dims_ok(dims) ? rows_total(*dims) : -1; }
+
+size_t moe_workspace_size(const moe_dims* dims) {
+  return dims_ok(dims) ? ws_layout(*dims).bytes : 0;
+}
+
+int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const float* bias,
+                  int32_t* topk_idx, float* topk_w, float* probs, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (dims->E % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (dims->T > 0 && (!x || !wg || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+  return launch_gate_topk(*dims, x, wg, bias, topk_idx, topk_w, probs, stream);
+}
+
+int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void* x,
+                      int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* row_of,
+                      void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!counts || !offsets || !sorted_ids || !ws_ok(dims, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!topk_idx || !x || !row_of || !x_perm)) return MOE_ERR_INVALID_ARG;
+  return launch_permute(*dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_perm, ws,
+                        stream);
+}
+
+int grouped_gemm_set_groups(const moe_dims* dims, const int32_t* counts, int32_t* offsets,
+                            void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!counts || !offsets || !ws_ok(dims, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
+  return launch_set_groups(*dims, counts, offsets, ws, stream);
+}
+
+int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, const void* x,
+                     const void* w1, const void* w2, void* h, void* a1, void* y, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!ws || !x_perm || !w1 || !w2 || !h || !y || (dims->S > 0 && !x)) return MOE_ERR_INVALID_ARG;
+  GemmOperands o{};
+  o.a0 = x_perm;
+  o.a1 = x;
+  o.b0 = w1;
+  o.out = h;
+  o.out2 = a1;
+  rc = launch_grouped_gemm(MODE_FWD1, *dims, ws, o, stream);
+  if (rc) return rc;
+  GemmOperands o2{};
+  o2.a0 = h;
+  o2.b0 = w2;
+  o2.out = y;
+  return launch_grouped_gemm(MODE_FWD2, *dims, ws, o2, stream);
+}
+
+int grouped_gemm_bwd_dx(const moe_dims* dims, const void* ws, int which, const void* dy_routed,
+                        const void* dy_shared, const void* w, const void* a1, void* out,
+                        void* stream) {
+  int rc = check_shape(dims, true);
+  if (rc) return rc;
+  if (!ws || !dy_routed || !w || !out) return MOE_ERR_INVALID_ARG;
+  GemmOperands o{};
+  o.a0 = dy_routed;
+  o.b0 = w;
+  o.out = out;
+  if (which == MOE_GEMM2) {
+    if (!a1 || (dims->S > 0 && !dy_shared)) return MOE_ERR_INVALID_ARG;
+    o.a1 = dy_shared;
+    o.aux = a1;
+    return launch_grouped_gemm(MODE_DX2, *dims, ws, o, stream);
+  }
+  if (which == MOE_GEMM1) return launch_grouped_gemm(MODE_DX1, *dims, ws, o, stream);
+  return MOE_ERR_INVALID_ARG;
+}
+
+int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const void* lhs_routed,
+                        const void* lhs_shared, const void* rhs_routed, const void* rhs_shared,
+                        float* dw, int accumulate, void* stream) {
+  int rc = check_shape(dims, true);
+  if (rc) return rc;
+  if (!ws || !lhs_routed || !rhs_routed || !dw || (accumulate != 0 && accumulate != 1))
+    return MOE_ERR_INVALID_ARG;
+  GemmOperands o{};
+  o.a0 = lhs_routed;
+  o.b0 = rhs_routed;
+  o.out = dw;
+  o.accumulate = accumulate;
+  if (which == MOE_GEMM2) {
+    if (dims->S > 0 && !lhs_shared) return MOE_ERR_INVALID_ARG;
+    o.a1 = lhs_shared;
+    return launch_grouped_gemm(MODE_DW2, *dims, ws, o, stream);
+  }
+  if (which == MOE_GEMM1) {
+    if (dims->S > 0 && !rhs_shared) return MOE_ERR_INVALID_ARG;
+    o.b1 = rhs_shared;
+    return launch_grouped_gemm(MODE_DW1, *dims, ws, o, stream);
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,
+                void* out, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (dims->T > 0 && (!y || !row_of || !out)) return MOE_ERR_INVALID_ARG;
+  return launch_combine(*dims, y, row_of, topk_w, out, stream);
+}
+
+int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, const void* y,
+                    const int32_t* row_of, const float* topk_w, void* dy_routed, float* dw,
+                    void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!ws || !dy_routed) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!dout || !y || !row_of || !topk_w || !dw)) return MOE_ERR_INVALID_ARG;
+  return launch_combine_bwd(*dims, ws, dout, y, row_of, topk_w, dy_routed, dw, stream);
+}
+
+int moe_get_device_status(void* ws, int32_t* status_out, void* stream) {
+  if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  *status_out = v;
+  return MOE_OK;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_BAD_ROUTING: return "MOE_ERR_BAD_ROUTING";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// moe_internal.cuh -- workspace layout and records shared by the kernels of
+// libmoe.so (host and device).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// One group of the grouped GEMM: a routed expert (g < E) or a shared expert.
+//   a_row    first row of the group in its A source (x_perm for routed groups,
+//            x for shared groups, i.e. 0)
+//   out_row  first row of the group in the grouped row space [0, Rt)
+//   rows     real rows (tokens) of the group
+//   rows_pad rows rounded up to the pad block (shared groups: T)
+struct GroupRec {
+  int32_t a_row, out_row, rows, rows_pad;
+};
+
+constexpr int kChunk = 1024;      // routed assignments per histogram chunk
+constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] m-tiles total
+
+struct WsLayout {
+  size_t groups;        // GroupRec[G]
+  size_t mtile_prefix;  // int32[G + 1]  prefix of ceil(rows_pad / 128)
+  size_t dw_order;      // int32[G]      groups by padded rows, largest first
+  size_t chunk_hist;    // int32[nchunks * E]
+  size_t bytes;
+  int nchunks;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(const moe_dims& dm) {
+  WsLayout L;
+  const int G = dm.E + dm.S;
+  const int64_t assignments = dm.T * dm.k;
+  L.nchunks = (int)((assignments + kChunk - 1) / kChunk);
+  if (L.nchunks < 1) L.nchunks = 1;
+  size_t off = kHeaderWords * sizeof(int32_t);
+  L.groups = off = align_up(off, 16);
+  off += sizeof(GroupRec) * G;
+  L.mtile_prefix = off = align_up(off, 16);
+  off += sizeof(int32_t) * (G + 1);
+  L.dw_order = off = align_up(off, 16);
+  off += sizeof(int32_t) * G;
+  L.chunk_hist = off = align_up(off, 16);
+  off += sizeof(int32_t) * (size_t)L.nchunks * dm.E;
+  L.bytes = align_up(off, 256);
+  return L;
+}
+
+inline int64_t rows_routed(const moe_dims& dm) {
+  return dm.rows_cap > 0 ? dm.rows_cap : dm.T * dm.k + (int64_t)dm.E * (dm.P - 1);
+}
+inline int64_t rows_total(const moe_dims& dm) { return rows_routed(dm) + (int64_t)dm.S * dm.T; }
+
+// Launch helpers implemented in the .cu files (all return a moe_status).
+int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const float* bias,
+                     int32_t* idx, float* w, float* probs, void* stream);
+int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_t* counts,
+                   int32_t* offsets, int32_t* sorted_ids, int32_t* row_of, void* x_perm, void* ws,
+                   void* stream);
+int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offsets, void* ws,
+                      void* stream);
+int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, const float* w,
+                   void* out, void* stream);
+int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
+                       const int32_t* row_of, const float* w, void* dy, float* dw, void* stream);
+
+enum GemmMode { MODE_FWD1 = 0, MODE_FWD2, MODE_DX2, MODE_DX1, MODE_DW2, MODE_DW1 };
+
+// Operand set of one grouped GEMM call (device pointers).
+struct GemmOperands {
+  const void* a0;  // A source (routed rows / grouped row space)
+  const void* a1;  // A source for shared groups (FWD1: x, DX2 / DW2: upstream grad)
+  const void* b0;  // B source (weights, or rhs rows for DW)
+  const void* b1;  // B source for shared groups (DW1: x)
+  void* out;
+  void* out2;       // FWD1: saved pre-activations (nullable)
+  const void* aux;  // DX2: saved pre-activations
+  int accumulate;
+};
+
+int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
+                        const GemmOperands& ops, void* stream);
+
+}  // namespace moe

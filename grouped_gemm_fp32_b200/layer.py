@@ -1,0 +1,93 @@
+"""One MoE FFN layer driven through the C ABI of libmoe.so.
+
+``MoEBuffers`` owns the activations and workspace of one layer (torch device
+tensors: torch is used for memory only); ``forward`` and ``backward`` issue the
+C-ABI calls in the layer's order on one stream.  Every arithmetic step runs in
+libmoe.so.
+
+Layer (dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
+and "Load balancing"; §3.2 "Efficient implementation of Grouped GEMM"):
+    forward   moe_gate_topk -> moe_permute_align -> grouped_gemm_fwd -> moe_combine
+    backward  moe_combine_bwd -> grouped_gemm_bwd_dx(GEMM2) -> grouped_gemm_bwd_dw(GEMM2)
+              -> grouped_gemm_bwd_dx(GEMM1) -> grouped_gemm_bwd_dw(GEMM1)
+              -> moe_combine(weights = NULL)  (un-permute-sum of the dX rows)
+The backward returns the gradient through the experts and the combine weights;
+the router's own gradient is not part of this path.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+class MoEBuffers:
+    def __init__(self, dims: L.MoeDims, device="cuda", train: bool = False):
+        self.dims = dims
+        self.train = train
+        T, d, E, k, S, I = dims.T, dims.d, dims.E, dims.k, dims.S, dims.I
+        G = E + S
+        self.Rr = L.moe_rows_routed(dims)
+        self.Rt = L.moe_rows_total(dims)
+        if self.Rr < 0:
+            raise ValueError(f"invalid dims {dims}")
+        dev = torch.device(device)
+        i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+        e = lambda *s, dt=bf: torch.empty(*s, dtype=dt, device=dev)
+        self.ws = torch.zeros(L.moe_workspace_size(dims), dtype=torch.uint8, device=dev)
+        self.topk_idx = e(T, k, dt=i32)
+        self.topk_w = e(T, k, dt=f32)
+        self.counts = e(E, dt=i32)
+        self.offsets = e(E + 1, dt=i32)
+        self.sorted_ids = e(self.Rr, dt=i32)
+        self.row_of = e(T, k, dt=i32)
+        self.x_perm = e(self.Rr, d)
+        self.h = e(self.Rt, I)
+        self.a1 = e(self.Rt, 2 * I) if train else None
+        self.y = e(self.Rt, d)
+        self.out = e(T, d)
+        if train:
+            self.dy = e(self.Rr, d)
+            self.dw_comb = e(T, k, dt=f32)
+            self.da = e(self.Rt, 2 * I)
+            self.dxp = e(self.Rt, d)
+            self.dx = e(T, d)
+            self.dw1 = e(G, 2 * I, d, dt=f32)
+            self.dw2 = e(G, d, I, dt=f32)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in vars(self).values()
+                   if isinstance(t, torch.Tensor))
+
+
+def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
+    """out = MoE(x).  x [T, d] bf16, wg [E, d] f32, bias [E] f32, w1 [G, 2I, d], w2 [G, d, I].
+
+    ``routing=(topk_idx, topk_w)`` (device int32 / f32 [T, k]) replaces the gate's
+    choice, e.g. to run the experts on a routing decided elsewhere."""
+    dm = b.dims
+    if routing is None:
+        L.moe_gate_topk(dm, x, wg, bias, b.topk_idx, b.topk_w, None, stream)
+    else:
+        b.topk_idx.copy_(routing[0])
+        b.topk_w.copy_(routing[1])
+    L.moe_permute_align(dm, b.topk_idx, x, b.counts, b.offsets, b.sorted_ids, b.row_of, b.x_perm,
+                        b.ws, stream)
+    L.grouped_gemm_fwd(dm, b.ws, b.x_perm, x, w1, w2, b.h, b.a1, b.y, stream)
+    L.moe_combine(dm, b.y, b.row_of, b.topk_w, b.out, stream)
+    return b.out
+
+
+def backward(b: MoEBuffers, x, dout, w1, w2, stream=None):
+    """Gradients after ``forward``: dx [T, d] (through the experts), dw1, dw2 (f32) and the
+    combine-weight gradient dw_comb [T, k]."""
+    if not b.train:
+        raise ValueError("buffers were allocated without train=True")
+    dm = b.dims
+    L.moe_combine_bwd(dm, b.ws, dout, b.y, b.row_of, b.topk_w, b.dy, b.dw_comb, stream)
+    L.grouped_gemm_bwd_dx(dm, b.ws, L.MOE_GEMM2, b.dy, dout, w2, b.a1, b.da, stream)
+    L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM2, b.dy, dout, b.h, None, b.dw2, 0, stream)
+    L.grouped_gemm_bwd_dx(dm, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, stream)
+    L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x, b.dw1, 0, stream)
+    L.moe_combine(dm, b.dxp, b.row_of, None, b.dx, stream)
+    return b.dx, b.dw1, b.dw2, b.dw_comb

@@ -1,0 +1,204 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE FFN layer library (libmoe.so).
+ *
+ * The layer is the fine-grained MoE FFN of dots.llm1 (dots.llm1 Technical
+ * Report, §Architecture "Mixture of Experts layer" and "Load balancing";
+ * §3.2 "Efficient implementation of Grouped GEMM"):
+ *
+ *   1. FP32 gate:        logit = X Wg^T in FP32                (moe_gate_topk)
+ *   2. aux-loss-free top-k: p = softmax(logit), s = p + bias, top-k of s,
+ *                        w = p renormalised over the chosen k  (moe_gate_topk)
+ *   3. permute into per-expert segments padded to P rows       (moe_permute_align)
+ *   4. grouped SwiGLU expert GEMMs, routed + shared experts    (grouped_gemm_fwd)
+ *   5. weighted combine                                        (moe_combine)
+ *   backward: combine bwd, dX and dW grouped GEMMs             (moe_combine_bwd,
+ *             grouped_gemm_bwd_dx, grouped_gemm_bwd_dw, moe_combine)
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates or frees device memory.  Row-major, densely packed.
+ *   - bf16 tensors are passed as `void*` holding IEEE bfloat16 values.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise the host, except moe_get_device_status.
+ *   - Argument and shape errors return a negative moe_status before anything is
+ *     launched.  Errors found on the device (a bounded wait that ran out, an
+ *     inconsistent group table) are written to a status word inside the
+ *     workspace and read with moe_get_device_status.
+ *
+ * Shapes (struct moe_dims): T tokens, d hidden, E routed experts, k experts per
+ * token, S shared experts, I expert intermediate size, P pad block.
+ *   G  = E + S groups; group e < E is routed expert e, group E + s is shared s.
+ *   Rr = routed row capacity = dims.rows_cap, or T*k + E*(P-1) when 0.
+ *   Rt = Rr + S*T rows of the "grouped row space": routed expert e owns rows
+ *        [off_e, off_e + roundup(c_e, P)); shared expert s owns rows
+ *        [Rr + s*T, Rr + (s+1)*T) (one row per token, in token order).
+ * Weights: W1 [G, 2I, d] bf16 (rows 0..I-1 gate projection, I..2I-1 up
+ * projection), W2 [G, d, I] bf16, Wg [E, d] f32, bias [E] f32.
+ * Supported: d % 64 == 0, I % 64 == 0, 1 <= k <= E <= 256, S <= 2, P % 8 == 0,
+ * P >= 8, Rt * max(d, 2I) < 2^31; the backward needs P % 64 == 0.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,       /* null pointer, bad enum value, ws too small */
+  MOE_ERR_UNSUPPORTED_SHAPE = -2, /* shape outside the supported set above */
+  MOE_ERR_CUDA = -3,              /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = -4,    /* (device) a bounded wait in a kernel ran out */
+  MOE_ERR_BAD_ROUTING = -5        /* (device) padded rows exceed Rr, or bad expert id */
+} moe_status;
+
+typedef struct moe_dims {
+  int64_t T;        /* tokens */
+  int32_t d;        /* hidden size */
+  int32_t E;        /* routed experts */
+  int32_t k;        /* routed experts per token */
+  int32_t S;        /* shared experts */
+  int32_t I;        /* expert intermediate size */
+  int32_t P;        /* pad block of a routed segment (rows) */
+  int64_t rows_cap; /* Rr, rows of the routed row space; 0 => T*k + E*(P-1) */
+} moe_dims;
+
+/* Which GEMM of the expert FFN a backward call works on. */
+enum { MOE_GEMM1 = 1, /* gate|up projection  A1 = A W1^T  (N = 2I, K = d) */
+       MOE_GEMM2 = 2  /* down projection     Y  = H W2^T  (N = d,  K = I) */ };
+
+/* Rr and Rt as defined above (-1 for invalid dims). */
+int64_t moe_rows_routed(const moe_dims* dims);
+int64_t moe_rows_total(const moe_dims* dims);
+
+/* Bytes of device workspace that the calls taking `ws` need.  One workspace
+ * serves a whole layer: moe_permute_align (or grouped_gemm_set_groups) writes
+ * the group table into it, and the GEMM and combine-backward calls read it. */
+size_t moe_workspace_size(const moe_dims* dims);
+
+/* Gate and aux-loss-free top-k routing.
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts
+ * layer" (the gating layer runs in FP32, top-6 of 128 routed experts) and
+ * "Load balancing" (a per-expert bias is added to the affinity scores only to
+ * decide the top-k routing).
+ *   x     [T, d]  bf16          hidden states
+ *   wg    [E, d]  f32           gate weights
+ *   bias  [E]     f32           selection bias (may be NULL: zero)
+ * Out:
+ *   topk_idx [T, k] int32       chosen experts, biased score descending, equal
+ *                               scores to the lower expert index
+ *   topk_w   [T, k] f32         p[e_j] / sum_j p[e_j] (unbiased, renormalised)
+ *   probs    [T, E] f32         softmax affinities (may be NULL)
+ * logits are accumulated in FP32; p uses expf. */
+int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const float* bias,
+                  int32_t* topk_idx, float* topk_w, float* probs, void* stream);
+
+/* Permutation into per-expert segments padded to P rows, plus the group table.
+ * Passage: dots.llm1 Technical Report, §3.2 "Efficient implementation of
+ * Grouped GEMM" (each expert's token segment M_i is aligned to a fixed block,
+ * so one tile belongs to one expert) and §Architecture "Load balancing" (no
+ * token is dropped: segments grow with the load, there is no capacity).
+ *   topk_idx [T, k] int32 (from moe_gate_topk or the caller), x [T, d] bf16
+ * Out:
+ *   counts     [E]      int32   c_e, tokens routed to expert e
+ *   offsets    [E + 1]  int32   off_0 = 0, off_{e+1} = off_e + roundup(c_e, P)
+ *   sorted_ids [Rr]     int32   token of each routed row (ascending inside a
+ *                               segment), -1 on pad rows and rows >= off_E
+ *   row_of     [T, k]   int32   routed row of (t, j)
+ *   x_perm     [Rr, d]  bf16    x_perm[row_of[t, j]] = x[t]; pad rows zero;
+ *                               rows >= off_E are not written
+ *   ws / ws_bytes               workspace (group table written here)
+ * Deterministic: the same input gives the same output bit for bit.  An expert
+ * id outside [0, E) or off_E > Rr sets MOE_ERR_BAD_ROUTING in the device
+ * status and leaves an empty group table. */
+int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void* x,
+                      int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* row_of,
+                      void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Group table from given per-expert row counts, for callers that already hold
+ * the permuted rows (the grouped GEMM used on its own).  counts [E] int32
+ * (device); writes offsets [E + 1] (device) and the group table in ws, with
+ * segments padded to P as in moe_permute_align. */
+int grouped_gemm_set_groups(const moe_dims* dims, const int32_t* counts, int32_t* offsets,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Forward grouped GEMMs of the expert FFNs (routed + shared), SwiGLU fused.
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
+ * (fine-grained two-layer SwiGLU experts; 2 shared experts see every token)
+ * and §3.2 (one tile = one expert's aligned segment).
+ *   ws       workspace holding the group table
+ *   x_perm   [Rr, d] bf16  A rows of the routed groups
+ *   x        [T, d]  bf16  A rows of the shared groups (may be NULL when S = 0)
+ *   w1 [G, 2I, d] bf16, w2 [G, d, I] bf16
+ * Out (grouped row space, rows of each group up to its padded size):
+ *   h  [Rt, I]  bf16  H = silu(A W1g^T) * (A W1u^T), from the FP32 accumulator
+ *   a1 [Rt, 2I] bf16  [A W1g^T | A W1u^T], saved for the backward (may be NULL)
+ *   y  [Rt, d]  bf16  Y = H W2^T
+ * bf16 operands, FP32 accumulation in tensor memory (tcgen05). */
+int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, const void* x,
+                     const void* w1, const void* w2, void* h, void* a1, void* y, void* stream);
+
+/* Backward data-gradient grouped GEMMs.
+ *   which = MOE_GEMM2: dH = dY W2, then the SwiGLU backward with the saved a1:
+ *       dG = dH * U * s * (1 + G (1 - s)), s = sigmoid(G);  dU = dH * silu(G)
+ *     dy_routed [Rr, d] bf16 (from moe_combine_bwd), dy_shared [T, d] bf16 (the
+ *     upstream gradient itself; may be NULL when S = 0), w = w2, a1 [Rt, 2I]
+ *     -> out = dA [Rt, 2I] bf16 ([dG | dU])
+ *   which = MOE_GEMM1: dX_perm = dA W1
+ *     dy_routed = dA [Rt, 2I] bf16, dy_shared ignored, w = w1, a1 ignored
+ *     -> out = dX rows [Rt, d] bf16 (reduce with moe_combine, topk_w = NULL) */
+int grouped_gemm_bwd_dx(const moe_dims* dims, const void* ws, int which, const void* dy_routed,
+                        const void* dy_shared, const void* w, const void* a1, void* out,
+                        void* stream);
+
+/* Backward weight-gradient grouped GEMMs; the reduction runs over each group's
+ * (padded) rows.
+ *   which = MOE_GEMM2: dW2_g = dY_g^T H_g
+ *     lhs_routed = dY [Rr, d], lhs_shared = upstream gradient [T, d],
+ *     rhs_routed = H [Rt, I], rhs_shared ignored  -> dw = dW2 [G, d, I] f32
+ *   which = MOE_GEMM1: dW1_g = dA_g^T A_g
+ *     lhs_routed = dA [Rt, 2I], lhs_shared ignored,
+ *     rhs_routed = x_perm [Rr, d], rhs_shared = x [T, d] -> dw = dW1 [G, 2I, d] f32
+ * accumulate = 0 overwrites dw (an expert with no rows gets zeros);
+ * accumulate = 1 adds to it. */
+int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const void* lhs_routed,
+                        const void* lhs_shared, const void* rhs_routed, const void* rhs_shared,
+                        float* dw, int accumulate, void* stream);
+
+/* Weighted combine (un-permute).
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
+ * (each token's output sums its 6 routed experts and the 2 shared experts).
+ *   y [Rt, d] bf16 (grouped row space), row_of [T, k], topk_w [T, k] f32
+ *   out[t] = sum_j topk_w[t, j] * y[row_of[t, j]] + sum_s y[Rr + s*T + t]
+ * accumulated in FP32, stored bf16 into out [T, d].  topk_w = NULL uses weight 1
+ * for every routed row: the un-permute-sum that turns dX rows into dX. */
+int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,
+                void* out, void* stream);
+
+/* Backward of the weighted combine.
+ *   dout [T, d] bf16, y [Rt, d] bf16 (forward output rows), row_of, topk_w
+ * Out:
+ *   dy_routed [Rr, d] bf16   dy[row_of[t, j]] = topk_w[t, j] * dout[t];
+ *                            pad rows of every segment set to zero
+ *   dw        [T, k]  f32    dw[t, j] = sum_c dout[t, c] * y[row_of[t, j], c]
+ * The shared experts' dY is dout itself (no copy). */
+int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, const void* y,
+                    const int32_t* row_of, const float* topk_w, void* dy_routed, float* dw,
+                    void* stream);
+
+/* Reads and clears the device status word of `ws` (synchronises `stream`).
+ * *status_out receives MOE_OK or the first device error recorded. */
+int moe_get_device_status(void* ws, int32_t* status_out, void* stream);
+
+/* Human-readable name of a moe_status value. */
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

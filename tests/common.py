@@ -1,0 +1,104 @@
+"""Helpers shared by the tests: workload inputs, device upload, tolerances."""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+# Floating-point bar for bf16-in / FP32-accumulate outputs and gradients:
+# max|got - ref| <= REL_TOL * max|ref| per output tensor.
+REL_TOL = 2e-2
+# Routing indices must match except for tokens whose oracle margin between the
+# k-th and (k+1)-th biased score is below this.
+MARGIN_EXEMPT = 1e-5
+# Combine weights: absolute tolerance (FP32 softmax against the FP64 oracle).
+W_TOL = 1e-5
+
+
+def fitted_bias(name: str) -> np.ndarray:
+    vals = []
+    with open(os.path.join(GOLDEN, f"{name}_bias.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                vals.append(float(line))
+    return np.array(vals, dtype=np.float32)
+
+
+def workload_inputs(name: str, with_weights: bool = True) -> dict:
+    wl = synth.WORKLOADS[name]
+    bias = fitted_bias(name) if name in ("skewed", "train") else None
+    return synth.make_inputs(wl, with_weights=with_weights, bias_override=bias)
+
+
+def dims_of(wl_or_dims):
+    from grouped_gemm_fp32_b200 import MoeDims
+    dm = wl_or_dims.dims if hasattr(wl_or_dims, "dims") else wl_or_dims
+    return MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
+
+
+def dev(a, bf16: bool = False):
+    """numpy -> CUDA tensor (uint16 bit patterns become torch.bfloat16)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if bf16:
+        t = t.view(torch.bfloat16)
+    return t.cuda()
+
+
+def host(t) -> np.ndarray:
+    """CUDA tensor -> numpy (bf16 widened to float64)."""
+    import torch
+    if t.dtype == torch.bfloat16:
+        return t.float().cpu().numpy().astype(np.float64)
+    return t.cpu().numpy()
+
+
+def rel_err(got, ref) -> float:
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    scale = np.max(np.abs(ref))
+    return float(np.max(np.abs(got - ref)) / (scale if scale > 0 else 1.0))
+
+
+def assert_close(got, ref, what: str, tol: float = REL_TOL):
+    e = rel_err(got, ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    assert e <= tol, f"{what}: max|diff|/max|ref| = {e:.3e} > {tol}"
+    return e
+
+
+_ROUTING_CACHE: dict = {}
+
+
+def oracle_routing(name: str):
+    """Oracle router on a workload's own inputs (cached per process):
+    (probs, idx, w, margin) with idx/w in the oracle's order."""
+    if name not in _ROUTING_CACHE:
+        import oracle
+        inp = workload_inputs(name, with_weights=False)
+        k = synth.WORKLOADS[name].dims.k
+        _ROUTING_CACHE[name] = oracle.route(oracle.gate_logits(inp["x"], inp["wg"]), inp["bias"], k)
+    return _ROUTING_CACHE[name]
+
+
+def check_routing(gidx, gw, probs, oidx, ow, margin, bias):
+    """GPU routing vs the oracle: identical wherever the oracle margin is >= 1e-5;
+    elsewhere the GPU's picks must still be within 1e-5 of the oracle's k-th score.
+    Returns the mask of tokens routed identically."""
+    same = np.all(gidx == oidx, axis=1)
+    exempt = margin < MARGIN_EXEMPT
+    bad = ~same & ~exempt
+    assert not bad.any(), f"{bad.sum()} tokens routed differently with margin >= {MARGIN_EXEMPT}"
+    s = probs + bias[None, :].astype(np.float64)
+    k = oidx.shape[1]
+    for t in np.nonzero(~same)[0]:
+        kth = s[t, oidx[t, k - 1]]
+        assert len(set(gidx[t])) == k
+        assert np.all(s[t, gidx[t]] >= kth - MARGIN_EXEMPT), t
+    if same.any():
+        assert np.max(np.abs(gw[same] - ow[same])) <= W_TOL
+    return same

@@ -1,0 +1,106 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every entry point
+that include/moe.h declares (CPU only: no kernel is launched here).  The
+host-side parts that need no GPU (row counts, workspace size, argument and
+shape validation, status strings) are exercised too."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from grouped_gemm_fp32_b200 import build
+    build.build()
+    import grouped_gemm_fp32_b200 as moe
+    return moe
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\**([a-z_][a-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_layer_calls():
+    names = declared_functions()
+    for n in ("moe_gate_topk", "moe_permute_align", "grouped_gemm_fwd", "grouped_gemm_bwd_dx",
+              "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.lib_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    from grouped_gemm_fp32_b200._lib import EXPORTS
+    assert set(EXPORTS) == set(declared_functions())
+
+
+def test_library_is_sm100a_only(lib):
+    # the fat binary holds sm_100a code (cuobjdump is not used: list the ELF sections' arch tags
+    # through the build flags instead)
+    from grouped_gemm_fp32_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+
+
+def test_row_counts_and_workspace(lib):
+    d = lib.MoeDims.of(8192, 4096, 128, 6, 2, 1408, 128)
+    assert lib.moe_rows_routed(d) == 8192 * 6 + 128 * 127
+    assert lib.moe_rows_total(d) == 8192 * 6 + 128 * 127 + 2 * 8192
+    assert lib.moe_workspace_size(d) >= 16 * 4 + 130 * 16
+    d2 = lib.MoeDims.of(8192, 4096, 16, 1, 0, 1408, 128, 8192)
+    assert lib.moe_rows_routed(d2) == 8192 and lib.moe_rows_total(d2) == 8192
+    bad = lib.MoeDims.of(-1, 4096, 16, 1, 0, 1408, 128)
+    assert lib.moe_rows_routed(bad) == -1 and lib.moe_workspace_size(bad) == 0
+
+
+def _call(lib, name, *args):
+    return getattr(lib.load(), name)(*args)
+
+
+def test_validation_rejects_before_any_launch(lib):
+    L = lib.load()
+    ok = lib.MoeDims.of(64, 128, 8, 2, 1, 64, 16)
+    nul = None
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    # unsupported shapes
+    for bad in (lib.MoeDims.of(64, 100, 8, 2, 1, 64, 16),    # d % 64
+                lib.MoeDims.of(64, 128, 8, 2, 1, 96, 16),    # I % 64
+                lib.MoeDims.of(64, 128, 300, 2, 1, 64, 16),  # E > 256
+                lib.MoeDims.of(64, 128, 8, 9, 1, 64, 16),    # k > E
+                lib.MoeDims.of(64, 128, 8, 2, 1, 64, 12)):   # P % 8
+        assert L.moe_combine(ctypes.byref(bad), p, p, p, p, nul) == -2
+    # backward needs P % 64 == 0
+    assert L.grouped_gemm_bwd_dx(ctypes.byref(ok), p, 1, p, p, p, p, p, nul) == -2
+    # null pointers / bad enum / small workspace
+    assert L.moe_gate_topk(ctypes.byref(ok), nul, p, p, p, p, nul, nul) == -1
+    assert L.moe_permute_align(ctypes.byref(ok), p, p, p, p, p, p, p, p, 8, nul) == -1
+    ok64 = lib.MoeDims.of(64, 128, 8, 2, 1, 64, 64)
+    assert L.grouped_gemm_bwd_dx(ctypes.byref(ok64), p, 7, p, p, p, p, p, nul) == -1
+    assert L.grouped_gemm_bwd_dw(ctypes.byref(ok64), p, 2, p, p, p, p, p, 5, nul) == -1
+    assert L.moe_gate_topk(None, p, p, p, p, p, nul, nul) == -1
+
+
+def test_status_strings(lib):
+    assert lib.moe_status_string(0) == "MOE_OK"
+    assert lib.moe_status_string(-4) == "MOE_ERR_DEVICE_TIMEOUT"
+    assert lib.moe_status_string(-5) == "MOE_ERR_BAD_ROUTING"
+    assert lib.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import grouped_gemm_fp32_b200._lib as L
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "_LIB_PATH", str(tmp_path / "libmoe.so"))
+    with pytest.raises(ImportError):
+        L.load()
