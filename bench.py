@@ -9,6 +9,8 @@ One step = one pass of the whole hot path over one batch:
                    SwiGLU GEMMs, combine) + backward (combine bwd, dX and dW
                    grouped GEMMs, SwiGLU bwd, un-permute-sum).
   layer:           T=8192, same layer, forward only.
+  gemm_only:       the grouped GEMM forward alone (16 groups x 512 rows, d=4096,
+                   I=1408): a small case for profiles, not the headline.
 Inputs are synthetic (seeded generator), resident in HBM for ``value``; the
 weights alone (4.5 GB) exceed L2, so no flush is needed between steps.
 
@@ -42,7 +44,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="train", choices=["train", "layer"])
+    ap.add_argument("--workload", default="train", choices=["train", "layer", "gemm_only"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -242,19 +244,32 @@ def run_ours(args):
 
     wl, inp = workload(args.workload)
     dm = wl.dims
-    dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P)
+    dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
     train = wl.backward
+    gemm_only = wl.group_rows is not None
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
     x, w1, w2 = bf(inp["x"]), bf(inp["w1"]), bf(inp["w2"])
-    wg = torch.from_numpy(inp["wg"]).to(dev)
-    bias = torch.from_numpy(inp["bias"]).to(dev)
+    wg = torch.from_numpy(inp["wg"]).to(dev) if not gemm_only else None
+    bias = torch.from_numpy(inp["bias"]).to(dev) if not gemm_only else None
     dout = bf(inp["dout"]) if train else None
     b = layer.MoEBuffers(dims, device=dev, train=train)
+    if gemm_only:
+        counts = torch.tensor(wl.group_rows, dtype=torch.int32, device=dev)
+        moe.grouped_gemm_set_groups(dims, counts, b.offsets, b.ws)
     torch.cuda.synchronize()
 
     def step(s, xx=x, gg=dout, ev=None):
+        if gemm_only:
+            if ev is not None:
+                ev["t0"].append(torch.cuda.Event(enable_timing=True))
+                ev["t0"][-1].record(s)
+            moe.grouped_gemm_fwd(dims, b.ws, xx, None, w1, w2, b.h, None, b.y, s)
+            if ev is not None:
+                ev["fwd"].append(torch.cuda.Event(enable_timing=True))
+                ev["fwd"][-1].record(s)
+            return
         if ev is None:
             layer.forward(b, xx, wg, bias, w1, w2, stream=s)
             if train:
@@ -316,7 +331,7 @@ def run_ours(args):
     tokens_per_s = world * dm.T / (ms / 1000.0)
 
     # ---- per-call breakdown (separate instrumented pass; not the headline)
-    names = ["t0", "gate", "permute", "fwd", "combine"] + (
+    names = (["t0", "fwd"] if gemm_only else ["t0", "gate", "permute", "fwd", "combine"]) + (
         ["combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute"] if train else [])
     ev = {n: [] for n in names}
     nprof = max(3, min(args.steps, 20))
@@ -339,6 +354,7 @@ def run_ours(args):
     # ---- e2e: pinned host inputs in, results out, through the same C ABI calls
     hx = torch.from_numpy(inp["x"]).view(torch.bfloat16).pin_memory()
     hd = torch.from_numpy(inp["dout"]).view(torch.bfloat16).pin_memory() if train else None
+    out_dev = b.y[: dm.T] if gemm_only else b.out
     ho = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory()
     hdx = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() if train else None
     dx_in = torch.empty_like(x)
@@ -351,7 +367,7 @@ def run_ours(args):
         if train:
             dd_in.copy_(hd, non_blocking=True)
         step(stream, xx=dx_in, gg=dd_in)
-        ho.copy_(b.out, non_blocking=True)
+        ho.copy_(out_dev, non_blocking=True)
         if train:
             hdx.copy_(b.dx, non_blocking=True)
 
@@ -373,7 +389,7 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after timing: {moe.moe_status_string(status)}")
 
-    launches_per_step = 1 + 5 + 2 + 1 + ((2 + 4 + 1) if train else 0)
+    launches_per_step = 2 if gemm_only else 1 + 5 + 2 + 1 + ((2 + 4 + 1) if train else 0)
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -396,7 +412,7 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not gemm_only:
         line["cpu_baseline"] = cpu_baseline(wl, inp)
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -86,19 +86,35 @@ def oracle_routing(name: str):
 
 
 def check_routing(gidx, gw, probs, oidx, ow, margin, bias):
-    """GPU routing vs the oracle: identical wherever the oracle margin is >= 1e-5;
-    elsewhere the GPU's picks must still be within 1e-5 of the oracle's k-th score.
-    Returns the mask of tokens routed identically."""
-    same = np.all(gidx == oidx, axis=1)
+    """GPU routing vs the oracle.
+
+    * The chosen SET is identical wherever the oracle margin (k-th minus
+      (k+1)-th biased score) is >= 1e-5; elsewhere every GPU pick must score
+      within 1e-5 of the oracle's k-th.
+    * The ORDER (biased score descending) is identical except between chosen
+      experts whose oracle scores differ by less than 1e-5: the GPU's order must
+      be non-increasing in the oracle's scores up to 1e-5.
+    * Weights match per expert within W_TOL.
+    Returns (same_set mask [T], align [T, k]) with gidx[t, align[t, j]] == oidx[t, j]
+    for tokens of the same set."""
+    T, k = oidx.shape
+    s = probs + bias[None, :].astype(np.float64)
+    same = np.sort(gidx, axis=1) == np.sort(oidx, axis=1)
+    same = np.all(same, axis=1)
     exempt = margin < MARGIN_EXEMPT
     bad = ~same & ~exempt
-    assert not bad.any(), f"{bad.sum()} tokens routed differently with margin >= {MARGIN_EXEMPT}"
-    s = probs + bias[None, :].astype(np.float64)
-    k = oidx.shape[1]
+    assert not bad.any(), f"{bad.sum()} tokens chose a different expert set with margin >= {MARGIN_EXEMPT}"
     for t in np.nonzero(~same)[0]:
         kth = s[t, oidx[t, k - 1]]
         assert len(set(gidx[t])) == k
         assert np.all(s[t, gidx[t]] >= kth - MARGIN_EXEMPT), t
+    gs = np.take_along_axis(s, gidx.astype(np.int64), axis=1)
+    assert np.all(gs[:, :-1] >= gs[:, 1:] - MARGIN_EXEMPT), "GPU order is not by biased score"
+    align = np.zeros((T, k), dtype=np.int64)
+    for t in np.nonzero(same)[0]:
+        pos = {int(e): j for j, e in enumerate(gidx[t])}
+        align[t] = [pos[int(e)] for e in oidx[t]]
     if same.any():
-        assert np.max(np.abs(gw[same] - ow[same])) <= W_TOL
-    return same
+        gw_al = np.take_along_axis(gw, align, axis=1)
+        assert np.max(np.abs(gw_al[same] - ow[same])) <= W_TOL
+    return same, align

@@ -93,7 +93,8 @@ def test_layer_forward_matches_oracle(name, nsample):
     wl = synth.WORKLOADS[name]
     S = wl.dims.S
     p, oidx, ow, margin = oracle_routing(name)
-    same = check_routing(host(b.topk_idx), host(b.topk_w), p, oidx, ow, margin, inp["bias"])
+    same, align = check_routing(host(b.topk_idx), host(b.topk_w), p, oidx, ow, margin,
+                                inp["bias"])
     T = wl.dims.T
     if nsample is None:
         tokens = np.nonzero(same)[0]
@@ -110,7 +111,7 @@ def test_layer_forward_matches_oracle(name, nsample):
     assert_close(host(out)[tokens], ref, f"{name} out")
     # the expert output rows behind the combine
     Y = host(b.y)
-    rof = host(b.row_of)
+    rof = np.take_along_axis(host(b.row_of), align, axis=1)  # in the oracle's pick order
     assert_close(Y[rof[tokens]], yr, f"{name} routed Y rows")
     for s in range(S):
         assert_close(Y[b.Rr + s * T + tokens], ys[:, s], f"{name} shared Y rows {s}")

@@ -34,10 +34,12 @@ def test_gate_topk_matches_oracle(name):
     dm = dims_of(wl)
     idx, w, probs = _gate(dm, dev(inp["x"], True), dev(inp["wg"]), dev(inp["bias"]))
     p, oidx, ow, margin = oracle_routing(name)
-    same = check_routing(host(idx), host(w), p, oidx, ow, margin, inp["bias"])
+    same, align = check_routing(host(idx), host(w), p, oidx, ow, margin, inp["bias"])
     assert np.max(np.abs(host(probs) - p)) <= W_TOL
     np.testing.assert_allclose(host(w).sum(axis=1), 1.0, atol=1e-5)
-    print(f"{name}: {int((~same).sum())} of {dm.T} tokens exempt (margin < {MARGIN_EXEMPT})")
+    order_diff = int((np.any(align != np.arange(dm.k), axis=1) & same).sum())
+    print(f"{name}: {int((~same).sum())} of {dm.T} tokens chose another near-tied set "
+          f"(margin < {MARGIN_EXEMPT}); {order_diff} ordered two near-tied picks differently")
 
 
 def test_gate_ties_go_to_lower_index():
