@@ -88,7 +88,7 @@ __global__ void groups_kernel(int32_t* __restrict__ hist, int nchunks, int E, in
     if (bad) atomicCAS(ws_header, 0, MOE_ERR_BAD_ROUTING);
   }
   __syncthreads();
-  if (tid <= E) offsets[tid] = s_scan[tid];
+  for (int e = tid; e <= E; e += blockDim.x) offsets[e] = s_scan[e];
   for (int g = tid; g < G; g += blockDim.x) {
     GroupRec r;
     if (g < E) {
