@@ -16,8 +16,8 @@ _lib = None
 MOE_GEMM1, MOE_GEMM2 = 1, 2
 EXPORTS = (
     "moe_rows_routed", "moe_rows_total", "moe_workspace_size", "moe_gate_topk",
-    "moe_permute_align", "grouped_gemm_set_groups", "grouped_gemm_fwd", "grouped_gemm_bwd_dx",
-    "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd", "moe_get_device_status",
+    "moe_permute_align", "moe_permute_align_static", "grouped_gemm_set_groups",
+    "grouped_gemm_fwd", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd", "moe_get_device_status",
     "moe_status_string",
 )
 
@@ -63,6 +63,7 @@ def load():
         "moe_workspace_size": (sz, [D]),
         "moe_gate_topk": (i32, [D, vp, vp, vp, vp, vp, vp, vp]),
         "moe_permute_align": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "moe_permute_align_static": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "grouped_gemm_set_groups": (i32, [D, vp, vp, vp, sz, vp]),
         "grouped_gemm_fwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "grouped_gemm_bwd_dx": (i32, [D, vp, i32, vp, vp, vp, vp, vp, vp]),
@@ -129,6 +130,14 @@ def moe_permute_align(dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_
     _ck(load().moe_permute_align(ctypes.byref(dims), _p(topk_idx), _p(x), _p(counts),
                                  _p(offsets), _p(sorted_ids), _p(row_of), _p(x_perm), _p(ws),
                                  nbytes, _s(stream)), "moe_permute_align")
+
+
+def moe_permute_align_static(dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_perm,
+                             stream=None):
+    """moe_permute_align for callers that cannot allocate: no workspace argument."""
+    _ck(load().moe_permute_align_static(ctypes.byref(dims), _p(topk_idx), _p(x), _p(counts),
+                                        _p(offsets), _p(sorted_ids), _p(row_of), _p(x_perm),
+                                        _s(stream)), "moe_permute_align_static")
 
 
 def grouped_gemm_set_groups(dims, counts, offsets, ws, stream=None):

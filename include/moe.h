@@ -34,8 +34,9 @@
  *        [Rr + s*T, Rr + (s+1)*T) (one row per token, in token order).
  * Weights: W1 [G, 2I, d] bf16 (rows 0..I-1 gate projection, I..2I-1 up
  * projection), W2 [G, d, I] bf16, Wg [E, d] f32, bias [E] f32.
- * Supported: d % 64 == 0, I % 64 == 0, 1 <= k <= E <= 256, S <= 2, P % 8 == 0,
- * P >= 8, Rt * max(d, 2I) < 2^31; the backward needs P % 64 == 0.
+ * Supported: d % 64 == 0, I % 64 == 0, 1 <= k <= E <= 256 (E % 8 == 0 for the
+ * gate), S <= 8, P % 8 == 0, P >= 8, Rt < 2^31, T*k < 2^31; the backward needs
+ * P % 64 == 0.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -118,6 +119,30 @@ int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const fl
 int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void* x,
                       int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* row_of,
                       void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_permute_align without a workspace argument: the same outputs, with the
+ * scratch (status header, group table, chunk histograms) held in a fixed
+ * 1 MiB device array inside the library.  (The pages have no counterpart: this
+ * is an allocation-free form of the call above.)  It serves callers that cannot
+ * allocate device memory or keep a workspace alive between calls -- code inside
+ * a host framework whose allocator owns every device buffer, foreign-function
+ * callers that pass only inputs and outputs, paths where cudaMalloc is not
+ * allowed.  It calls no cudaMalloc or cudaFree.
+ *   - Limit: the call's scratch, moe_workspace_size(dims), must be at most
+ *     1 MiB (about 2 million routed assignments at E = 128); larger shapes
+ *     return MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - The array is shared by every call in the process and keeps the last
+ *     call's contents; each call clears what must start at zero.  Calls whose
+ *     executions overlap on the GPU (other streams, other threads) race on it
+ *     and must be serialised by the caller.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Routing errors (expert id outside [0, E), padded rows above Rr) leave
+ *     sorted_ids at -1 and x_perm unwritten; no device status is kept. */
+int moe_permute_align_static(const moe_dims* dims, const int32_t* topk_idx, const void* x,
+                             int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
+                             int32_t* row_of, void* x_perm, void* stream);
 
 /* Group table from given per-expert row counts, for callers that already hold
  * the permuted rows (the grouped GEMM used on its own).  counts [E] int32
