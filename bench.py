@@ -11,6 +11,8 @@ One step = one pass of the whole hot path over one batch:
   layer:           T=8192, same layer, forward only.
   gemm_only:       the grouped GEMM forward alone (16 groups x 512 rows, d=4096,
                    I=1408): a small case for profiles, not the headline.
+  train_small:     train with E=16, T=2048 (same rows per expert): profiles.
+  gate_only:       the gate + top-k alone on the layer shapes: profiles.
 Inputs are synthetic (seeded generator), resident in HBM for ``value``; the
 weights alone (4.5 GB) exceed L2, so no flush is needed between steps.
 
@@ -44,7 +46,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="train", choices=["train", "layer", "gemm_only"])
+    ap.add_argument("--workload", default="train",
+                    choices=["train", "layer", "gemm_only", "train_small", "gate_only"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -69,6 +72,9 @@ def fitted_bias(name):
 
 def workload(name):
     import synth
+    if name == "gate_only":
+        wl = synth.WORKLOADS["layer"]
+        return wl, synth.make_inputs(wl, with_weights=False)
     wl = synth.WORKLOADS[name]
     return wl, synth.make_inputs(wl, bias_override=fitted_bias(name))
 
@@ -247,20 +253,40 @@ def run_ours(args):
     dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
     train = wl.backward
     gemm_only = wl.group_rows is not None
+    gate_only = args.workload == "gate_only"
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
-    x, w1, w2 = bf(inp["x"]), bf(inp["w1"]), bf(inp["w2"])
+    x = bf(inp["x"])
+    w1 = bf(inp["w1"]) if not gate_only else None
+    w2 = bf(inp["w2"]) if not gate_only else None
     wg = torch.from_numpy(inp["wg"]).to(dev) if not gemm_only else None
     bias = torch.from_numpy(inp["bias"]).to(dev) if not gemm_only else None
     dout = bf(inp["dout"]) if train else None
-    b = layer.MoEBuffers(dims, device=dev, train=train)
+    if gate_only:
+        class _GateBufs:  # the gate's outputs only
+            topk_idx = torch.empty(dm.T, dm.k, dtype=torch.int32, device=dev)
+            topk_w = torch.empty(dm.T, dm.k, dtype=torch.float32, device=dev)
+            ws = torch.zeros(moe.moe_workspace_size(dims), dtype=torch.uint8, device=dev)
+            out = torch.empty(dm.T, dm.d, dtype=torch.bfloat16, device=dev)
+        b = _GateBufs()
+    else:
+        b = layer.MoEBuffers(dims, device=dev, train=train)
     if gemm_only:
         counts = torch.tensor(wl.group_rows, dtype=torch.int32, device=dev)
         moe.grouped_gemm_set_groups(dims, counts, b.offsets, b.ws)
     torch.cuda.synchronize()
 
     def step(s, xx=x, gg=dout, ev=None):
+        if gate_only:
+            if ev is not None:
+                ev["t0"].append(torch.cuda.Event(enable_timing=True))
+                ev["t0"][-1].record(s)
+            moe.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, s)
+            if ev is not None:
+                ev["gate"].append(torch.cuda.Event(enable_timing=True))
+                ev["gate"][-1].record(s)
+            return
         if gemm_only:
             if ev is not None:
                 ev["t0"].append(torch.cuda.Event(enable_timing=True))
@@ -331,7 +357,8 @@ def run_ours(args):
     tokens_per_s = world * dm.T / (ms / 1000.0)
 
     # ---- per-call breakdown (separate instrumented pass; not the headline)
-    names = (["t0", "fwd"] if gemm_only else ["t0", "gate", "permute", "fwd", "combine"]) + (
+    names = (["t0", "gate"] if gate_only else
+             ["t0", "fwd"] if gemm_only else ["t0", "gate", "permute", "fwd", "combine"]) + (
         ["combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute"] if train else [])
     ev = {n: [] for n in names}
     nprof = max(3, min(args.steps, 20))
@@ -343,7 +370,7 @@ def run_ours(args):
     for i in range(1, len(names)):
         a, c = ev[names[i - 1]], ev[names[i]]
         per[names[i]] = sum(x0.elapsed_time(x1) for x0, x1 in zip(a, c)) / nprof
-    flops = gemm_flops(dm, train)
+    flops = gemm_flops(dm, train) if not gate_only else {"gate": 2 * dm.T * dm.d * dm.E}
     gemm_ms = sum(per[k] for k in flops)
     gemm_tflops = sum(flops.values()) / (gemm_ms / 1000.0) / 1e12
     pk, pk_src = peaks()
@@ -389,7 +416,8 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after timing: {moe.moe_status_string(status)}")
 
-    launches_per_step = 2 if gemm_only else 1 + 5 + 2 + 1 + ((2 + 4 + 1) if train else 0)
+    launches_per_step = (1 if gate_only else 2 if gemm_only else
+                         1 + 5 + 2 + 1 + ((2 + 4 + 1) if train else 0))
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -412,7 +440,7 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not gemm_only:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not (gemm_only or gate_only):
         line["cpu_baseline"] = cpu_baseline(wl, inp)
     if rank == 0:
         print(json.dumps(line), flush=True)

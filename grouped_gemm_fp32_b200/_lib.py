@@ -18,13 +18,16 @@ EXPORTS = (
     "moe_rows_routed", "moe_rows_total", "moe_workspace_size", "moe_gate_topk",
     "moe_permute_align", "moe_permute_align_static", "grouped_gemm_set_groups",
     "grouped_gemm_fwd", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd", "moe_get_device_status",
-    "moe_status_string",
+    "moe_status_string", "moe_last_cuda_error",
 )
 
 
 class MoeError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what} failed: {moe_status_string(status)} ({status})")
+        msg = f"{what} failed: {moe_status_string(status)} ({status})"
+        if status == -3:
+            msg += f": {moe_last_cuda_error()}"
+        super().__init__(msg)
         self.status = status
 
 
@@ -72,6 +75,7 @@ def load():
         "moe_combine_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_get_device_status": (i32, [vp, vp, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
+        "moe_last_cuda_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -105,6 +109,10 @@ def _ck(rc: int, what: str):
 
 def moe_status_string(status: int) -> str:
     return load().moe_status_string(int(status)).decode()
+
+
+def moe_last_cuda_error() -> str:
+    return load().moe_last_cuda_error().decode()
 
 
 def moe_rows_routed(dims: MoeDims) -> int:

@@ -135,7 +135,7 @@ int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, con
   else
     combine_kernel_any<<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k, dm.S, Rr,
                                                       o);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
@@ -148,7 +148,7 @@ int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, con
   combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(
       reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), row_of, w, dm.T,
       dm.d / 8, dm.k, reinterpret_cast<uint4*>(dy), dw);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

@@ -6,12 +6,14 @@
 // and "Load balancing" (a per-expert bias is added to the affinity scores only
 // to decide the top-k routing).
 //
-// One CTA owns TM tokens and all E experts.  The logits tile [TM, E] is an
+// One CTA owns a tile of tokens and all E experts.  The logits tile [TM, E] is an
 // FP32 SIMT GEMM (no tensor cores: the gate is the one FP32 contraction of the
 // layer): X and Wg are staged through shared memory in K chunks of 32, each
 // thread accumulates 4 tokens x 8 experts in registers, so every Wg value
 // loaded from L2 is reused TM times.  TM is chosen so the grid is about one
-// CTA per SM.  The finished logits go to shared memory and each warp then
+// CTA per SM; the next K chunk is prefetched into registers while the current
+// one is multiplied (one barrier per chunk).  The finished logits go to shared
+// memory and each warp then
 // routes one token at a time: softmax (max-subtracted, expf), s = p + bias,
 // k rounds of a warp-shuffle arg-max (equal s -> lower index), and the
 // renormalised weights.
@@ -23,81 +25,18 @@
 namespace moe {
 namespace {
 
-constexpr int KC = 32;  // K chunk
+constexpr int KC = 32;    // K chunk
+constexpr int MAXV = 4;   // 16-byte prefetch registers per thread and operand
 
-__global__ void gate_topk_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wg,
-                                 const float* __restrict__ bias, int64_t T, int d, int E, int k,
-                                 int TM, int32_t* __restrict__ topk_idx,
-                                 float* __restrict__ topk_w, float* __restrict__ probs) {
-  extern __shared__ float sm[];
-  const int NE = E / 8;                 // expert groups (8 experts each)
-  const int tid = threadIdx.x;
-  const int eg = tid % NE, tg = tid / NE;  // this thread: experts 8eg.., tokens 4tg..
-  const bool active = tg < TM / 4;         // the block is padded to whole warps
-  const int64_t t0 = (int64_t)blockIdx.x * TM;
-  const int nthreads = blockDim.x;
+constexpr int MAX_THREADS = 512;
 
-  float* Xs = sm;             // [KC][TM]  transposed token chunk
-  float* Ws = sm + KC * TM;   // [KC][E]   transposed gate chunk
-
-  float acc[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-
-  for (int k0 = 0; k0 < d; k0 += KC) {
-    // stage X[t0 .. t0+TM, k0 .. k0+KC) (bf16 -> f32, exact) and Wg[:, k0 .. k0+KC)
-    for (int i = tid; i < TM * (KC / 8); i += nthreads) {
-      const int r = i / (KC / 8), c8 = (i % (KC / 8)) * 8;
-      const int64_t t = t0 + r;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < T) v = *reinterpret_cast<const uint4*>(x + t * d + k0 + c8);
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        Xs[(c8 + 2 * p) * TM + r] = __uint_as_float(u[p] << 16);
-        Xs[(c8 + 2 * p + 1) * TM + r] = __uint_as_float(u[p] & 0xFFFF0000u);
-      }
-    }
-    for (int i = tid; i < E * (KC / 4); i += nthreads) {
-      const int e = i / (KC / 4), c4 = (i % (KC / 4)) * 4;
-      const float4 v = *reinterpret_cast<const float4*>(wg + (int64_t)e * d + k0 + c4);
-      Ws[(c4 + 0) * E + e] = v.x;
-      Ws[(c4 + 1) * E + e] = v.y;
-      Ws[(c4 + 2) * E + e] = v.z;
-      Ws[(c4 + 3) * E + e] = v.w;
-    }
-    __syncthreads();
-    if (active) {
-#pragma unroll 8
-      for (int kk = 0; kk < KC; ++kk) {
-        const float4 xa = *reinterpret_cast<const float4*>(Xs + kk * TM + tg * 4);
-        const float4 w0 = *reinterpret_cast<const float4*>(Ws + kk * E + eg * 8);
-        const float4 w1 = *reinterpret_cast<const float4*>(Ws + kk * E + eg * 8 + 4);
-        const float xv[4] = {xa.x, xa.y, xa.z, xa.w};
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
-      }
-    }
-    __syncthreads();
-  }
-
-  // logits tile -> shared memory [TM][E]
-  float* L = sm;
-  if (active) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) L[(tg * 4 + i) * E + eg * 8 + j] = acc[i][j];
-  }
-  __syncthreads();
-
-  // routing: one warp per token
-  const int warp = tid >> 5, lane = tid & 31, nwarps = nthreads >> 5;
+// Routing of the TM tokens whose logits sit in shared memory L[TM][E]: one warp
+// per token.
+__device__ __forceinline__ void route_tile(const float* L, int64_t t0, int TM, int64_t T, int E,
+                                           int k, const float* __restrict__ bias,
+                                           int32_t* __restrict__ topk_idx,
+                                           float* __restrict__ topk_w, float* __restrict__ probs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int per = (E + 31) / 32;  // experts per lane (<= 8)
   for (int r = warp; r < TM; r += nwarps) {
     const int64_t t = t0 + r;
@@ -162,6 +101,239 @@ __global__ void gate_topk_kernel(const __nv_bfloat16* __restrict__ x, const floa
   }
 }
 
+// Generic path (any E % 8 == 0): 4 tokens x 8 experts per thread.
+__global__ void __launch_bounds__(MAX_THREADS)
+    gate_topk_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wg,
+                                 const float* __restrict__ bias, int64_t T, int d, int E, int k,
+                                 int TM, int32_t* __restrict__ topk_idx,
+                                 float* __restrict__ topk_w, float* __restrict__ probs) {
+  extern __shared__ float sm[];
+  const int NE = E / 8;                    // expert groups (8 experts each)
+  const int tid = threadIdx.x;
+  const int eg = tid % NE, tg = tid / NE;  // this thread: experts 8eg.., tokens 4tg..
+  const bool active = tg < TM / 4;         // the block is padded to whole warps
+  const int64_t t0 = (int64_t)blockIdx.x * TM;
+  const int nthreads = blockDim.x;
+  const int buf_floats = KC * (TM + E);    // one stage: Xs [KC][TM] then Ws [KC][E]
+
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  // Prefetch of one K chunk into registers.  X: 16-byte piece (row r, cols c8..c8+7)
+  // for i = r + TM * (c8 / 8); W: (expert e, cols c4..c4+3) for i = e + E * (c4 / 4).
+  // Consecutive threads take consecutive rows / experts, so the transposed
+  // shared-memory stores below hit consecutive banks.
+  uint4 xr[MAXV];
+  float4 wr[MAXV];
+  auto load_chunk = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < MAXV; ++u) {
+      const int i = tid + u * nthreads;
+      if (i < TM * (KC / 8)) {
+        const int r = i % TM, c8 = (i / TM) * 8;
+        const int64_t t = t0 + r;
+        xr[u] = t < T ? *reinterpret_cast<const uint4*>(x + t * d + k0 + c8) : make_uint4(0, 0, 0, 0);
+      }
+      if (i < E * (KC / 4)) {
+        const int e = i % E, c4 = (i / E) * 4;
+        wr[u] = *reinterpret_cast<const float4*>(wg + (int64_t)e * d + k0 + c4);
+      }
+    }
+  };
+  auto store_chunk = [&](float* buf) {
+    float* Xs = buf;
+    float* Ws = buf + KC * TM;
+#pragma unroll
+    for (int u = 0; u < MAXV; ++u) {
+      const int i = tid + u * nthreads;
+      if (i < TM * (KC / 8)) {
+        const int r = i % TM, c8 = (i / TM) * 8;
+        const uint32_t w4[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          Xs[(c8 + 2 * p) * TM + r] = __uint_as_float(w4[p] << 16);
+          Xs[(c8 + 2 * p + 1) * TM + r] = __uint_as_float(w4[p] & 0xFFFF0000u);
+        }
+      }
+      if (i < E * (KC / 4)) {
+        const int e = i % E, c4 = (i / E) * 4;
+        Ws[(c4 + 0) * E + e] = wr[u].x;
+        Ws[(c4 + 1) * E + e] = wr[u].y;
+        Ws[(c4 + 2) * E + e] = wr[u].z;
+        Ws[(c4 + 3) * E + e] = wr[u].w;
+      }
+    }
+  };
+
+  const int nchunks = d / KC;
+  load_chunk(0);
+  store_chunk(sm);
+  __syncthreads();
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + 1 < nchunks) load_chunk((c + 1) * KC);  // in flight while this chunk computes
+    const float* Xs = sm + (c & 1) * buf_floats;
+    const float* Ws = Xs + KC * TM;
+    if (active) {
+#pragma unroll 8
+      for (int kk = 0; kk < KC; ++kk) {
+        const float4 xa = *reinterpret_cast<const float4*>(Xs + kk * TM + tg * 4);
+        const float4 w0 = *reinterpret_cast<const float4*>(Ws + kk * E + eg * 8);
+        const float4 w1 = *reinterpret_cast<const float4*>(Ws + kk * E + eg * 8 + 4);
+        const float xv[4] = {xa.x, xa.y, xa.z, xa.w};
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+      }
+    }
+    if (c + 1 < nchunks) store_chunk(sm + ((c + 1) & 1) * buf_floats);
+    __syncthreads();
+  }
+
+  // logits tile -> shared memory [TM][E]
+  float* L = sm;
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) L[(tg * 4 + i) * E + eg * 8 + j] = acc[i][j];
+  }
+  __syncthreads();
+
+  route_tile(L, t0, TM, T, E, k, bias, topk_idx, topk_w, probs);
+}
+
+
+// Fast path (E % 32 == 0): 32 tokens per CTA, 4 tokens x 4 experts per thread,
+// E * 2 threads (8 warps for E = 128).
+//  * Wg chunks [E][32] are copied into shared memory unchanged with cp.async
+//    (whole 128-byte rows: coalesced, no register staging), three chunks in
+//    flight; X chunks are widened to f32 through registers one chunk ahead.
+//  * Thread (tg, eg) owns tokens tg + 8i and experts eg + (E/4) j and reads
+//    4 consecutive K values of each as one float4.  Rows are padded to 36
+//    floats, so the 8 expert rows / 4 token rows a warp reads at once fall in
+//    distinct banks: every read is a conflict-free broadcast, 8 reads per 64
+//    FFMAs.  Small CTAs let several share an SM to hide latency.
+constexpr int TM32 = 32;
+constexpr int RS = KC + 4;  // padded row stride (floats)
+constexpr int WSTAGES = 3;
+
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(512)
+    gate_topk_kernel_t32(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wg,
+                         const float* __restrict__ bias, int64_t T, int d, int E, int k,
+                         int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                         float* __restrict__ probs) {
+  extern __shared__ float sm[];
+  float* Ws = sm;                          // [WSTAGES][E][RS]
+  float* Xs = sm + WSTAGES * E * RS;       // [2][TM32][RS]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int EQ = E / 4;                          // expert groups
+  const int WE = E / 32;                         // warps across the experts
+  const int eg = (warp % WE) * 8 + (lane & 7);   // experts eg + EQ * j
+  const int tg = (warp / WE) * 4 + (lane >> 3);  // tokens tg + 8 * i  (tg < 8)
+  const int64_t t0 = (int64_t)blockIdx.x * TM32;
+  const int nthreads = blockDim.x;  // 2E
+
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+
+  auto issue_w = [&](int c) {  // Wg[:, 32c .. 32c+32) -> stage c % 3, 8 pieces of 16 B a row
+    float* dst = Ws + (c % WSTAGES) * E * RS;
+    for (int i = tid; i < E * 8; i += nthreads) {
+      const int e = i >> 3, q = i & 7;
+      cp_async16(dst + e * RS + q * 4, wg + (int64_t)e * d + c * KC + q * 4);
+    }
+  };
+  uint4 xr;
+  const bool has_x = tid < TM32 * (KC / 8);  // 128 pieces of 8 bf16
+  const int xrow = tid % TM32, xc8 = (tid / TM32) * 8;
+  auto load_x = [&](int c) {
+    if (has_x) {
+      const int64_t t = t0 + xrow;
+      xr = t < T ? *reinterpret_cast<const uint4*>(x + t * d + c * KC + xc8)
+                 : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto store_x = [&](int c) {
+    if (has_x) {
+      float* dst = Xs + (c & 1) * TM32 * RS + xrow * RS + xc8;
+      const uint32_t w4[4] = {xr.x, xr.y, xr.z, xr.w};
+      *reinterpret_cast<float4*>(dst) =
+          make_float4(__uint_as_float(w4[0] << 16), __uint_as_float(w4[0] & 0xFFFF0000u),
+                      __uint_as_float(w4[1] << 16), __uint_as_float(w4[1] & 0xFFFF0000u));
+      *reinterpret_cast<float4*>(dst + 4) =
+          make_float4(__uint_as_float(w4[2] << 16), __uint_as_float(w4[2] & 0xFFFF0000u),
+                      __uint_as_float(w4[3] << 16), __uint_as_float(w4[3] & 0xFFFF0000u));
+    }
+  };
+
+  const int n = d / KC;
+  issue_w(0);
+  cp_async_commit();
+  if (n > 1) issue_w(1);
+  cp_async_commit();
+  load_x(0);
+  store_x(0);
+  if (n > 1) load_x(1);
+  for (int c = 0; c < n; ++c) {
+    cp_async_wait<1>();  // this thread's copies of chunk c have landed
+    __syncthreads();     // everyone's have; chunk c - 1 is no longer being read
+    if (c + 2 < n) issue_w(c + 2);
+    cp_async_commit();   // (possibly empty: keeps the group count uniform)
+    if (c + 1 < n) store_x(c + 1);
+    if (c + 2 < n) load_x(c + 2);
+    const float* W = Ws + (c % WSTAGES) * E * RS;
+    const float* X = Xs + (c & 1) * TM32 * RS;
+#pragma unroll 2
+    for (int kk = 0; kk < KC; kk += 4) {
+      float4 xv[4], wv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(X + (tg + 8 * i) * RS + kk);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wv[j] = *reinterpret_cast<const float4*>(W + (eg + EQ * j) * RS + kk);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] = fmaf(xv[i].x, wv[j].x, acc[i][j]);
+          acc[i][j] = fmaf(xv[i].y, wv[j].y, acc[i][j]);
+          acc[i][j] = fmaf(xv[i].z, wv[j].z, acc[i][j]);
+          acc[i][j] = fmaf(xv[i].w, wv[j].w, acc[i][j]);
+        }
+    }
+  }
+  __syncthreads();
+
+  float* L = sm;  // logits tile [32][E] (reuses the Wg stages)
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) L[(tg + 8 * i) * E + eg + EQ * j] = acc[i][j];
+  __syncthreads();
+  route_tile(L, t0, TM32, T, E, k, bias, topk_idx, topk_w, probs);
+}
+
 }  // namespace
 
 int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const float* bias,
@@ -175,27 +347,46 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
   }
   const int64_t T = dm.T;
   if (T == 0) return MOE_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dm.E % 32 == 0 && dm.E <= 256) {
+    const int threads = 2 * dm.E;
+    const size_t smem = sizeof(float) * RS * (WSTAGES * dm.E + 2 * TM32);  // >= [32][E] logits
+    if (smem > 48 * 1024 &&
+        !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel_t32,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return MOE_ERR_CUDA;
+    const int64_t blocks = (T + TM32 - 1) / TM32;
+    gate_topk_kernel_t32<<<(unsigned)blocks, threads, smem, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), wg, bias, T, dm.d, dm.E, dm.k, idx, w, probs);
+    return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
+  }
   // about one CTA per SM: TM tokens per CTA, a multiple of 4 in [4, 128]
   int64_t per = (T + num_sms - 1) / num_sms;
   int TM = (int)((per + 3) / 4 * 4);
   if (TM < 4) TM = 4;
   if (TM > 128) TM = 128;
   const int NE = dm.E / 8;
-  while (TM > 4 && (TM / 4) * NE > 1024) TM -= 4;
-  const int threads = ((TM / 4) * NE + 31) / 32 * 32;
-  const size_t stage_bytes = sizeof(float) * KC * (TM + dm.E);
+  while (TM > 4 && (TM / 4) * NE > MAX_THREADS) TM -= 4;
+  auto r32 = [](int v) { return (v + 31) / 32 * 32; };
+  int threads = r32((TM / 4) * NE);
+  // every thread's share of a chunk must fit its MAXV prefetch registers
+  while (threads < MAX_THREADS &&
+         (TM * (KC / 8) > MAXV * threads || dm.E * (KC / 4) > MAXV * threads))
+    threads += 32;
+  if (TM * (KC / 8) > MAXV * threads || dm.E * (KC / 4) > MAXV * threads)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  const size_t stage_bytes = 2 * sizeof(float) * KC * (TM + dm.E);
   const size_t logit_bytes = sizeof(float) * (size_t)TM * dm.E;
   const size_t smem = stage_bytes > logit_bytes ? stage_bytes : logit_bytes;
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(gate_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  }
+  if (smem > 48 * 1024 &&
+      !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem)))
+    return MOE_ERR_CUDA;
   const int64_t blocks = (T + TM - 1) / TM;
-  gate_topk_kernel<<<(unsigned)blocks, threads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+  gate_topk_kernel<<<(unsigned)blocks, threads, smem, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(x), wg, bias, T, dm.d, dm.E, dm.k, TM, idx, w,
       probs);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

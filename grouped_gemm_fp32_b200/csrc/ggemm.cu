@@ -4,16 +4,22 @@
 // Passage: dots.llm1 Technical Report, §3.2 "Efficient implementation of
 // Grouped GEMM".  Every expert's token segment is padded to a fixed block, so
 // a 128-row tile never straddles two experts and scheduling reduces to that of
-// a plain GEMM: tiles are (group, m-tile, n-tile) triples enumerated from a
-// per-group prefix of m-tile counts that is built on the device (no host
+// a plain GEMM: tiles are (group, 256-row tile, n-tile) triples enumerated from
+// a per-group prefix of 256-row tile counts that is built on the device (no host
 // round trip).  The pages' version targets sm_90 warpgroup MMA; this one is
-// written for sm_100a: one CTA per SM walks tiles persistently,
-//   warp 0        TMA producer (4-stage shared-memory ring, 48 KB a stage)
-//   warp 1        tensor-memory owner and single-thread tcgen05.mma issuer
-//   warps 2..5    epilogue: tcgen05.ld of the FP32 accumulator, fused
-//                 SwiGLU / SwiGLU-backward / bf16 or f32 store
-// with two 128x256 FP32 accumulators in tensor memory so the epilogue of one
-// tile overlaps the MMAs of the next.
+// written for sm_100a.  CTAs run in pairs (a 2-CTA cluster, one CTA per SM) and
+// walk 256 x 256 tiles persistently with the paired tcgen05.mma (cta_group::2):
+// each CTA stages its own 128 rows of A and half of B (N/2 columns), so one
+// SM's shared memory feeds half the B traffic of a 1-CTA 128 x 256 tile.
+//   warp 0        TMA producer of this CTA's halves (6-stage ring, 32 KB a stage);
+//                 completions are counted on the leader CTA's barriers
+//   warp 1        tensor-memory owner; in the leader CTA the single-thread
+//                 tcgen05.mma issuer for the pair
+//   warps 2..9    epilogue of this CTA's 128 accumulator rows (two warps per
+//                 32-lane quarter, each on half the columns): tcgen05.ld, fused
+//                 SwiGLU / SwiGLU-backward, bf16 or f32 stores
+// with two 256-column FP32 accumulators in tensor memory per CTA so the
+// epilogue of one tile overlaps the MMAs of the next.
 //
 // Six GEMMs of the expert FFN share this kernel (A is M x K, B is N x K):
 //   FWD1  A = x rows (K-major)     B = W1 gate|up rows (K-major)  -> SwiGLU -> H (+ A1)
@@ -36,14 +42,16 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128;           // UMMA M (rows of A per tile)
+constexpr int BM = 128;           // rows of A per CTA (the pair's UMMA M is 256)
+constexpr int PM = 2 * BM;        // rows of a pair tile
 constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;    // 16 KB
-constexpr int B_BYTES = 256 * BK * 2;   // 32 KB (N up to 256)
-constexpr int NUM_THREADS = 192;
+constexpr int MAX_STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;    // 16 KB: this CTA's 128 rows of A
+constexpr int B_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of B (N/2 <= 128)
+constexpr int EPI_WARPS = 8;            // two per tensor-memory lane quarter
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;     // two 256-column FP32 accumulators
-constexpr int MAX_GROUPS = 264;
+constexpr int MAX_GROUPS = 264;  // E <= 256 routed + S <= 8 shared
 
 struct GemmArgs {
   int* status;
@@ -54,7 +62,7 @@ struct GemmArgs {
   int K;             // reduction length (FWD/DX)
   int n_out;         // valid output columns
   int m_out;         // DW: valid output rows
-  int NT, MT;        // n-tiles per group; DW: m-tiles per group
+  int NT, MT;        // n-tiles per group; DW: 256-row m-tiles per group
   int hn;            // FWD1: H columns per tile (64 or 128)
   int I;             // FWD1 / DX2: intermediate size
   int b_group_rows;  // rows one group occupies in B's 2-D view
@@ -67,49 +75,64 @@ struct GemmArgs {
   uint64_t budget_ns;
 };
 
+// full[] and tempty[] are used in the leader CTA only (both CTAs' producers and
+// epilogues signal the leader's); empty[] and tfull[] exist in both CTAs and
+// receive the leader's multicast commits.
 struct SmemCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  int total_tiles;
 };
 
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + STAGES * (A_BYTES + B_BYTES) +
-                              sizeof(SmemCtl) + sizeof(GroupRec) * MAX_GROUPS +
-                              sizeof(int) * (MAX_GROUPS + 1) + sizeof(int) * MAX_GROUPS + 64;
+template <int MODE>
+__host__ __device__ constexpr int stages_of() {
+  return MAX_STAGES;
+}
+
+template <int MODE>
+constexpr size_t smem_bytes() {
+  return 1024 /* alignment slack */ + stages_of<MODE>() * (A_BYTES + B_BYTES) +
+         sizeof(SmemCtl) + 64;
+}
 
 struct TileInfo {
   int g, m0, n0, nkb;
 };
 
+__device__ __forceinline__ GroupRec load_group(const GemmArgs& a, int g) {
+  const int4 v = __ldg(reinterpret_cast<const int4*>(a.groups) + g);
+  return GroupRec{v.x, v.y, v.z, v.w};
+}
+
 template <int MODE>
-__device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a, const GroupRec* sg,
-                                                const int* spre, const int* sord) {
+__device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
   TileInfo t;
   if constexpr (MODE == MODE_DW2 || MODE == MODE_DW1) {
     const int per = a.MT * a.NT;
     const int gi = tile / per, local = tile - gi * per;
-    t.g = sord[gi];
+    t.g = __ldg(a.dw_order + gi);
     const int nt = local / a.MT, mt = local - nt * a.MT;
-    t.m0 = mt * BM;
+    t.m0 = mt * PM;
     t.n0 = nt * 256;
-    t.nkb = (sg[t.g].rows_pad + BK - 1) / BK;  // the tail block reads zeros past the end
+    t.nkb = (load_group(a, t.g).rows_pad + BK - 1) / BK;  // the tail block reads zeros past the end
   } else {
-    // largest g with spre[g] * NT <= tile  (spre is non-decreasing)
+    // largest g with prefix[g] * NT <= tile  (the prefix is non-decreasing)
+    const int* pre = a.mtile_prefix;
     int lo = 0, hi = a.G - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (spre[mid] * a.NT <= tile) lo = mid; else hi = mid - 1;
+      if (__ldg(pre + mid) * a.NT <= tile) lo = mid; else hi = mid - 1;
     }
     t.g = lo;
-    const int mt_g = spre[lo + 1] - spre[lo];
-    const int local = tile - spre[lo] * a.NT;
+    const int p0 = __ldg(pre + lo);
+    const int mt_g = __ldg(pre + lo + 1) - p0;
+    const int local = tile - p0 * a.NT;
     const int nt = local / mt_g, mt = local - nt * mt_g;
-    t.m0 = mt * BM;
+    t.m0 = mt * PM;
     t.n0 = nt * (MODE == MODE_FWD1 ? a.hn : 256);
     t.nkb = a.K / BK;
   }
@@ -149,13 +172,15 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v)
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ggemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                 const __grid_constant__ CUtensorMap tmC /* DX2: saved [G | U] */,
                  const GemmArgs args) {
   constexpr bool A_MN = (MODE == MODE_DW2 || MODE == MODE_DW1);
   constexpr bool B_MN = (MODE != MODE_FWD1 && MODE != MODE_FWD2);
   constexpr bool IS_DW = A_MN;
+  constexpr int STAGES = stages_of<MODE>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -163,28 +188,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sB + STAGES * B_BYTES);
-  GroupRec* sg = reinterpret_cast<GroupRec*>(ctl + 1);
-  int* spre = reinterpret_cast<int*>(sg + MAX_GROUPS);
-  int* sord = spre + (MAX_GROUPS + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   volatile int* abort_flag = &ctl->abort_flag;
 
-  for (int i = threadIdx.x; i < args.G; i += NUM_THREADS) {
-    sg[i] = args.groups[i];
-    spre[i] = args.mtile_prefix[i];
-    sord[i] = args.dw_order[i];
-  }
   if (threadIdx.x == 0) {
-    spre[args.G] = args.mtile_prefix[args.G];
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ctl->tfull[a], 1);
-      mbar_init(&ctl->tempty[a], 4);
+      mbar_init(&ctl->tempty[a], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
@@ -193,28 +212,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    if (MODE == MODE_DX2) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  const int total_tiles = IS_DW ? args.G * args.MT * args.NT : spre[args.G] * args.NT;
+  const int total_tiles =
+      IS_DW ? args.G * args.MT * args.NT : __ldg(args.mtile_prefix + args.G) * args.NT;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, lastpar = 0;
-      const uint32_t a_bytes = A_BYTES;
-      const uint32_t b_bytes = (MODE == MODE_FWD1) ? (uint32_t)(2 * args.hn * BK * 2) : B_BYTES;
+      const uint32_t b_bytes = (MODE == MODE_FWD1) ? (uint32_t)(args.hn * BK * 2) : B_BYTES;
+      const uint32_t pair_bytes = 2 * (A_BYTES + b_bytes);  // both CTAs' copies
+      const int roff = (int)rank * BM;                       // this CTA's 128 rows / columns
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileInfo t = decode_tile<MODE>(tile, args, sg, spre, sord);
-        const GroupRec gr = sg[t.g];
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+        const TileInfo t = decode_tile<MODE>(tile, args);
+        const GroupRec gr = load_group(args, t.g);
         const bool shared = t.g >= args.E;
         for (int kb = 0; kb < t.nkb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1, abort_flag, args.status,
@@ -222,27 +245,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          uint64_t* fb = &ctl->full[stage];
-          mbar_arrive_expect_tx(fb, a_bytes + b_bytes);
+          if (leader) mbar_arrive_expect_tx(&ctl->full[stage], pair_bytes);
+          const uint32_t fb = map_to_rank(&ctl->full[stage], 0);
           uint8_t* a_dst = sA + stage * A_BYTES;
           uint8_t* b_dst = sB + stage * B_BYTES;
           const int k0 = kb * BK;
           if constexpr (MODE == MODE_FWD1) {
-            tma_load_2d(a_dst, shared ? &tmA1 : &tmA0, fb, k0, (shared ? 0 : gr.a_row) + t.m0);
-            const int brow = t.g * args.b_group_rows + t.n0;
-            tma_load_2d(b_dst, &tmB0, fb, k0, brow);
-            tma_load_2d(b_dst + args.hn * 128, &tmB0, fb, k0, brow + args.I);
+            // A: rows m0 + roff; B: the leader stages the gate rows, the peer the up rows
+            tma_load_2d_pair(a_dst, shared ? &tmA1 : &tmA0, fb, k0,
+                             (shared ? 0 : gr.a_row) + t.m0 + roff);
+            tma_load_2d_pair(b_dst, &tmB0, fb, k0,
+                             t.g * args.b_group_rows + t.n0 + (leader ? 0 : args.I));
           } else if constexpr (MODE == MODE_FWD2) {
-            tma_load_2d(a_dst, &tmA0, fb, k0, gr.out_row + t.m0);
-            tma_load_2d(b_dst, &tmB0, fb, k0, t.g * args.b_group_rows + t.n0);
+            tma_load_2d_pair(a_dst, &tmA0, fb, k0, gr.out_row + t.m0 + roff);
+            tma_load_2d_pair(b_dst, &tmB0, fb, k0, t.g * args.b_group_rows + t.n0 + roff);
           } else if constexpr (MODE == MODE_DX2 || MODE == MODE_DX1) {
-            if constexpr (MODE == MODE_DX2)
-              tma_load_2d(a_dst, shared ? &tmA1 : &tmA0, fb, k0, (shared ? 0 : gr.a_row) + t.m0);
-            else
-              tma_load_2d(a_dst, &tmA0, fb, k0, gr.out_row + t.m0);
+            if constexpr (MODE == MODE_DX2) {
+              // the epilogue of this tile reads the saved [G | U] of its rows: start
+              // pulling them into L2 now, a whole K loop ahead
+              if (kb == 0) {
+                const int y = gr.out_row + t.m0 + roff;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                  if (t.n0 + c * 64 < args.I) {
+                    tma_prefetch_l2_2d(&tmC, t.n0 + c * 64, y);
+                    tma_prefetch_l2_2d(&tmC, args.I + t.n0 + c * 64, y);
+                  }
+              }
+              tma_load_2d_pair(a_dst, shared ? &tmA1 : &tmA0, fb, k0,
+                               (shared ? 0 : gr.a_row) + t.m0 + roff);
+            } else {
+              tma_load_2d_pair(a_dst, &tmA0, fb, k0, gr.out_row + t.m0 + roff);
+            }
             const int brow = t.g * args.b_group_rows + k0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tma_load_2d(b_dst + c * 8192, &tmB0, fb, t.n0 + c * 64, brow);
+            for (int c = 0; c < 2; ++c)
+              tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + roff + c * 64, brow);
           } else {  // DW2 / DW1: K runs over the group's rows
             const CUtensorMap* ma;
             const CUtensorMap* mb;
@@ -259,9 +297,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               brow = shared ? 0 : gr.a_row;
             }
 #pragma unroll
-            for (int c = 0; c < 2; ++c) tma_load_2d(a_dst + c * 8192, ma, fb, t.m0 + c * 64, arow + k0);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tma_load_2d(b_dst + c * 8192, mb, fb, t.n0 + c * 64, brow + k0);
+            for (int c = 0; c < 2; ++c) {
+              tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
+              tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + roff + c * 64, brow + k0);
+            }
           }
           issued |= 1u << stage;
           lastpar = (lastpar & ~(1u << stage)) | (phase << stage);
@@ -271,23 +310,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      // Every copy this thread started must land before the CTA may exit.
-      for (int s = 0; s < STAGES; ++s)
-        if (issued & (1u << s)) {
-          volatile int never = 0;
-          mbar_wait(&ctl->full[s], (lastpar >> s) & 1u, &never, args.status,
-                    MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
-        }
+      // The leader's full barriers count both CTAs' copies: once they have
+      // completed, every copy either CTA started has landed.
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) {
+            volatile int never = 0;
+            mbar_wait(&ctl->full[s], (lastpar >> s) & 1u, &never, args.status,
+                      MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
+          }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    // ------------------------------------------------- MMA issuer (leader) --
+    if (leader && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
-        const TileInfo t = decode_tile<MODE>(tile, args, sg, spre, sord);
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs, ++it) {
+        const TileInfo t = decode_tile<MODE>(tile, args);
         const int acc = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
         if (!mbar_wait(&ctl->tempty[acc], (use & 1u) ^ 1u, abort_flag, args.status,
@@ -310,29 +351,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                      : smem_desc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
                                      : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            umma_f16(d_tmem, ad, bd, args.idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_f16_pair(d_tmem, ad, bd, args.idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(&ctl->empty[stage]);
+          umma_commit_pair(&ctl->empty[stage], 0x3);  // frees this stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&ctl->tfull[acc]);
+        umma_commit_pair(&ctl->tfull[acc], 0x3);  // both CTAs' epilogues may read
       }
-      // Drain: all MMAs issued by this thread complete before tensor memory is freed.
-      umma_commit(&ctl->drain);
+      // Drain: every MMA issued completes before tensor memory is freed.
+      umma_commit_pair(&ctl->drain, 0x1);
       volatile int never = 0;
       mbar_wait(&ctl->drain, 0, &never, args.status, MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue --
-    const int q = warp & 3;  // this warp may read TMEM lanes [32q, 32q + 32)
-    const int r_in_tile = q * 32 + lane;
+    // Warps 2..9: warp w reads tensor-memory lanes [32q, 32q + 32), q = w % 4,
+    // and the half h of the accumulator's columns.
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    const int r_in_tile = (int)rank * BM + q * 32 + lane;  // row within the 256-row pair tile
+    const uint32_t tempty_leader[2] = {map_to_rank(&ctl->tempty[0], 0),
+                                       map_to_rank(&ctl->tempty[1], 0)};
+    // hand the accumulator back to the leader's MMA thread once this warp's last
+    // columns are in registers
+    auto release = [&](int acc) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(tempty_leader[acc]);
+    };
     int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      const TileInfo t = decode_tile<MODE>(tile, args, sg, spre, sord);
+    for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
+      const TileInfo t = decode_tile<MODE>(tile, args);
       const int acc = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (!mbar_wait(&ctl->tfull[acc], use & 1u, abort_flag, args.status, MOE_ERR_DEVICE_TIMEOUT,
@@ -340,7 +393,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
-      const GroupRec gr = sg[t.g];
+      const GroupRec gr = load_group(args, t.g);
       uint32_t r[32];
       float v[32];
       if constexpr (MODE == MODE_FWD1) {
@@ -349,10 +402,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int64_t orow = (int64_t)gr.out_row + rloc;
         __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0;
         __nv_bfloat16* A1 = reinterpret_cast<__nv_bfloat16*>(args.out2);
-        for (int c0 = 0; c0 < args.hn; c0 += 32) {
+        const int cb = h * (args.hn >> 1), ce = cb + (args.hn >> 1);  // this warp's H columns
+        for (int c0 = cb; c0 < ce; c0 += 32) {
           uint32_t u[32];
           tmem_ld32_sync(taddr + c0, r);
           tmem_ld32_sync(taddr + args.hn + c0, u);
+          if (c0 + 32 >= ce) release(acc);
           if (rv) {
             float hv[32];
 #pragma unroll
@@ -372,19 +427,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
+        if (cb >= ce) release(acc);
       } else if constexpr (MODE == MODE_FWD2 || MODE == MODE_DX1) {
         const int rloc = t.m0 + r_in_tile;
         const bool rv = rloc < gr.rows_pad;
         const int64_t orow = (int64_t)gr.out_row + rloc;
         __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0;
-        for (int c0 = 0; c0 < 256 && t.n0 + c0 < args.n_out; c0 += 32) {
+        const int cb = h * 128, ce = min(cb + 128, args.n_out - t.n0);
+        for (int c0 = cb; c0 < ce; c0 += 32) {
           tmem_ld32_sync(taddr + c0, r);
+          if (c0 + 32 >= ce) release(acc);
           if (rv) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
             store_bf16x32(O + c0, v);
           }
         }
+        if (cb >= ce) release(acc);
       } else if constexpr (MODE == MODE_DX2) {
         const int rloc = t.m0 + r_in_tile;
         const bool rv = rloc < gr.rows_pad;
@@ -392,13 +451,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const __nv_bfloat16* A1 =
             reinterpret_cast<const __nv_bfloat16*>(args.aux) + orow * args.ld_aux;
         __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out;
-        for (int c0 = 0; c0 < 256 && t.n0 + c0 < args.I; c0 += 32) {
-          tmem_ld32_sync(taddr + c0, r);
-          if (rv) {
-            const int col = t.n0 + c0;
-            float gv[32], uv[32], dg[32], du[32];
+        const int cb = h * 128, ce = min(cb + 128, args.I - t.n0);
+        for (int c0 = cb; c0 < ce; c0 += 32) {
+          const int col = t.n0 + c0;
+          float gv[32], uv[32];
+          if (rv) {  // issue the saved-activation loads before waiting on tensor memory
             load_bf16x32(A1 + col, gv);
             load_bf16x32(A1 + args.I + col, uv);
+          }
+          tmem_ld32_sync(taddr + c0, r);
+          if (c0 + 32 >= ce) release(acc);
+          if (rv) {
+            float dg[32], du[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float dh = __uint_as_float(r[i]);
@@ -411,46 +475,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             store_bf16x32(dA + args.I + col, du);
           }
         }
+        if (cb >= ce) release(acc);
       } else {  // DW2 / DW1: f32 output [G, m_out, n_out]
-        const int m = t.m0 + r_in_tile;
-        const bool rv = m < args.m_out;
-        float* O = reinterpret_cast<float*>(args.out) +
-                   ((int64_t)t.g * args.m_out + m) * (int64_t)args.n_out + t.n0;
-        for (int c0 = 0; c0 < 256 && t.n0 + c0 < args.n_out; c0 += 32) {
-          if (t.nkb > 0) {
-            tmem_ld32_sync(taddr + c0, r);
+        // 16-lane loads: 4 consecutive lanes hold 8 consecutive columns of one row,
+        // so every 8-byte store instruction writes 8 complete 32-byte row segments.
+        const int rb = t.m0 + (int)rank * BM + q * 32;  // this warp's 32 output rows
+        const bool wvalid = rb < args.m_out;             // m_out % 32 == 0: all or none
+        float* O = reinterpret_cast<float*>(args.out) + (int64_t)t.g * args.m_out * args.n_out;
+        const int cb = h * 128, ce = min(cb + 128, args.n_out - t.n0);
+        const int rsub = lane >> 2, csub = 2 * (lane & 3);
+        for (int c0 = cb; c0 < ce; c0 += 64) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          } else {
+          for (int half = 0; half < 2; ++half) {
+            if (t.nkb > 0) {
+              tmem_ld16x256_x8_sync(taddr + ((uint32_t)(16 * half) << 16) + c0, r);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-          }
-          if (rv) {
-            float4* o4 = reinterpret_cast<float4*>(O + c0);
+              for (int i = 0; i < 32; ++i) r[i] = 0u;
+            }
+            if (half == 1 && c0 + 64 >= ce) release(acc);
+            if (wvalid && !((t.nkb == 0) && args.accumulate)) {
+              const int64_t row0 = rb + 16 * half + rsub;
+              float* p0 = O + row0 * args.n_out + t.n0 + c0 + csub;
+              float* p1 = p0 + 8 * (int64_t)args.n_out;
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              float4 w = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-              if (args.accumulate) {
-                const float4 o = o4[q4];
-                w.x += o.x; w.y += o.y; w.z += o.z; w.w += o.w;
+              for (int i = 0; i < 8; ++i) {
+                float2 a = make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+                float2 b = make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                float2* d0 = reinterpret_cast<float2*>(p0 + 8 * i);
+                float2* d1 = reinterpret_cast<float2*>(p1 + 8 * i);
+                if (args.accumulate) {
+                  const float2 o0 = *d0, o1 = *d1;
+                  a.x += o0.x; a.y += o0.y; b.x += o1.x; b.y += o1.y;
+                }
+                *d0 = a;
+                *d1 = b;
               }
-              o4[q4] = w;
             }
           }
         }
+        if (cb >= ce) release(acc);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // neither CTA leaves while the other may still signal it or use the pair's memory
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -474,36 +549,54 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 matrix [rows, cols] (row-major, cols contiguous), box {64, box_rows}, 128B swizzle.
+// Row-major bf16 matrix [rows, cols] (cols contiguous); box = 64 elements (128
+// bytes) of a row x box_rows rows, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc || base == nullptr) return false;
+  const int esz = 2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 template <int MODE>
 int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
-                const CUtensorMap& b1, const GemmArgs& args, cudaStream_t st) {
+                const CUtensorMap& b1, const CUtensorMap& c, const GemmArgs& args,
+                cudaStream_t st) {
   static int num_sms = 0;
   static bool attr_set = false;
+  constexpr size_t kSmem = smem_bytes<MODE>();
+  static_assert(kSmem <= 232448, "shared memory per CTA exceeds 227 KB");
   if (!attr_set) {
-    if (cudaFuncSetAttribute(ggemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(ggemm_kernel<MODE>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem)))
       return MOE_ERR_CUDA;
     int dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    num_sms &= ~1;  // whole CTA pairs, one CTA per SM
+    // A pair needs two co-scheduled SMs: launch only as many pairs as can be
+    // resident at once, so the static tile split has no late-starting pairs.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)num_sms);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = kSmem;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, ggemm_kernel<MODE>, &cfg) == cudaSuccess &&
+        clusters > 0 && 2 * clusters < num_sms)
+      num_sms = 2 * clusters;
+    cudaGetLastError();  // a failed query only leaves the default grid
     attr_set = true;
   }
-  ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmemBytes, st>>>(a0, a1, b0, b1, args);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmem, st>>>(a0, a1, b0, b1, c, args);
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 uint64_t wait_budget_ns() {
@@ -540,7 +633,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   a.accumulate = ops.accumulate;
   a.budget_ns = wait_budget_ns();
 
-  CUtensorMap m0{}, m1{}, n0{}, n1{};
+  CUtensorMap m0{}, m1{}, n0{}, n1{}, c0{};
   bool ok = true;
   // a dummy map stands in for unused slots (never read by the kernel)
   auto same = [](CUtensorMap& dst, const CUtensorMap& src) { dst = src; };
@@ -556,13 +649,13 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.b_group_rows = 2 * I;
       a.ld_out = I;
       a.ld_out2 = 2 * I;
-      a.idesc = idesc_bf16_f32(BM, 2 * hn, false, false);
+      a.idesc = idesc_bf16_f32(PM, 2 * hn, false, false);
       ok &= make_map(&m0, ops.a0, Rr, d, BM);
       if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map(&n0, ops.b0, (int64_t)G * 2 * I, d, hn);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, a, st);
+      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, a, st);
     }
     case MODE_FWD2: {
       a.K = I;
@@ -570,13 +663,13 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.n_out = d;
       a.b_group_rows = d;
       a.ld_out = d;
-      a.idesc = idesc_bf16_f32(BM, 256, false, false);
+      a.idesc = idesc_bf16_f32(PM, 256, false, false);
       ok &= make_map(&m0, ops.a0, Rt, I, BM);
       same(m1, m0);
-      ok &= make_map(&n0, ops.b0, (int64_t)G * d, I, 256);
+      ok &= make_map(&n0, ops.b0, (int64_t)G * d, I, 128);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, a, st);
+      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, a, st);
     }
     case MODE_DX2: {
       a.K = d;
@@ -585,13 +678,14 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.b_group_rows = d;
       a.ld_out = 2 * I;
       a.ld_aux = 2 * I;
-      a.idesc = idesc_bf16_f32(BM, 256, false, true);
+      a.idesc = idesc_bf16_f32(PM, 256, false, true);
       ok &= make_map(&m0, ops.a0, Rr, d, BM);
       if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map(&n0, ops.b0, (int64_t)G * d, I, 64);
       same(n1, n0);
+      ok &= make_map(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX2>(m0, m1, n0, n1, a, st);
+      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, a, st);
     }
     case MODE_DX1: {
       a.K = 2 * I;
@@ -599,39 +693,39 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.n_out = d;
       a.b_group_rows = 2 * I;
       a.ld_out = d;
-      a.idesc = idesc_bf16_f32(BM, 256, false, true);
+      a.idesc = idesc_bf16_f32(PM, 256, false, true);
       ok &= make_map(&m0, ops.a0, Rt, 2 * I, BM);
       same(m1, m0);
       ok &= make_map(&n0, ops.b0, (int64_t)G * 2 * I, d, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX1>(m0, m1, n0, n1, a, st);
+      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, a, st);
     }
     case MODE_DW2: {  // dW2_g [d, I] = dY_g^T H_g
       a.m_out = d;
       a.n_out = I;
-      a.MT = (d + BM - 1) / BM;
+      a.MT = (d + PM - 1) / PM;
       a.NT = (I + 255) / 256;
-      a.idesc = idesc_bf16_f32(BM, 256, true, true);
+      a.idesc = idesc_bf16_f32(PM, 256, true, true);
       ok &= make_map(&m0, ops.a0, Rr, d, 64);
       if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, 64); else same(m1, m0);
       ok &= make_map(&n0, ops.b0, Rt, I, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW2>(m0, m1, n0, n1, a, st);
+      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, a, st);
     }
     case MODE_DW1: {  // dW1_g [2I, d] = dA_g^T X_g
       a.m_out = 2 * I;
       a.n_out = d;
-      a.MT = (2 * I) / BM;
+      a.MT = (2 * I + PM - 1) / PM;
       a.NT = (d + 255) / 256;
-      a.idesc = idesc_bf16_f32(BM, 256, true, true);
+      a.idesc = idesc_bf16_f32(PM, 256, true, true);
       ok &= make_map(&m0, ops.a0, Rt, 2 * I, 64);
       same(m1, m0);
       ok &= make_map(&n0, ops.b0, Rr, d, 64);
       if (dm.S > 0) ok &= make_map(&n1, ops.b1, T, d, 64); else same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW1>(m0, m1, n0, n1, a, st);
+      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, a, st);
     }
   }
   return MOE_ERR_INVALID_ARG;

@@ -7,6 +7,20 @@
 
 using namespace moe;
 
+namespace moe {
+
+namespace {
+thread_local cudaError_t g_last_error = cudaSuccess;
+}
+
+bool cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return true;
+  g_last_error = e;
+  return false;
+}
+
+}  // namespace moe
+
 namespace {
 
 bool dims_ok(const moe_dims* dm) {
@@ -161,14 +175,17 @@ int moe_get_device_status(void* ws, int32_t* status_out, void* stream) {
   if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int32_t v = 0;
-  if (cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
+  if (!cuda_ok(cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st)) ||
+      !cuda_ok(cudaStreamSynchronize(st)))
     return MOE_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
+  if (!cuda_ok(cudaMemsetAsync(ws, 0, sizeof(int32_t), st)) || !cuda_ok(cudaStreamSynchronize(st)))
     return MOE_ERR_CUDA;
   *status_out = v;
   return MOE_OK;
+}
+
+const char* moe_last_cuda_error(void) {
+  return g_last_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_error);
 }
 
 const char* moe_status_string(int status) {

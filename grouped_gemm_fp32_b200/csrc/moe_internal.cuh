@@ -4,9 +4,14 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "../../include/moe.h"
 
 namespace moe {
+
+// Records the error of a failing CUDA call for moe_last_cuda_error(); true on success.
+bool cuda_ok(cudaError_t e);
 
 // One group of the grouped GEMM: a routed expert (g < E) or a shared expert.
 //   a_row    first row of the group in its A source (x_perm for routed groups,
@@ -19,11 +24,12 @@ struct GroupRec {
 };
 
 constexpr int kChunk = 1024;      // routed assignments per histogram chunk
-constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] m-tiles total
+constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] tiles total,
+                                  // [3] routing valid, [4] bad expert id seen
 
 struct WsLayout {
   size_t groups;        // GroupRec[G]
-  size_t mtile_prefix;  // int32[G + 1]  prefix of ceil(rows_pad / 128)
+  size_t mtile_prefix;  // int32[G + 1]  prefix of ceil(rows_pad / 256) (pair tiles)
   size_t dw_order;      // int32[G]      groups by padded rows, largest first
   size_t chunk_hist;    // int32[nchunks * E]
   size_t bytes;

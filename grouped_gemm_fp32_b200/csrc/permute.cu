@@ -11,7 +11,7 @@
 //   1. hist:     each chunk of 1024 (t, j) assignments counts its experts.
 //   2. groups:   one CTA turns the chunk counts into per-chunk bases (exclusive
 //                scan over chunks per expert), pads each c_e to P, scans the
-//                experts, and writes the group table, the m-tile prefix and the
+//                experts, and writes the group table, the tile prefix and the
 //                heavy-first group order used by the weight-gradient GEMMs.
 //   3. scatter:  each chunk ranks its assignments in order (warp match + per-
 //                warp counts) and writes sorted_ids and row_of.
@@ -103,7 +103,7 @@ __global__ void groups_kernel(int32_t* __restrict__ hist, int nchunks, int E, in
       r.rows_pad = (int32_t)T;
     }
     groups[g] = r;  // (routed g < E <= 256 is handled by thread g, which holds c_g)
-    s_mt[g] = (r.rows_pad + 127) / 128;
+    s_mt[g] = (r.rows_pad + 255) / 256;  // 256-row tiles of the paired-CTA GEMM
     s_pad[g] = r.rows_pad;
   }
   __syncthreads();
@@ -243,7 +243,7 @@ static int launch_groups(const moe_dims& dm, int32_t* hist, int nchunks, int32_t
                                    reinterpret_cast<int32_t*>(wsb + L.mtile_prefix),
                                    reinterpret_cast<int32_t*>(wsb + L.dw_order),
                                    reinterpret_cast<int*>(wsb));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_t* counts,
@@ -257,12 +257,12 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
   const int64_t n = dm.T * dm.k;
   const int64_t Rr = rows_routed(dm);
 
-  if (cudaMemsetAsync(sorted_ids, 0xFF, sizeof(int32_t) * Rr, st) != cudaSuccess ||
-      cudaMemsetAsync(wsb + 3 * sizeof(int), 0, 2 * sizeof(int), st) != cudaSuccess)
+  if (!cuda_ok(cudaMemsetAsync(sorted_ids, 0xFF, sizeof(int32_t) * Rr, st)) ||
+      !cuda_ok(cudaMemsetAsync(wsb + 3 * sizeof(int), 0, 2 * sizeof(int), st)))
     return MOE_ERR_CUDA;
   if (n > 0) {
     hist_kernel<<<L.nchunks, 256, 0, st>>>(idx, n, dm.E, hist, status);
-  } else if (cudaMemsetAsync(hist, 0, sizeof(int32_t) * dm.E, st) != cudaSuccess) {
+  } else if (!cuda_ok(cudaMemsetAsync(hist, 0, sizeof(int32_t) * dm.E, st))) {
     return MOE_ERR_CUDA;
   }
   int rc = launch_groups(dm, hist, L.nchunks, counts, offsets, ws, st);
@@ -283,7 +283,7 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
                                                          reinterpret_cast<uint4*>(x_perm), status);
   zero_pad_rows_kernel<<<dm.E, 256, 0, st>>>(reinterpret_cast<const GroupRec*>(wsb + L.groups),
                                              row_vec, reinterpret_cast<uint4*>(x_perm));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offsets, void* ws,
@@ -292,9 +292,9 @@ int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offset
   const WsLayout L = ws_layout(dm);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
   int32_t* hist = reinterpret_cast<int32_t*>(wsb + L.chunk_hist);
-  if (cudaMemcpyAsync(hist, counts, sizeof(int32_t) * dm.E, cudaMemcpyDeviceToDevice, st) !=
-          cudaSuccess ||
-      cudaMemsetAsync(wsb + 3 * sizeof(int), 0, 2 * sizeof(int), st) != cudaSuccess)
+  if (!cuda_ok(cudaMemcpyAsync(hist, counts, sizeof(int32_t) * dm.E, cudaMemcpyDeviceToDevice,
+                               st)) ||
+      !cuda_ok(cudaMemsetAsync(wsb + 3 * sizeof(int), 0, 2 * sizeof(int), st)))
     return MOE_ERR_CUDA;
   return launch_groups(dm, hist, 1, nullptr, offsets, ws, st);
 }
@@ -305,7 +305,7 @@ int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, 
   const uint8_t* wsb = reinterpret_cast<const uint8_t*>(ws);
   zero_pad_rows_kernel<<<dm.E, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const GroupRec*>(wsb + L.groups), cols / 8, reinterpret_cast<uint4*>(m));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

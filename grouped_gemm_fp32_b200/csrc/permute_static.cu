@@ -30,14 +30,14 @@ void* scratch_for_current_device(int* rc) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (!cuda_ok(cudaGetDevice(&dev)) || dev < 0 || dev >= kMaxDevices) {
     *rc = MOE_ERR_CUDA;
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) {
+    if (!cuda_ok(cudaGetSymbolAddress(&p, g_permute_scratch)) || p == nullptr) {
       *rc = MOE_ERR_CUDA;
       return nullptr;
     }
@@ -72,8 +72,8 @@ extern "C" int moe_permute_align_static(const moe_dims* dims, const int32_t* top
   if (rc != MOE_OK) return rc;
   // The array keeps whatever the previous call left: start every call from a
   // clean header (status word and routing flags).
-  if (cudaMemsetAsync(ws, 0, kHeaderWords * sizeof(int32_t),
-                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (!cuda_ok(cudaMemsetAsync(ws, 0, kHeaderWords * sizeof(int32_t),
+                               reinterpret_cast<cudaStream_t>(stream))))
     return MOE_ERR_CUDA;
   return launch_permute(*dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_perm, ws,
                         stream);

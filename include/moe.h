@@ -219,6 +219,10 @@ int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, cons
  * *status_out receives MOE_OK or the first device error recorded. */
 int moe_get_device_status(void* ws, int32_t* status_out, void* stream);
 
+/* The CUDA error string behind the calling thread's most recent MOE_ERR_CUDA
+ * ("no error" if there was none). */
+const char* moe_last_cuda_error(void);
+
 /* Human-readable name of a moe_status value. */
 const char* moe_status_string(int status);
 

@@ -11,6 +11,7 @@ Workloads follow the configurations the layer is measured on:
 * ``layer``     T=8192, d=4096, E=128 top-6, S=2, I=1408, pad 128, seed 2.
 * ``skewed``    as ``layer`` with a Zipf(1.2)-shaped load bias, seed 3.
 * ``train``     T=16384, rest as ``layer``, forward+backward, seed 4.
+* ``train_small`` T=2048, E=16, rest as ``train`` (a small case for profiles), seed 5.
 
 Stream ids: 1 hidden states X (or the permuted A of ``gemm_only``), 2 gate
 weights Wg, 3 selection bias, 4 W1 (gate|up), 5 W2 (down), 6 upstream grad.
@@ -147,6 +148,10 @@ WORKLOADS = {
     "skewed": Workload("skewed", Dims(T=8192, d=4096, E=128, k=6, S=2, I=1408, P=128), seed=3),
     "train": Workload("train", Dims(T=16384, d=4096, E=128, k=6, S=2, I=1408, P=128), seed=4,
                       backward=True),
+    # profiling stand-in for ``train``: the same ~768 rows per routed expert and
+    # the same d, I, k, P, with 16 experts so a capture holds ~2.5 GB
+    "train_small": Workload("train_small", Dims(T=2048, d=4096, E=16, k=6, S=2, I=1408, P=128),
+                            seed=5, backward=True),
 }
 
 
