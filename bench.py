@@ -378,38 +378,54 @@ def run_ours(args):
     gemm_detail = {k: {"ms": round(per[k], 4), "tflops": round(flops[k] / per[k] / 1e9, 1)}
                    for k in flops}
 
-    # ---- e2e: pinned host inputs in, results out, through the same C ABI calls
-    hx = torch.from_numpy(inp["x"]).view(torch.bfloat16).pin_memory()
-    hd = torch.from_numpy(inp["dout"]).view(torch.bfloat16).pin_memory() if train else None
-    out_dev = b.y[: dm.T] if gemm_only else b.out
-    ho = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory()
-    hdx = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() if train else None
-    dx_in = torch.empty_like(x)
-    dd_in = torch.empty_like(dout) if train else None
-    h2d = hx.numel() * 2 + (hd.numel() * 2 if train else 0)
-    d2h = ho.numel() * 2 + (hdx.numel() * 2 if train else 0)
+    # ---- e2e: pinned host inputs in, results out, every step, through the same
+    # C-ABI calls; neighbouring steps' copies overlap compute (layer.HostPipeline)
+    pinned = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
+    e2e_note = "inputs H2D and results D2H every step, overlapped with neighbouring steps"
+    if gate_only or gemm_only:
+        hx = pinned(inp["x"])
+        ho = torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory()
+        dx_in = torch.empty_like(x)
+        h2d, d2h = hx.numel() * 2, ho.numel() * 2
+        out_dev = b.y[: dm.T] if gemm_only else b.out
 
-    def e2e_step():
-        dx_in.copy_(hx, non_blocking=True)
-        if train:
-            dd_in.copy_(hd, non_blocking=True)
-        step(stream, xx=dx_in, gg=dd_in)
-        ho.copy_(out_dev, non_blocking=True)
-        if train:
-            hdx.copy_(b.dx, non_blocking=True)
+        def e2e_run(nsteps):
+            with torch.cuda.stream(stream):
+                for _ in range(nsteps):
+                    dx_in.copy_(hx, non_blocking=True)
+                    step(stream, xx=dx_in)
+                    ho.copy_(out_dev, non_blocking=True)
+        e2e_streams = [stream]
+        e2e_note = "inputs H2D and results D2H every step, serialised with compute"
+    else:
+        pipe = layer.HostPipeline(dims, w1, w2, wg, bias, train, device=dev)
+        hx = [pinned(inp["x"])]
+        hd = [pinned(inp["dout"])] if train else [None]
+        ho = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        hdx = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        h2d = hx[0].numel() * 2 + (hd[0].numel() * 2 if train else 0)
+        d2h = ho[0].numel() * 2 + (hdx[0].numel() * 2 if train else 0)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            e2e_step()
-    stream.synchronize()
+        def e2e_run(nsteps):
+            pipe.run(hx, hd, ho, hdx, nsteps)
+        e2e_streams = [pipe.up, pipe.compute, pipe.down]
+
+    e2e_run(2)
+    for sst in e2e_streams:
+        sst.synchronize()
     barrier(world)
     ne2e = max(3, args.steps // 2)
+    torch.cuda.synchronize(dev)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        f0.record(stream)
-        for _ in range(ne2e):
-            e2e_step()
-        f1.record(stream)
+    f0.record(e2e_streams[0])
+    for sst in e2e_streams[1:]:
+        sst.wait_event(f0)
+    e2e_run(ne2e)
+    for sst in e2e_streams[:-1]:
+        ev = torch.cuda.Event()
+        ev.record(sst)
+        e2e_streams[-1].wait_event(ev)
+    f1.record(e2e_streams[-1])
     f1.synchronize()
     e2e_ms = dist_max(f0.elapsed_time(f1) / ne2e, world, dev)
     status = moe.moe_get_device_status(b.ws, stream)
@@ -436,7 +452,8 @@ def run_ours(args):
         "grouped_gemm": gemm_detail,
         "breakdown_ms": {k: round(v, 4) for k, v in per.items()},
         "e2e": {"value": world * dm.T / (e2e_ms / 1000.0), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "note": e2e_note},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }

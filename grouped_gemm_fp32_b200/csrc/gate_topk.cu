@@ -208,8 +208,8 @@ __global__ void __launch_bounds__(MAX_THREADS)
 }
 
 
-// Fast path (E % 32 == 0): 32 tokens per CTA, 4 tokens x 4 experts per thread,
-// E * 2 threads (8 warps for E = 128).
+// Fast path (E % 32 == 0): 8 * TI tokens per CTA (32 or 64), TI tokens x 4
+// experts per thread, E * 2 threads (8 warps for E = 128).
 //  * Wg chunks [E][32] are copied into shared memory unchanged with cp.async
 //    (whole 128-byte rows: coalesced, no register staging), three chunks in
 //    flight; X chunks are widened to f32 through registers one chunk ahead.
@@ -218,7 +218,6 @@ __global__ void __launch_bounds__(MAX_THREADS)
 //    floats, so the 8 expert rows / 4 token rows a warp reads at once fall in
 //    distinct banks: every read is a conflict-free broadcast, 8 reads per 64
 //    FFMAs.  Small CTAs let several share an SM to hide latency.
-constexpr int TM32 = 32;
 constexpr int RS = KC + 4;  // padded row stride (floats)
 constexpr int WSTAGES = 3;
 
@@ -236,11 +235,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// TI = token rows per thread (4 or 8): the CTA covers TM = 8 * TI tokens.
+template <int TI>
 __global__ void __launch_bounds__(512)
     gate_topk_kernel_t32(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wg,
                          const float* __restrict__ bias, int64_t T, int d, int E, int k,
                          int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                          float* __restrict__ probs) {
+  constexpr int TM32 = 8 * TI;             // tokens of this CTA
   extern __shared__ float sm[];
   float* Ws = sm;                          // [WSTAGES][E][RS]
   float* Xs = sm + WSTAGES * E * RS;       // [2][TM32][RS]
@@ -252,9 +254,9 @@ __global__ void __launch_bounds__(512)
   const int64_t t0 = (int64_t)blockIdx.x * TM32;
   const int nthreads = blockDim.x;  // 2E
 
-  float acc[4][4];
+  float acc[TI][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < TI; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
 
@@ -265,26 +267,36 @@ __global__ void __launch_bounds__(512)
       cp_async16(dst + e * RS + q * 4, wg + (int64_t)e * d + c * KC + q * 4);
     }
   };
-  uint4 xr;
-  const bool has_x = tid < TM32 * (KC / 8);  // 128 pieces of 8 bf16
-  const int xrow = tid % TM32, xc8 = (tid / TM32) * 8;
+  // X pieces of 8 bf16: TM32 * 4 of them, at most 2 per thread (2E >= 64 threads... E >= 32)
+  constexpr int XP = (TM32 * (KC / 8) + 63) / 64;
+  uint4 xr[XP];
   auto load_x = [&](int c) {
-    if (has_x) {
-      const int64_t t = t0 + xrow;
-      xr = t < T ? *reinterpret_cast<const uint4*>(x + t * d + c * KC + xc8)
-                 : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < XP; ++u) {
+      const int i = tid + u * nthreads;
+      if (i < TM32 * (KC / 8)) {
+        const int xrow = i % TM32, xc8 = (i / TM32) * 8;
+        const int64_t t = t0 + xrow;
+        xr[u] = t < T ? *reinterpret_cast<const uint4*>(x + t * d + c * KC + xc8)
+                      : make_uint4(0, 0, 0, 0);
+      }
     }
   };
   auto store_x = [&](int c) {
-    if (has_x) {
-      float* dst = Xs + (c & 1) * TM32 * RS + xrow * RS + xc8;
-      const uint32_t w4[4] = {xr.x, xr.y, xr.z, xr.w};
-      *reinterpret_cast<float4*>(dst) =
-          make_float4(__uint_as_float(w4[0] << 16), __uint_as_float(w4[0] & 0xFFFF0000u),
-                      __uint_as_float(w4[1] << 16), __uint_as_float(w4[1] & 0xFFFF0000u));
-      *reinterpret_cast<float4*>(dst + 4) =
-          make_float4(__uint_as_float(w4[2] << 16), __uint_as_float(w4[2] & 0xFFFF0000u),
-                      __uint_as_float(w4[3] << 16), __uint_as_float(w4[3] & 0xFFFF0000u));
+#pragma unroll
+    for (int u = 0; u < XP; ++u) {
+      const int i = tid + u * nthreads;
+      if (i < TM32 * (KC / 8)) {
+        const int xrow = i % TM32, xc8 = (i / TM32) * 8;
+        float* dst = Xs + (c & 1) * TM32 * RS + xrow * RS + xc8;
+        const uint32_t w4[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+        *reinterpret_cast<float4*>(dst) =
+            make_float4(__uint_as_float(w4[0] << 16), __uint_as_float(w4[0] & 0xFFFF0000u),
+                        __uint_as_float(w4[1] << 16), __uint_as_float(w4[1] & 0xFFFF0000u));
+        *reinterpret_cast<float4*>(dst + 4) =
+            make_float4(__uint_as_float(w4[2] << 16), __uint_as_float(w4[2] & 0xFFFF0000u),
+                        __uint_as_float(w4[3] << 16), __uint_as_float(w4[3] & 0xFFFF0000u));
+      }
     }
   };
 
@@ -307,13 +319,13 @@ __global__ void __launch_bounds__(512)
     const float* X = Xs + (c & 1) * TM32 * RS;
 #pragma unroll 2
     for (int kk = 0; kk < KC; kk += 4) {
-      float4 xv[4], wv[4];
+      float4 xv[TI], wv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const float4*>(X + (tg + 8 * i) * RS + kk);
+      for (int i = 0; i < TI; ++i) xv[i] = *reinterpret_cast<const float4*>(X + (tg + 8 * i) * RS + kk);
 #pragma unroll
       for (int j = 0; j < 4; ++j) wv[j] = *reinterpret_cast<const float4*>(W + (eg + EQ * j) * RS + kk);
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < TI; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           acc[i][j] = fmaf(xv[i].x, wv[j].x, acc[i][j]);
@@ -325,9 +337,9 @@ __global__ void __launch_bounds__(512)
   }
   __syncthreads();
 
-  float* L = sm;  // logits tile [32][E] (reuses the Wg stages)
+  float* L = sm;  // logits tile [TM32][E] (reuses the Wg stages)
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < TI; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) L[(tg + 8 * i) * E + eg + EQ * j] = acc[i][j];
   __syncthreads();
@@ -349,15 +361,30 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
   if (T == 0) return MOE_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dm.E % 32 == 0 && dm.E <= 256) {
+    // 64 tokens per CTA (half the Wg staging per token) while that still gives
+    // every SM at least ~1.5 CTAs; 32 otherwise.
+    const bool wide = T >= (int64_t)64 * num_sms * 3 / 2;
+    const int TMv = wide ? 64 : 32;
     const int threads = 2 * dm.E;
-    const size_t smem = sizeof(float) * RS * (WSTAGES * dm.E + 2 * TM32);  // >= [32][E] logits
-    if (smem > 48 * 1024 &&
-        !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel_t32,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-      return MOE_ERR_CUDA;
-    const int64_t blocks = (T + TM32 - 1) / TM32;
-    gate_topk_kernel_t32<<<(unsigned)blocks, threads, smem, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(x), wg, bias, T, dm.d, dm.E, dm.k, idx, w, probs);
+    size_t smem = sizeof(float) * RS * (WSTAGES * dm.E + 2 * TMv);
+    if (smem < sizeof(float) * (size_t)TMv * dm.E) smem = sizeof(float) * (size_t)TMv * dm.E;
+    const int64_t blocks = (T + TMv - 1) / TMv;
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (wide) {
+      if (smem > 48 * 1024 &&
+          !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel_t32<8>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+        return MOE_ERR_CUDA;
+      gate_topk_kernel_t32<8><<<(unsigned)blocks, threads, smem, st>>>(xb, wg, bias, T, dm.d, dm.E,
+                                                                      dm.k, idx, w, probs);
+    } else {
+      if (smem > 48 * 1024 &&
+          !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel_t32<4>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+        return MOE_ERR_CUDA;
+      gate_topk_kernel_t32<4><<<(unsigned)blocks, threads, smem, st>>>(xb, wg, bias, T, dm.d, dm.E,
+                                                                      dm.k, idx, w, probs);
+    }
     return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
   }
   // about one CTA per SM: TM tokens per CTA, a multiple of 4 in [4, 128]

@@ -91,3 +91,74 @@ def backward(b: MoEBuffers, x, dout, w1, w2, stream=None):
     L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x, b.dw1, 0, stream)
     L.moe_combine(dm, b.dxp, b.row_of, None, b.dx, stream)
     return b.dx, b.dw1, b.dw2, b.dw_comb
+
+
+class HostPipeline:
+    """Forward (+ backward) steps fed from and returned to pinned host memory,
+    with the copies of neighbouring steps overlapped with compute.
+
+    Two device buffer sets alternate: while step i computes on set i % 2, the
+    inputs of step i + 1 are copied in on an upload stream and the results of
+    step i - 1 are copied out on a download stream.  Every step still moves its
+    inputs host -> device and its results device -> host; only the overlap is
+    added.  All arithmetic runs in libmoe.so; torch provides memory and streams.
+    """
+
+    def __init__(self, dims: L.MoeDims, w1, w2, wg, bias, train: bool, device="cuda"):
+        self.dims, self.train = dims, train
+        self.w1, self.w2, self.wg, self.bias = w1, w2, wg, bias
+        dev = torch.device(device)
+        T, d = dims.T, dims.d
+        self.bufs = [MoEBuffers(dims, device=dev, train=train) for _ in range(2)]
+        e = lambda: torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        self.x = [e(), e()]
+        self.dout = [e(), e()] if train else [None, None]
+        self.compute = torch.cuda.Stream(device=dev)
+        self.up = torch.cuda.Stream(device=dev)
+        self.down = torch.cuda.Stream(device=dev)
+        self.uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+        self.computed = [torch.cuda.Event(), torch.cuda.Event()]
+        self.downloaded = [torch.cuda.Event(), torch.cuda.Event()]
+        self.consumed = [torch.cuda.Event(), torch.cuda.Event()]
+        for ev in self.downloaded + self.consumed:
+            ev.record(self.compute)
+
+    def _upload(self, j, hx, hd):
+        with torch.cuda.stream(self.up):
+            self.up.wait_event(self.consumed[j])      # step j-2 no longer reads set j
+            self.x[j].copy_(hx, non_blocking=True)
+            if self.train:
+                self.dout[j].copy_(hd, non_blocking=True)
+            self.uploaded[j].record(self.up)
+
+    def run(self, host_x, host_dout, host_out, host_dx, steps: int):
+        """``steps`` steps; step i reads host_x[i % n] (and host_dout) and writes
+        host_out[i % n] (and host_dx).  Returns after all copies are issued;
+        synchronise the streams (or ``self.down``) to wait for the results."""
+        n = len(host_x)
+        self._upload(0, host_x[0], host_dout[0] if self.train else None)
+        for i in range(steps):
+            j = i & 1
+            if i + 1 < steps:
+                self._upload(1 - j, host_x[(i + 1) % n],
+                             host_dout[(i + 1) % n] if self.train else None)
+            b = self.bufs[j]
+            s = self.compute
+            with torch.cuda.stream(s):
+                s.wait_event(self.uploaded[j])
+                s.wait_event(self.downloaded[j])  # results of step i-2 have left set j
+                forward(b, self.x[j], self.wg, self.bias, self.w1, self.w2, stream=s)
+                if self.train:
+                    backward(b, self.x[j], self.dout[j], self.w1, self.w2, stream=s)
+                self.computed[j].record(s)
+                self.consumed[j].record(s)
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(self.computed[j])
+                host_out[i % n].copy_(b.out, non_blocking=True)
+                if self.train:
+                    host_dx[i % n].copy_(b.dx, non_blocking=True)
+                self.downloaded[j].record(self.down)
+
+    def synchronize(self):
+        for st in (self.up, self.compute, self.down):
+            st.synchronize()
