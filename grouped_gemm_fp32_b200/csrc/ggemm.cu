@@ -223,6 +223,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  // Waits that only make sure work already started has finished (copies in
+  // flight, MMAs issued) get a long budget of their own, so a short wait budget
+  // can never let this CTA free tensor memory or exit under them.
+  const uint64_t drain_budget = args.budget_ns > 2000000000ull ? args.budget_ns : 2000000000ull;
+  // A role that gives up tells the peer CTA too, so both stop issuing work.
+  const uint32_t peer_abort = map_to_rank(&ctl->abort_flag, rank ^ 1u);
+  auto abort_pair = [&]() {
+    *abort_flag = 1;
+    st_shared_cluster_u32(peer_abort, 1u);
+  };
   const int total_tiles =
       IS_DW ? args.G * args.MT * args.NT : __ldg(args.mtile_prefix + args.G) * args.NT;
 
@@ -242,6 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < t.nkb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1, abort_flag, args.status,
                          MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
+            abort_pair();
             ok = false;
             break;
           }
@@ -317,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (issued & (1u << s)) {
             volatile int never = 0;
             mbar_wait(&ctl->full[s], (lastpar >> s) & 1u, &never, args.status,
-                      MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
+                      MOE_ERR_DEVICE_TIMEOUT, drain_budget);
           }
     }
   } else if (warp == 1) {
@@ -332,13 +343,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int acc = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
         if (!mbar_wait(&ctl->tempty[acc], (use & 1u) ^ 1u, abort_flag, args.status,
-                       MOE_ERR_DEVICE_TIMEOUT, args.budget_ns))
+                       MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
+          abort_pair();
           break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
         for (int kb = 0; kb < t.nkb; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, abort_flag, args.status,
                          MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
+            abort_pair();
             ok = false;
             break;
           }
@@ -365,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       // Drain: every MMA issued completes before tensor memory is freed.
       umma_commit_pair(&ctl->drain, 0x1);
       volatile int never = 0;
-      mbar_wait(&ctl->drain, 0, &never, args.status, MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
+      mbar_wait(&ctl->drain, 0, &never, args.status, MOE_ERR_DEVICE_TIMEOUT, drain_budget);
     }
   } else {
     // ------------------------------------------------------------ epilogue --
@@ -389,8 +403,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const int acc = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (!mbar_wait(&ctl->tfull[acc], use & 1u, abort_flag, args.status, MOE_ERR_DEVICE_TIMEOUT,
-                     args.budget_ns))
+                     args.budget_ns)) {
+        abort_pair();
         break;
+      }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * 256) + ((uint32_t)(q * 32) << 16);
       const GroupRec gr = load_group(args, t.g);
@@ -520,6 +536,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   }
 
   tc_fence_before();
+  __syncthreads();
+  // After an abort, copies the peer started for this pair may still be landing
+  // (their completions are counted on the leader's barriers, which the
+  // aborting roles stopped waiting on): give them time before either CTA leaves.
+  if (*abort_flag && threadIdx.x == 0) spin_ns(100000);
   __syncthreads();
   cluster_sync();  // neither CTA leaves while the other may still signal it or use the pair's memory
   tc_fence_after();

@@ -6,7 +6,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/moe.h"
+#include "moe.h"  // include/ is on the include path
 
 namespace moe {
 
