@@ -72,6 +72,7 @@ struct GemmArgs {
   int64_t ld_out, ld_out2, ld_aux;
   int accumulate;
   uint32_t idesc;
+  uint32_t idesc_narrow;  // N = 128 (modes whose B is N-major)
   uint64_t budget_ns;
 };
 
@@ -101,6 +102,7 @@ constexpr size_t smem_bytes() {
 
 struct TileInfo {
   int g, m0, n0, nkb;
+  int nw;  // N of this tile's MMA: 256, or 128 for a last tile with <= 128 columns left
 };
 
 __device__ __forceinline__ GroupRec load_group(const GemmArgs& a, int g) {
@@ -119,6 +121,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     t.m0 = mt * PM;
     t.n0 = nt * 256;
     t.nkb = (load_group(a, t.g).rows_pad + BK - 1) / BK;  // the tail block reads zeros past the end
+    t.nw = (a.n_out - t.n0 > 128) ? 256 : 128;
   } else {
     // largest g with prefix[g] * NT <= tile  (the prefix is non-decreasing)
     const int* pre = a.mtile_prefix;
@@ -135,6 +138,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     t.m0 = mt * PM;
     t.n0 = nt * (MODE == MODE_FWD1 ? a.hn : 256);
     t.nkb = a.K / BK;
+    t.nw = (MODE == MODE_DX2 || MODE == MODE_DX1) && (a.n_out - t.n0 <= 128) ? 128 : 256;
   }
   return t;
 }
@@ -241,14 +245,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, lastpar = 0;
-      const uint32_t b_bytes = (MODE == MODE_FWD1) ? (uint32_t)(args.hn * BK * 2) : B_BYTES;
-      const uint32_t pair_bytes = 2 * (A_BYTES + b_bytes);  // both CTAs' copies
-      const int roff = (int)rank * BM;                       // this CTA's 128 rows / columns
+      const int roff = (int)rank * BM;                       // this CTA's 128 rows of A
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<MODE>(tile, args);
         const GroupRec gr = load_group(args, t.g);
         const bool shared = t.g >= args.E;
+        // this CTA's half of B: N/2 columns from n0 + rank * N/2, in 64-column chunks
+        const int bchunks = t.nw / 128;
+        const int boff = (int)rank * (t.nw / 2);
+        const uint32_t b_bytes = (MODE == MODE_FWD1) ? (uint32_t)(args.hn * BK * 2)
+                                 : B_MN ? (uint32_t)(bchunks * 8192) : (uint32_t)B_BYTES;
+        const uint32_t pair_bytes = 2 * (A_BYTES + b_bytes);  // both CTAs' copies
         for (int kb = 0; kb < t.nkb; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1, abort_flag, args.status,
                          MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
@@ -289,9 +297,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               tma_load_2d_pair(a_dst, &tmA0, fb, k0, gr.out_row + t.m0 + roff);
             }
             const int brow = t.g * args.b_group_rows + k0;
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + roff + c * 64, brow);
+            for (int c = 0; c < bchunks; ++c)
+              tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + boff + c * 64, brow);
           } else {  // DW2 / DW1: K runs over the group's rows
             const CUtensorMap* ma;
             const CUtensorMap* mb;
@@ -308,10 +315,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               brow = shared ? 0 : gr.a_row;
             }
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2; ++c)
               tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
-              tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + roff + c * 64, brow + k0);
-            }
+            for (int c = 0; c < bchunks; ++c)
+              tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + boff + c * 64, brow + k0);
           }
           issued |= 1u << stage;
           lastpar = (lastpar & ~(1u << stage)) | (phase << stage);
@@ -349,6 +356,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+        const uint32_t idesc = t.nw == 256 ? args.idesc : args.idesc_narrow;
         for (int kb = 0; kb < t.nkb; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, abort_flag, args.status,
                          MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
@@ -365,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                      : smem_desc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
                                      : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            umma_f16_pair(d_tmem, ad, bd, args.idesc, (kb | kk) != 0 ? 1u : 0u);
+            umma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair(&ctl->empty[stage], 0x3);  // frees this stage in both CTAs
           if (++stage == STAGES) {
@@ -700,6 +708,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.ld_out = 2 * I;
       a.ld_aux = 2 * I;
       a.idesc = idesc_bf16_f32(PM, 256, false, true);
+      a.idesc_narrow = idesc_bf16_f32(PM, 128, false, true);
       ok &= make_map(&m0, ops.a0, Rr, d, BM);
       if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map(&n0, ops.b0, (int64_t)G * d, I, 64);
@@ -715,6 +724,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.b_group_rows = 2 * I;
       a.ld_out = d;
       a.idesc = idesc_bf16_f32(PM, 256, false, true);
+      a.idesc_narrow = idesc_bf16_f32(PM, 128, false, true);
       ok &= make_map(&m0, ops.a0, Rt, 2 * I, BM);
       same(m1, m0);
       ok &= make_map(&n0, ops.b0, (int64_t)G * 2 * I, d, 64);
@@ -728,6 +738,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.MT = (d + PM - 1) / PM;
       a.NT = (I + 255) / 256;
       a.idesc = idesc_bf16_f32(PM, 256, true, true);
+      a.idesc_narrow = idesc_bf16_f32(PM, 128, true, true);
       ok &= make_map(&m0, ops.a0, Rr, d, 64);
       if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, 64); else same(m1, m0);
       ok &= make_map(&n0, ops.b0, Rt, I, 64);
@@ -741,6 +752,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.MT = (2 * I + PM - 1) / PM;
       a.NT = (d + 255) / 256;
       a.idesc = idesc_bf16_f32(PM, 256, true, true);
+      a.idesc_narrow = idesc_bf16_f32(PM, 128, true, true);
       ok &= make_map(&m0, ops.a0, Rt, 2 * I, 64);
       same(m1, m0);
       ok &= make_map(&n0, ops.b0, Rr, d, 64);
