@@ -90,6 +90,34 @@ def gemm_flops(dm, backward):
     return f
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ggemm_dram_traffic_train.txt")
+TRAFFIC_SOURCES = ["ggemm.cu", "sm100.cuh", "moe_internal.cuh", "permute.cu"]
+
+
+def gemm_traffic(name):
+    """DRAM bytes of one step's grouped-GEMM launches, from the committed ncu capture
+    of the train workload, while the kernel sources still hash to the captured ones
+    (None otherwise: the counters no longer describe the kernel that runs)."""
+    import hashlib
+    if name != "train" or not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture for this workload"
+    fields = {}
+    for line in open(TRAFFIC_FILE):
+        if ":" in line and not line.startswith("#"):
+            key, val = line.split(":", 1)
+            fields[key.strip()] = val.strip()
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "grouped_gemm_fp32_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != fields.get("sources_sha256"):
+        return None, "kernel sources changed since the capture"
+    return float(fields["dram_bytes_per_step"]), (
+        f"ncu dram__bytes_read.sum + dram__bytes_write.sum over the step's six GEMM launches "
+        f"({os.path.relpath(TRAFFIC_FILE, ROOT)}); algorithmic "
+        f"{float(fields['algorithmic_bytes_per_step']):.4g} B")
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -374,6 +402,7 @@ def run_ours(args):
     gemm_ms = sum(per[k] for k in flops)
     gemm_tflops = sum(flops.values()) / (gemm_ms / 1000.0) / 1e12
     pk, pk_src = peaks()
+    traffic, traffic_note = gemm_traffic(args.workload)
     sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     gemm_detail = {k: {"ms": round(per[k], 4), "tflops": round(flops[k] / per[k] / 1e9, 1)}
                    for k in flops}
@@ -448,7 +477,8 @@ def run_ours(args):
                      "frac": gemm_tflops / sustained,
                      "peak_kind": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
                      "frac_of_burst_peak": gemm_tflops / pk["bf16_tflops"],
-                     "traffic": None},
+                     "traffic": traffic, "traffic_unit": "bytes per step",
+                     "traffic_note": traffic_note},
         "grouped_gemm": gemm_detail,
         "breakdown_ms": {k: round(v, 4) for k, v in per.items()},
         "e2e": {"value": world * dm.T / (e2e_ms / 1000.0), "unit": "tokens/s",
