@@ -310,7 +310,7 @@ def run_ours(args):
             if ev is not None:
                 ev["t0"].append(torch.cuda.Event(enable_timing=True))
                 ev["t0"][-1].record(s)
-            moe.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, s)
+            moe.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, b.ws, s)
             if ev is not None:
                 ev["gate"].append(torch.cuda.Event(enable_timing=True))
                 ev["gate"][-1].record(s)
@@ -333,7 +333,7 @@ def run_ours(args):
         L = moe
         rec = lambda k: ev[k].append(torch.cuda.Event(enable_timing=True)) or ev[k][-1].record(s)
         rec("t0")
-        L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, s)
+        L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, b.ws, s)
         rec("gate")
         L.moe_permute_align(dims, b.topk_idx, xx, b.counts, b.offsets, b.sorted_ids, b.row_of,
                             b.x_perm, b.ws, s)

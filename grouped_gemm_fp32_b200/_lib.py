@@ -64,7 +64,7 @@ def load():
         "moe_rows_routed": (i64, [D]),
         "moe_rows_total": (i64, [D]),
         "moe_workspace_size": (sz, [D]),
-        "moe_gate_topk": (i32, [D, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_gate_topk": (i32, [D, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_permute_align": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "moe_permute_align_static": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "grouped_gemm_set_groups": (i32, [D, vp, vp, vp, sz, vp]),
@@ -127,9 +127,11 @@ def moe_workspace_size(dims: MoeDims) -> int:
     return int(load().moe_workspace_size(ctypes.byref(dims)))
 
 
-def moe_gate_topk(dims, x, wg, bias, topk_idx, topk_w, probs=None, stream=None):
+def moe_gate_topk(dims, x, wg, bias, topk_idx, topk_w, probs, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
     _ck(load().moe_gate_topk(ctypes.byref(dims), _p(x), _p(wg), _p(bias), _p(topk_idx),
-                             _p(topk_w), _p(probs), _s(stream)), "moe_gate_topk")
+                             _p(topk_w), _p(probs), _p(ws), nbytes, _s(stream)),
+        "moe_gate_topk")
 
 
 def moe_permute_align(dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_perm, ws,

@@ -6,34 +6,79 @@
 // and "Load balancing" (a per-expert bias is added to the affinity scores only
 // to decide the top-k routing).
 //
-// One CTA owns a tile of tokens and all E experts.  The logits tile [TM, E] is an
-// FP32 SIMT GEMM (no tensor cores: the gate is the one FP32 contraction of the
-// layer): X and Wg are staged through shared memory in K chunks of 32, each
-// thread accumulates 4 tokens x 8 experts in registers, so every Wg value
-// loaded from L2 is reused TM times.  TM is chosen so the grid is about one
-// CTA per SM; the next K chunk is prefetched into registers while the current
-// one is multiplied (one barrier per chunk).  The finished logits go to shared
-// memory and each warp then
-// routes one token at a time: softmax (max-subtracted, expf), s = p + bias,
-// k rounds of a warp-shuffle arg-max (equal s -> lower index), and the
-// renormalised weights.
+// The logits X Wg^T are a dense [T, d] x [d, E] contraction, so they run on the
+// tensor cores, without giving up FP32 accuracy:
+//   * X is bf16, an exact tcgen05 kind::f16 operand;
+//   * every FP32 gate weight is split into three bf16 terms, w = hi + mid + lo
+//     with hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid).  Both
+//     differences are exact in FP32, and what the three terms miss is below
+//     2^-24 |w|, under FP32's own rounding of w;
+//   * a product of two bf16 values is exact in FP32;
+//   * the tensor cores' FP32 accumulation is not round-to-nearest: measured on
+//     the layer workload, one accumulator over all of d = 4096 drifts ~10x
+//     further from the exact logits than an FP32 FMA loop.  So each 64-wide K
+//     block accumulates from zero in tensor memory (12 MMAs over small partial
+//     sums), and the block results are added in FP32 registers with
+//     round-to-nearest; the truncations of different blocks then have random
+//     signs and the logits match an FP32 FMA loop's accuracy.
+//
+// split_wg_kernel writes the three planes [3][E_pad][d] (bf16, rows E..E_pad-1
+// zero) into the layer workspace.  gate_tc_kernel, one CTA per 128 tokens:
+//   warp 0, lane 0   TMA producer: per 64-wide K block the 128 x 64 tile of X
+//                    and the three E_pad x 64 tiles of the planes, 128-byte swizzle
+//   warp 1           tensor-memory owner; lane 0 issues, per K block, 12 MMAs
+//                    (four 16-wide K steps x hi, mid, lo; M = 128, N = E_pad) into
+//                    one of two E_pad-column accumulators, alternating
+//   warps 2..9       summing warps (two per tensor-memory lane quarter, one column
+//                    half each): add each finished block accumulator into FP32
+//                    registers, then write the logits to shared memory
+//   all warps        routing, one warp per token: softmax (max-subtracted, expf),
+//                    s = p + bias, k rounds of a warp-shuffle arg-max (equal s ->
+//                    lower index), the renormalised weights
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "moe_internal.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int KC = 32;    // K chunk
-constexpr int MAXV = 4;   // 16-byte prefetch registers per thread and operand
+constexpr int GT_BM = 128;                    // tokens per CTA (UMMA M)
+constexpr int GT_BK = 64;                     // K per stage: one 128-byte swizzle row
+constexpr int GT_SUM_WARPS = 8;                // two per tensor-memory lane quarter
+constexpr int GT_THREADS = 64 + 32 * GT_SUM_WARPS;
+constexpr int GT_MAX_STAGES = 6;
+constexpr int GT_A_BYTES = GT_BM * GT_BK * 2;  // 16 KB
+constexpr int GT_MAX_SMEM = 232448;            // 227 KB
 
-constexpr int MAX_THREADS = 512;
+struct GateArgs {
+  int* status;
+  const float* bias;
+  int32_t* topk_idx;
+  float* topk_w;
+  float* probs;
+  int64_t T;
+  int d, E, e_pad, k, stages;
+  uint32_t stage_bytes, tmem_cols, idesc;
+  uint64_t budget_ns;
+};
 
-// Routing of the TM tokens whose logits sit in shared memory L[TM][E]: one warp
-// per token.
-__device__ __forceinline__ void route_tile(const float* L, int64_t t0, int TM, int64_t T, int E,
-                                           int k, const float* __restrict__ bias,
+struct GateCtl {
+  uint64_t full[GT_MAX_STAGES];
+  uint64_t empty[GT_MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Routing of the TM tokens whose logits sit in shared memory, row r at L + r * LS:
+// one warp per token.
+__device__ __forceinline__ void route_tile(const float* L, int LS, int64_t t0, int TM, int64_t T,
+                                           int E, int k, const float* __restrict__ bias,
                                            int32_t* __restrict__ topk_idx,
                                            float* __restrict__ topk_w, float* __restrict__ probs) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -46,7 +91,7 @@ __device__ __forceinline__ void route_tile(const float* L, int64_t t0, int TM, i
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int e = lane + 32 * q;
-      p[q] = (q < per && e < E) ? L[r * E + e] : -INFINITY;
+      p[q] = (q < per && e < E) ? L[r * LS + e] : -INFINITY;
       m = fmaxf(m, p[q]);
     }
 #pragma unroll
@@ -101,318 +146,285 @@ __device__ __forceinline__ void route_tile(const float* L, int64_t t0, int TM, i
   }
 }
 
-// Generic path (any E % 8 == 0): 4 tokens x 8 experts per thread.
-__global__ void __launch_bounds__(MAX_THREADS)
-    gate_topk_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wg,
-                                 const float* __restrict__ bias, int64_t T, int d, int E, int k,
-                                 int TM, int32_t* __restrict__ topk_idx,
-                                 float* __restrict__ topk_w, float* __restrict__ probs) {
-  extern __shared__ float sm[];
-  const int NE = E / 8;                    // expert groups (8 experts each)
-  const int tid = threadIdx.x;
-  const int eg = tid % NE, tg = tid / NE;  // this thread: experts 8eg.., tokens 4tg..
-  const bool active = tg < TM / 4;         // the block is padded to whole warps
-  const int64_t t0 = (int64_t)blockIdx.x * TM;
-  const int nthreads = blockDim.x;
-  const int buf_floats = KC * (TM + E);    // one stage: Xs [KC][TM] then Ws [KC][E]
-
-  float acc[4][8];
+// wg [E, d] f32 -> planes [3][e_pad][d] bf16: hi, mid, lo with hi + mid + lo = w
+// to below 2^-24 |w| (rows E..e_pad-1 are zero).  Four columns per thread.
+__global__ void split_wg_kernel(const float* __restrict__ wg, int E, int e_pad, int d,
+                                __nv_bfloat16* __restrict__ planes) {
+  const int64_t n4 = (int64_t)e_pad * d / 4;
+  const int64_t plane = (int64_t)e_pad * d;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i * 4 / d;
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < E) w = reinterpret_cast<const float4*>(wg)[i];
+    const float v[4] = {w.x, w.y, w.z, w.w};
+    uint32_t hi[2], mid[2], lo[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int c = 0; c < 2; ++c) {
+      __nv_bfloat16 h[2], m[2], l[2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-
-  // Prefetch of one K chunk into registers.  X: 16-byte piece (row r, cols c8..c8+7)
-  // for i = r + TM * (c8 / 8); W: (expert e, cols c4..c4+3) for i = e + E * (c4 / 4).
-  // Consecutive threads take consecutive rows / experts, so the transposed
-  // shared-memory stores below hit consecutive banks.
-  uint4 xr[MAXV];
-  float4 wr[MAXV];
-  auto load_chunk = [&](int k0) {
-#pragma unroll
-    for (int u = 0; u < MAXV; ++u) {
-      const int i = tid + u * nthreads;
-      if (i < TM * (KC / 8)) {
-        const int r = i % TM, c8 = (i / TM) * 8;
-        const int64_t t = t0 + r;
-        xr[u] = t < T ? *reinterpret_cast<const uint4*>(x + t * d + k0 + c8) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < 2; ++u) {
+        const float f = v[2 * c + u];
+        h[u] = __float2bfloat16_rn(f);
+        const float r1 = f - __bfloat162float(h[u]);  // exact
+        m[u] = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(m[u]);  // exact
+        l[u] = __float2bfloat16_rn(r2);
       }
-      if (i < E * (KC / 4)) {
-        const int e = i % E, c4 = (i / E) * 4;
-        wr[u] = *reinterpret_cast<const float4*>(wg + (int64_t)e * d + k0 + c4);
-      }
+      __nv_bfloat162 ph = __halves2bfloat162(h[0], h[1]);
+      __nv_bfloat162 pm = __halves2bfloat162(m[0], m[1]);
+      __nv_bfloat162 pl = __halves2bfloat162(l[0], l[1]);
+      hi[c] = *reinterpret_cast<uint32_t*>(&ph);
+      mid[c] = *reinterpret_cast<uint32_t*>(&pm);
+      lo[c] = *reinterpret_cast<uint32_t*>(&pl);
     }
-  };
-  auto store_chunk = [&](float* buf) {
-    float* Xs = buf;
-    float* Ws = buf + KC * TM;
+    *reinterpret_cast<uint2*>(planes + i * 4) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(planes + plane + i * 4) = make_uint2(mid[0], mid[1]);
+    *reinterpret_cast<uint2*>(planes + 2 * plane + i * 4) = make_uint2(lo[0], lo[1]);
+  }
+}
+
+__global__ void __launch_bounds__(GT_THREADS, 1)
+    gate_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                   const GateArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  GateCtl* ctl = reinterpret_cast<GateCtl*>(smem + (size_t)a.stages * a.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * GT_BM;
+  const int nkb = a.d / GT_BK;
+  const uint32_t plane_bytes = (uint32_t)a.e_pad * GT_BK * 2;
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tfull[b], 1);
+      mbar_init(&ctl->tempty[b], GT_SUM_WARPS);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl->tmem_base, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  // waits for work already started (copies in flight, MMAs issued) get a long
+  // budget of their own, so the CTA never frees tensor memory or exits under them
+  const uint64_t drain_budget = a.budget_ns > 2000000000ull ? a.budget_ns : 2000000000ull;
+
+  // Logits of this thread's row, in registers: 32-column groups g = 2 i + h of the
+  // accumulator (h = this warp's column half), summed over the K blocks.
+  float sum[4][32];
+  const int ngroups = a.e_pad / 32;
+  const int q = warp & 3;             // tensor-memory lane quarter of a summing warp
+  const int h = (warp - 2) >> 2;      // its column half
+  const int row = q * 32 + lane;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, lastpar = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&ctl->empty[stage], phase ^ 1, abort_flag, a.status,
+                       MOE_ERR_DEVICE_TIMEOUT, a.budget_ns))
+          break;
+        mbar_arrive_expect_tx(&ctl->full[stage], GT_A_BYTES + 3 * plane_bytes);
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const int k0 = kb * GT_BK;
+        tma_load_2d(st, &tmX, &ctl->full[stage], k0, (int32_t)m0);  // rows past T read as zero
 #pragma unroll
-    for (int u = 0; u < MAXV; ++u) {
-      const int i = tid + u * nthreads;
-      if (i < TM * (KC / 8)) {
-        const int r = i % TM, c8 = (i / TM) * 8;
-        const uint32_t w4[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          Xs[(c8 + 2 * p) * TM + r] = __uint_as_float(w4[p] << 16);
-          Xs[(c8 + 2 * p + 1) * TM + r] = __uint_as_float(w4[p] & 0xFFFF0000u);
+        for (int j = 0; j < 3; ++j)
+          tma_load_2d(st + GT_A_BYTES + j * plane_bytes, &tmW, &ctl->full[stage], k0,
+                      j * a.e_pad);
+        issued |= 1u << stage;
+        lastpar = (lastpar & ~(1u << stage)) | (phase << stage);
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1;
         }
       }
-      if (i < E * (KC / 4)) {
-        const int e = i % E, c4 = (i / E) * 4;
-        Ws[(c4 + 0) * E + e] = wr[u].x;
-        Ws[(c4 + 1) * E + e] = wr[u].y;
-        Ws[(c4 + 2) * E + e] = wr[u].z;
-        Ws[(c4 + 3) * E + e] = wr[u].w;
-      }
+      // after an abort, stages may hold copies nobody consumed: let them land
+      if (*abort_flag)
+        for (int s = 0; s < a.stages; ++s)
+          if (issued & (1u << s)) {
+            volatile int never = 0;
+            mbar_wait(&ctl->full[s], (lastpar >> s) & 1u, &never, a.status,
+                      MOE_ERR_DEVICE_TIMEOUT, drain_budget);
+          }
     }
-  };
-
-  const int nchunks = d / KC;
-  load_chunk(0);
-  store_chunk(sm);
-  __syncthreads();
-  for (int c = 0; c < nchunks; ++c) {
-    if (c + 1 < nchunks) load_chunk((c + 1) * KC);  // in flight while this chunk computes
-    const float* Xs = sm + (c & 1) * buf_floats;
-    const float* Ws = Xs + KC * TM;
-    if (active) {
-#pragma unroll 8
-      for (int kk = 0; kk < KC; ++kk) {
-        const float4 xa = *reinterpret_cast<const float4*>(Xs + kk * TM + tg * 4);
-        const float4 w0 = *reinterpret_cast<const float4*>(Ws + kk * E + eg * 8);
-        const float4 w1 = *reinterpret_cast<const float4*>(Ws + kk * E + eg * 8 + 4);
-        const float xv[4] = {xa.x, xa.y, xa.z, xa.w};
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer --
+    // K block kb accumulates, from zero, into accumulator kb % 2; the summing
+    // warps add it to their FP32 registers and hand it back.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int acc = kb & 1;
+        const uint32_t use = (uint32_t)(kb >> 1);
+        if (!mbar_wait(&ctl->tempty[acc], (use & 1u) ^ 1u, abort_flag, a.status,
+                       MOE_ERR_DEVICE_TIMEOUT, a.budget_ns))
+          break;
+        if (!mbar_wait(&ctl->full[stage], phase, abort_flag, a.status, MOE_ERR_DEVICE_TIMEOUT,
+                       a.budget_ns))
+          break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * a.e_pad);
+        const uint32_t a_base = smem_u32(smem + (size_t)stage * a.stage_bytes);
+        const uint32_t b_base = a_base + GT_A_BYTES;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int kk = 0; kk < GT_BK / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(a_base + kk * 32, 16, 1024);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+          for (int j = 0; j < 3; ++j) {
+            const uint64_t bd = smem_desc_sw128(b_base + j * plane_bytes + kk * 32, 16, 1024);
+            umma_f16(d_tmem, ad, bd, a.idesc, (kk | j) != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&ctl->empty[stage]);
+        umma_commit(&ctl->tfull[acc]);
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
+      // every MMA issued has completed before tensor memory is freed
+      umma_commit(&ctl->drain);
+      volatile int never = 0;
+      mbar_wait(&ctl->drain, 0, &never, a.status, MOE_ERR_DEVICE_TIMEOUT, drain_budget);
     }
-    if (c + 1 < nchunks) store_chunk(sm + ((c + 1) & 1) * buf_floats);
-    __syncthreads();
-  }
-
-  // logits tile -> shared memory [TM][E]
-  float* L = sm;
-  if (active) {
+  } else {
+    // ----------------------------------------------------- summing warps --
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) L[(tg * 4 + i) * E + eg * 8 + j] = acc[i][j];
-  }
-  __syncthreads();
-
-  route_tile(L, t0, TM, T, E, k, bias, topk_idx, topk_w, probs);
-}
-
-
-// Fast path (E % 32 == 0): 8 * TI tokens per CTA (32 or 64), TI tokens x 4
-// experts per thread, E * 2 threads (8 warps for E = 128).
-//  * Wg chunks [E][32] are copied into shared memory unchanged with cp.async
-//    (whole 128-byte rows: coalesced, no register staging), three chunks in
-//    flight; X chunks are widened to f32 through registers one chunk ahead.
-//  * Thread (tg, eg) owns tokens tg + 8i and experts eg + (E/4) j and reads
-//    4 consecutive K values of each as one float4.  Rows are padded to 36
-//    floats, so the 8 expert rows / 4 token rows a warp reads at once fall in
-//    distinct banks: every read is a conflict-free broadcast, 8 reads per 64
-//    FFMAs.  Small CTAs let several share an SM to hide latency.
-constexpr int RS = KC + 4;  // padded row stride (floats)
-constexpr int WSTAGES = 3;
-
-__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-               "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// TI = token rows per thread (4 or 8): the CTA covers TM = 8 * TI tokens.
-template <int TI>
-__global__ void __launch_bounds__(512)
-    gate_topk_kernel_t32(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wg,
-                         const float* __restrict__ bias, int64_t T, int d, int E, int k,
-                         int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                         float* __restrict__ probs) {
-  constexpr int TM32 = 8 * TI;             // tokens of this CTA
-  extern __shared__ float sm[];
-  float* Ws = sm;                          // [WSTAGES][E][RS]
-  float* Xs = sm + WSTAGES * E * RS;       // [2][TM32][RS]
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int EQ = E / 4;                          // expert groups
-  const int WE = E / 32;                         // warps across the experts
-  const int eg = (warp % WE) * 8 + (lane & 7);   // experts eg + EQ * j
-  const int tg = (warp / WE) * 4 + (lane >> 3);  // tokens tg + 8 * i  (tg < 8)
-  const int64_t t0 = (int64_t)blockIdx.x * TM32;
-  const int nthreads = blockDim.x;  // 2E
-
-  float acc[TI][4];
+      for (int j = 0; j < 32; ++j) sum[i][j] = 0.0f;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int acc = kb & 1;
+      const uint32_t use = (uint32_t)(kb >> 1);
+      if (!mbar_wait(&ctl->tfull[acc], use & 1u, abort_flag, a.status, MOE_ERR_DEVICE_TIMEOUT,
+                     a.budget_ns))
+        break;
+      __syncwarp();  // tcgen05.ld is warp-collective
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * a.e_pad) + ((uint32_t)(q * 32) << 16);
 #pragma unroll
-  for (int i = 0; i < TI; ++i)
+      for (int i = 0; i < 4; ++i) {
+        const int g = 2 * i + h;
+        if (g < ngroups) {
+          uint32_t r[32];
+          tmem_ld32_sync(taddr + (uint32_t)(g * 32), r);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-
-  auto issue_w = [&](int c) {  // Wg[:, 32c .. 32c+32) -> stage c % 3, 8 pieces of 16 B a row
-    float* dst = Ws + (c % WSTAGES) * E * RS;
-    for (int i = tid; i < E * 8; i += nthreads) {
-      const int e = i >> 3, q = i & 7;
-      cp_async16(dst + e * RS + q * 4, wg + (int64_t)e * d + c * KC + q * 4);
-    }
-  };
-  // X pieces of 8 bf16: TM32 * 4 of them, at most 2 per thread (2E >= 64 threads... E >= 32)
-  constexpr int XP = (TM32 * (KC / 8) + 63) / 64;
-  uint4 xr[XP];
-  auto load_x = [&](int c) {
-#pragma unroll
-    for (int u = 0; u < XP; ++u) {
-      const int i = tid + u * nthreads;
-      if (i < TM32 * (KC / 8)) {
-        const int xrow = i % TM32, xc8 = (i / TM32) * 8;
-        const int64_t t = t0 + xrow;
-        xr[u] = t < T ? *reinterpret_cast<const uint4*>(x + t * d + c * KC + xc8)
-                      : make_uint4(0, 0, 0, 0);
-      }
-    }
-  };
-  auto store_x = [&](int c) {
-#pragma unroll
-    for (int u = 0; u < XP; ++u) {
-      const int i = tid + u * nthreads;
-      if (i < TM32 * (KC / 8)) {
-        const int xrow = i % TM32, xc8 = (i / TM32) * 8;
-        float* dst = Xs + (c & 1) * TM32 * RS + xrow * RS + xc8;
-        const uint32_t w4[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
-        *reinterpret_cast<float4*>(dst) =
-            make_float4(__uint_as_float(w4[0] << 16), __uint_as_float(w4[0] & 0xFFFF0000u),
-                        __uint_as_float(w4[1] << 16), __uint_as_float(w4[1] & 0xFFFF0000u));
-        *reinterpret_cast<float4*>(dst + 4) =
-            make_float4(__uint_as_float(w4[2] << 16), __uint_as_float(w4[2] & 0xFFFF0000u),
-                        __uint_as_float(w4[3] << 16), __uint_as_float(w4[3] & 0xFFFF0000u));
-      }
-    }
-  };
-
-  const int n = d / KC;
-  issue_w(0);
-  cp_async_commit();
-  if (n > 1) issue_w(1);
-  cp_async_commit();
-  load_x(0);
-  store_x(0);
-  if (n > 1) load_x(1);
-  for (int c = 0; c < n; ++c) {
-    cp_async_wait<1>();  // this thread's copies of chunk c have landed
-    __syncthreads();     // everyone's have; chunk c - 1 is no longer being read
-    if (c + 2 < n) issue_w(c + 2);
-    cp_async_commit();   // (possibly empty: keeps the group count uniform)
-    if (c + 1 < n) store_x(c + 1);
-    if (c + 2 < n) load_x(c + 2);
-    const float* W = Ws + (c % WSTAGES) * E * RS;
-    const float* X = Xs + (c & 1) * TM32 * RS;
-#pragma unroll 2
-    for (int kk = 0; kk < KC; kk += 4) {
-      float4 xv[TI], wv[4];
-#pragma unroll
-      for (int i = 0; i < TI; ++i) xv[i] = *reinterpret_cast<const float4*>(X + (tg + 8 * i) * RS + kk);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) wv[j] = *reinterpret_cast<const float4*>(W + (eg + EQ * j) * RS + kk);
-#pragma unroll
-      for (int i = 0; i < TI; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[i][j] = fmaf(xv[i].x, wv[j].x, acc[i][j]);
-          acc[i][j] = fmaf(xv[i].y, wv[j].y, acc[i][j]);
-          acc[i][j] = fmaf(xv[i].z, wv[j].z, acc[i][j]);
-          acc[i][j] = fmaf(xv[i].w, wv[j].w, acc[i][j]);
+          for (int j = 0; j < 32; ++j) sum[i][j] += __uint_as_float(r[j]);
         }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+    }
+  }
+  __syncwarp();
+
+  tc_fence_before();
+  __syncthreads();  // every role is done: the stages are free, the abort flag is final
+  const bool aborted = *abort_flag != 0;
+  // Logits to shared memory, row stride E + 1 (odd): thread `lane` writing row
+  // lane, column c hits bank (lane + c) % 32, so these stores are conflict-free.
+  float* L = reinterpret_cast<float*>(smem);
+  const int LS = a.E + 1;
+  if (warp >= 2 && !aborted) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int g = 2 * i + h;
+      if (g < ngroups)
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (g * 32 + j < a.E) L[row * LS + g * 32 + j] = sum[i][j];
     }
   }
   __syncthreads();
-
-  float* L = sm;  // logits tile [TM32][E] (reuses the Wg stages)
-#pragma unroll
-  for (int i = 0; i < TI; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) L[(tg + 8 * i) * E + eg + EQ * j] = acc[i][j];
-  __syncthreads();
-  route_tile(L, t0, TM32, T, E, k, bias, topk_idx, topk_w, probs);
+  if (!aborted)
+    route_tile(L, LS, m0, GT_BM, a.T, a.E, a.k, a.bias, a.topk_idx, a.topk_w, a.probs);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, a.tmem_cols);
+  }
 }
 
 }  // namespace
 
 int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const float* bias,
-                     int32_t* idx, float* w, float* probs, void* stream) {
-  static int num_sms = 0;
-  if (num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (num_sms <= 0) num_sms = 148;
-  }
+                     int32_t* idx, float* w, float* probs, void* ws, void* stream) {
   const int64_t T = dm.T;
   if (T == 0) return MOE_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dm.E % 32 == 0 && dm.E <= 256) {
-    // 64 tokens per CTA (half the Wg staging per token) while that still gives
-    // every SM at least ~1.5 CTAs; 32 otherwise.
-    const bool wide = T >= (int64_t)64 * num_sms * 3 / 2;
-    const int TMv = wide ? 64 : 32;
-    const int threads = 2 * dm.E;
-    size_t smem = sizeof(float) * RS * (WSTAGES * dm.E + 2 * TMv);
-    if (smem < sizeof(float) * (size_t)TMv * dm.E) smem = sizeof(float) * (size_t)TMv * dm.E;
-    const int64_t blocks = (T + TMv - 1) / TMv;
-    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-    if (wide) {
-      if (smem > 48 * 1024 &&
-          !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel_t32<8>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-        return MOE_ERR_CUDA;
-      gate_topk_kernel_t32<8><<<(unsigned)blocks, threads, smem, st>>>(xb, wg, bias, T, dm.d, dm.E,
-                                                                      dm.k, idx, w, probs);
-    } else {
-      if (smem > 48 * 1024 &&
-          !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel_t32<4>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-        return MOE_ERR_CUDA;
-      gate_topk_kernel_t32<4><<<(unsigned)blocks, threads, smem, st>>>(xb, wg, bias, T, dm.d, dm.E,
-                                                                      dm.k, idx, w, probs);
-    }
-    return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
+  const WsLayout L = ws_layout(dm);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  __nv_bfloat16* planes = reinterpret_cast<__nv_bfloat16*>(wsb + L.gate_split);
+  const int e_pad = L.e_pad;
+
+  {
+    const int64_t n4 = (int64_t)e_pad * dm.d / 4;
+    const int threads = 256;
+    int64_t blocks = (n4 + threads - 1) / threads;
+    if (blocks > 4096) blocks = 4096;
+    split_wg_kernel<<<(unsigned)blocks, threads, 0, st>>>(wg, dm.E, e_pad, dm.d, planes);
+    if (!cuda_ok(cudaGetLastError())) return MOE_ERR_CUDA;
   }
-  // about one CTA per SM: TM tokens per CTA, a multiple of 4 in [4, 128]
-  int64_t per = (T + num_sms - 1) / num_sms;
-  int TM = (int)((per + 3) / 4 * 4);
-  if (TM < 4) TM = 4;
-  if (TM > 128) TM = 128;
-  const int NE = dm.E / 8;
-  while (TM > 4 && (TM / 4) * NE > MAX_THREADS) TM -= 4;
-  auto r32 = [](int v) { return (v + 31) / 32 * 32; };
-  int threads = r32((TM / 4) * NE);
-  // every thread's share of a chunk must fit its MAXV prefetch registers
-  while (threads < MAX_THREADS &&
-         (TM * (KC / 8) > MAXV * threads || dm.E * (KC / 4) > MAXV * threads))
-    threads += 32;
-  if (TM * (KC / 8) > MAXV * threads || dm.E * (KC / 4) > MAXV * threads)
+
+  GateArgs a{};
+  a.status = reinterpret_cast<int*>(ws);
+  a.bias = bias;
+  a.topk_idx = idx;
+  a.topk_w = w;
+  a.probs = probs;
+  a.T = T;
+  a.d = dm.d;
+  a.E = dm.E;
+  a.e_pad = e_pad;
+  a.k = dm.k;
+  a.stage_bytes = (uint32_t)(GT_A_BYTES + 3 * e_pad * GT_BK * 2);  // a multiple of 1024
+  const size_t fixed = 1024 /* alignment slack */ + sizeof(GateCtl);
+  int stages = (int)((GT_MAX_SMEM - fixed) / a.stage_bytes);
+  if (stages > GT_MAX_STAGES) stages = GT_MAX_STAGES;
+  if (stages < 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+  a.stages = stages;
+  // the logits tile [128][E + 1] f32 reuses the stage buffers
+  if ((size_t)GT_BM * (dm.E + 1) * sizeof(float) > (size_t)stages * a.stage_bytes)
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  const size_t stage_bytes = 2 * sizeof(float) * KC * (TM + dm.E);
-  const size_t logit_bytes = sizeof(float) * (size_t)TM * dm.E;
-  const size_t smem = stage_bytes > logit_bytes ? stage_bytes : logit_bytes;
-  if (smem > 48 * 1024 &&
-      !cuda_ok(cudaFuncSetAttribute(gate_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem)))
+  uint32_t cols = 32;  // two accumulators of e_pad columns
+  while (cols < (uint32_t)(2 * e_pad)) cols <<= 1;
+  a.tmem_cols = cols;
+  a.idesc = idesc_bf16_f32(GT_BM, e_pad, false, false);
+  a.budget_ns = wait_budget_ns();
+
+  CUtensorMap mx{}, mw{};
+  if (!make_map_bf16(&mx, x, T, dm.d, GT_BM) ||
+      !make_map_bf16(&mw, planes, (int64_t)3 * e_pad, dm.d, e_pad))
     return MOE_ERR_CUDA;
-  const int64_t blocks = (T + TM - 1) / TM;
-  gate_topk_kernel<<<(unsigned)blocks, threads, smem, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(x), wg, bias, T, dm.d, dm.E, dm.k, TM, idx, w,
-      probs);
+  const size_t smem = fixed + (size_t)stages * a.stage_bytes;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (!cuda_ok(cudaFuncSetAttribute(gate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      GT_MAX_SMEM)))
+      return MOE_ERR_CUDA;
+    attr_set = true;
+  }
+  const int64_t blocks = (T + GT_BM - 1) / GT_BM;
+  gate_tc_kernel<<<(unsigned)blocks, GT_THREADS, smem, st>>>(mx, mw, a);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 

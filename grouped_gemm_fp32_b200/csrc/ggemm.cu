@@ -558,43 +558,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// ------------------------------------------------------------------ host side --
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// Row-major bf16 matrix [rows, cols] (cols contiguous); box = 64 elements (128
-// bytes) of a row x box_rows rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc || base == nullptr) return false;
-  const int esz = 2;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
-  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                   const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int MODE>
 int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
                 const CUtensorMap& b1, const CUtensorMap& c, const GemmArgs& args,
@@ -628,6 +591,45 @@ int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
+}  // namespace
+
+// ------------------------------------------------------------------ host side --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] (cols contiguous); box = 64 elements (128
+// bytes) of a row x box_rows rows, 128-byte swizzle.
+bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc || base == nullptr) return false;
+  const int esz = 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 uint64_t wait_budget_ns() {
   static uint64_t v = [] {
     const char* s = getenv("MOE_WAIT_BUDGET_NS");
@@ -636,7 +638,6 @@ uint64_t wait_budget_ns() {
   return v;
 }
 
-}  // namespace
 
 int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
                         const GemmOperands& ops, void* stream) {
@@ -679,9 +680,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.ld_out = I;
       a.ld_out2 = 2 * I;
       a.idesc = idesc_bf16_f32(PM, 2 * hn, false, false);
-      ok &= make_map(&m0, ops.a0, Rr, d, BM);
-      if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, BM); else same(m1, m0);
-      ok &= make_map(&n0, ops.b0, (int64_t)G * 2 * I, d, hn);
+      ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
+      if (dm.S > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
+      ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, hn);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, a, st);
@@ -693,9 +694,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.b_group_rows = d;
       a.ld_out = d;
       a.idesc = idesc_bf16_f32(PM, 256, false, false);
-      ok &= make_map(&m0, ops.a0, Rt, I, BM);
+      ok &= make_map_bf16(&m0, ops.a0, Rt, I, BM);
       same(m1, m0);
-      ok &= make_map(&n0, ops.b0, (int64_t)G * d, I, 128);
+      ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 128);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, a, st);
@@ -709,11 +710,11 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.ld_aux = 2 * I;
       a.idesc = idesc_bf16_f32(PM, 256, false, true);
       a.idesc_narrow = idesc_bf16_f32(PM, 128, false, true);
-      ok &= make_map(&m0, ops.a0, Rr, d, BM);
-      if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, BM); else same(m1, m0);
-      ok &= make_map(&n0, ops.b0, (int64_t)G * d, I, 64);
+      ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
+      if (dm.S > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
+      ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 64);
       same(n1, n0);
-      ok &= make_map(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
+      ok &= make_map_bf16(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
       if (!ok) return MOE_ERR_CUDA;
       return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, a, st);
     }
@@ -725,9 +726,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.ld_out = d;
       a.idesc = idesc_bf16_f32(PM, 256, false, true);
       a.idesc_narrow = idesc_bf16_f32(PM, 128, false, true);
-      ok &= make_map(&m0, ops.a0, Rt, 2 * I, BM);
+      ok &= make_map_bf16(&m0, ops.a0, Rt, 2 * I, BM);
       same(m1, m0);
-      ok &= make_map(&n0, ops.b0, (int64_t)G * 2 * I, d, 64);
+      ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, a, st);
@@ -739,9 +740,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.NT = (I + 255) / 256;
       a.idesc = idesc_bf16_f32(PM, 256, true, true);
       a.idesc_narrow = idesc_bf16_f32(PM, 128, true, true);
-      ok &= make_map(&m0, ops.a0, Rr, d, 64);
-      if (dm.S > 0) ok &= make_map(&m1, ops.a1, T, d, 64); else same(m1, m0);
-      ok &= make_map(&n0, ops.b0, Rt, I, 64);
+      ok &= make_map_bf16(&m0, ops.a0, Rr, d, 64);
+      if (dm.S > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, 64); else same(m1, m0);
+      ok &= make_map_bf16(&n0, ops.b0, Rt, I, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, a, st);
@@ -753,10 +754,10 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.NT = (d + 255) / 256;
       a.idesc = idesc_bf16_f32(PM, 256, true, true);
       a.idesc_narrow = idesc_bf16_f32(PM, 128, true, true);
-      ok &= make_map(&m0, ops.a0, Rt, 2 * I, 64);
+      ok &= make_map_bf16(&m0, ops.a0, Rt, 2 * I, 64);
       same(m1, m0);
-      ok &= make_map(&n0, ops.b0, Rr, d, 64);
-      if (dm.S > 0) ok &= make_map(&n1, ops.b1, T, d, 64); else same(n1, n0);
+      ok &= make_map_bf16(&n0, ops.b0, Rr, d, 64);
+      if (dm.S > 0) ok &= make_map_bf16(&n1, ops.b1, T, d, 64); else same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, a, st);
     }

@@ -57,16 +57,18 @@ int64_t moe_rows_routed(const moe_dims* dims) { return dims_ok(dims) ? rows_rout
 int64_t moe_rows_total(const moe_dims* dims) { return dims_ok(dims) ? rows_total(*dims) : -1; }
 
 size_t moe_workspace_size(const moe_dims* dims) {
-  return dims_ok(dims) ? ws_layout(*dims).bytes : 0;
+  return dims_ok(dims) ? ws_layout(*dims).total : 0;
 }
 
 int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const float* bias,
-                  int32_t* topk_idx, float* topk_w, float* probs, void* stream) {
+                  int32_t* topk_idx, float* topk_w, float* probs, void* ws, size_t ws_bytes,
+                  void* stream) {
   int rc = check_shape(dims, false);
   if (rc) return rc;
   if (dims->E % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!ws || ws_bytes < ws_layout(*dims).total) return MOE_ERR_INVALID_ARG;
   if (dims->T > 0 && (!x || !wg || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
-  return launch_gate_topk(*dims, x, wg, bias, topk_idx, topk_w, probs, stream);
+  return launch_gate_topk(*dims, x, wg, bias, topk_idx, topk_w, probs, ws, stream);
 }
 
 int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void* x,

@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "moe.h"  // include/ is on the include path
@@ -27,13 +28,18 @@ constexpr int kChunk = 1024;      // routed assignments per histogram chunk
 constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] tiles total,
                                   // [3] routing valid, [4] bad expert id seen
 
+// Layer workspace: the routing tables first (`bytes` of them), then the
+// gate's split weights.
 struct WsLayout {
   size_t groups;        // GroupRec[G]
   size_t mtile_prefix;  // int32[G + 1]  prefix of ceil(rows_pad / 256) (pair tiles)
   size_t dw_order;      // int32[G]      groups by padded rows, largest first
   size_t chunk_hist;    // int32[nchunks * E]
-  size_t bytes;
+  size_t bytes;         // end of the routing tables
+  size_t gate_split;    // bf16[3][e_pad][d]  the gate weights as hi, mid, lo planes
+  size_t total;         // whole workspace
   int nchunks;
+  int e_pad;            // E rounded up to a multiple of 32
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -54,6 +60,9 @@ inline WsLayout ws_layout(const moe_dims& dm) {
   L.chunk_hist = off = align_up(off, 16);
   off += sizeof(int32_t) * (size_t)L.nchunks * dm.E;
   L.bytes = align_up(off, 256);
+  L.e_pad = (dm.E + 31) / 32 * 32;
+  L.gate_split = align_up(L.bytes, 1024);
+  L.total = align_up(L.gate_split + (size_t)3 * L.e_pad * dm.d * 2, 256);
   return L;
 }
 
@@ -64,7 +73,7 @@ inline int64_t rows_total(const moe_dims& dm) { return rows_routed(dm) + (int64_
 
 // Launch helpers implemented in the .cu files (all return a moe_status).
 int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const float* bias,
-                     int32_t* idx, float* w, float* probs, void* stream);
+                     int32_t* idx, float* w, float* probs, void* ws, void* stream);
 int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_t* counts,
                    int32_t* offsets, int32_t* sorted_ids, int32_t* row_of, void* x_perm, void* ws,
                    void* stream);
@@ -88,6 +97,13 @@ struct GemmOperands {
   const void* aux;  // DX2: saved pre-activations
   int accumulate;
 };
+
+// Tensor map of a row-major bf16 matrix [rows, cols] (cols contiguous): box of
+// 64 columns (128 bytes) x box_rows rows, 128-byte swizzle, zero fill past the edges.
+bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows);
+
+// Wall-time budget of one bounded wait inside a kernel (MOE_WAIT_BUDGET_NS, default 4 s).
+uint64_t wait_budget_ns();
 
 int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
                         const GemmOperands& ops, void* stream);

@@ -67,7 +67,7 @@ def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
     choice, e.g. to run the experts on a routing decided elsewhere."""
     dm = b.dims
     if routing is None:
-        L.moe_gate_topk(dm, x, wg, bias, b.topk_idx, b.topk_w, None, stream)
+        L.moe_gate_topk(dm, x, wg, bias, b.topk_idx, b.topk_w, None, b.ws, stream)
     else:
         b.topk_idx.copy_(routing[0])
         b.topk_w.copy_(routing[1])

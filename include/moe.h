@@ -77,8 +77,12 @@ int64_t moe_rows_routed(const moe_dims* dims);
 int64_t moe_rows_total(const moe_dims* dims);
 
 /* Bytes of device workspace that the calls taking `ws` need.  One workspace
- * serves a whole layer: moe_permute_align (or grouped_gemm_set_groups) writes
- * the group table into it, and the GEMM and combine-backward calls read it. */
+ * serves a whole layer.  It starts with the routing tables (the status word,
+ * the group table, tile prefixes, per-chunk histograms): moe_permute_align (or
+ * grouped_gemm_set_groups) writes them, the GEMM and combine-backward calls
+ * read them.  After them, 1024-byte aligned, moe_gate_topk keeps the gate
+ * weights split into three bf16 planes, 3 * E_pad * d * 2 bytes with E_pad = E
+ * rounded up to a multiple of 32. */
 size_t moe_workspace_size(const moe_dims* dims);
 
 /* Gate and aux-loss-free top-k routing.
@@ -94,9 +98,18 @@ size_t moe_workspace_size(const moe_dims* dims);
  *                               scores to the lower expert index
  *   topk_w   [T, k] f32         p[e_j] / sum_j p[e_j] (unbiased, renormalised)
  *   probs    [T, E] f32         softmax affinities (may be NULL)
- * logits are accumulated in FP32; p uses expf. */
+ *   ws / ws_bytes               workspace of moe_workspace_size(dims) bytes: the
+ *                               call rewrites its gate-weight planes and may set
+ *                               its status word; the routing tables are untouched
+ * The logits are FP32 sums of exact FP32 products: each FP32 weight is split
+ * exactly into three bf16 terms (hi + mid + lo, exact to below 2^-24 |w|),
+ * x is bf16, and the tensor cores accumulate the products in FP32.  p uses
+ * expf.  Requires E % 8 == 0, E <= 256, d % 64 == 0.  A bounded wait that runs
+ * out on the device sets MOE_ERR_DEVICE_TIMEOUT in the status word and leaves
+ * the outputs of the affected tokens unwritten. */
 int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const float* bias,
-                  int32_t* topk_idx, float* topk_w, float* probs, void* stream);
+                  int32_t* topk_idx, float* topk_w, float* probs, void* ws, size_t ws_bytes,
+                  void* stream);
 
 /* Permutation into per-expert segments padded to P rows, plus the group table.
  * Passage: dots.llm1 Technical Report, §3.2 "Efficient implementation of
@@ -128,9 +141,10 @@ int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void*
  * a host framework whose allocator owns every device buffer, foreign-function
  * callers that pass only inputs and outputs, paths where cudaMalloc is not
  * allowed.  It calls no cudaMalloc or cudaFree.
- *   - Limit: the call's scratch, moe_workspace_size(dims), must be at most
- *     1 MiB (about 2 million routed assignments at E = 128); larger shapes
- *     return MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - Limit: the call's scratch, the routing-table part of the workspace
+ *     (moe_workspace_size(dims) without the gate's weight planes), must be at
+ *     most 1 MiB (about 2 million routed assignments at E = 128); larger
+ *     shapes return MOE_ERR_UNSUPPORTED_SHAPE.
  *   - The array is shared by every call in the process and keeps the last
  *     call's contents; each call clears what must start at zero.  Calls whose
  *     executions overlap on the GPU (other streams, other threads) race on it

@@ -83,12 +83,14 @@ def test_validation_rejects_before_any_launch(lib):
     # backward needs P % 64 == 0
     assert L.grouped_gemm_bwd_dx(ctypes.byref(ok), p, 1, p, p, p, p, p, nul) == -2
     # null pointers / bad enum / small workspace
-    assert L.moe_gate_topk(ctypes.byref(ok), nul, p, p, p, p, nul, nul) == -1
+    assert L.moe_gate_topk(ctypes.byref(ok), nul, p, p, p, p, nul, p, 1 << 30, nul) == -1
+    assert L.moe_gate_topk(ctypes.byref(ok), p, p, p, p, p, nul, p, 8, nul) == -1  # small ws
+    assert L.moe_gate_topk(ctypes.byref(ok), p, p, p, p, p, nul, nul, 1 << 30, nul) == -1
     assert L.moe_permute_align(ctypes.byref(ok), p, p, p, p, p, p, p, p, 8, nul) == -1
     ok64 = lib.MoeDims.of(64, 128, 8, 2, 1, 64, 64)
     assert L.grouped_gemm_bwd_dx(ctypes.byref(ok64), p, 7, p, p, p, p, p, nul) == -1
     assert L.grouped_gemm_bwd_dw(ctypes.byref(ok64), p, 2, p, p, p, p, p, 5, nul) == -1
-    assert L.moe_gate_topk(None, p, p, p, p, p, nul, nul) == -1
+    assert L.moe_gate_topk(None, p, p, p, p, p, nul, p, 1 << 30, nul) == -1
 
 
 def test_status_strings(lib):

@@ -22,7 +22,8 @@ def _gate(dm, x, wg, bias, with_probs=True):
     idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
     w = torch.empty(T, k, dtype=torch.float32, device="cuda")
     probs = torch.empty(T, E, dtype=torch.float32, device="cuda") if with_probs else None
-    moe.moe_gate_topk(dm, x, wg, bias, idx, w, probs)
+    ws = torch.zeros(moe.moe_workspace_size(dm), dtype=torch.uint8, device="cuda")
+    moe.moe_gate_topk(dm, x, wg, bias, idx, w, probs, ws)
     torch.cuda.synchronize()
     return idx, w, probs
 
@@ -54,6 +55,26 @@ def test_gate_ties_go_to_lower_index():
     assert np.array_equal(host(idx), oidx)
     assert list(oidx[0]) == [1, 2, 4]
     np.testing.assert_allclose(host(w), ow, atol=1e-7)
+
+
+def test_gate_resolves_fp32_weight_bits():
+    # Gate weights 1 + e * 2^-22 differ only below bf16's 8-bit significand; with x = +1, -1,
+    # +1, ... the logits are exactly e * 2^-11 (d = 4096), so an FP32 gate ranks the experts
+    # 7, 6, 5 (score gaps ~6e-5, above the margin exemption) where a gate that rounded Wg to
+    # bf16 would see equal logits and pick 0, 1, 2.  (FP32 gate: §Architecture "Mixture of
+    # Experts layer".)
+    T, d, E, k = 256, 4096, 8, 3
+    sign = np.where(np.arange(d) % 2 == 0, 1.0, -1.0).astype(np.float32)
+    x = np.tile((sign.view(np.uint32) >> 16).astype(np.uint16), (T, 1))
+    wg = np.ones((E, d), np.float32)
+    wg[:, 0::2] += (np.arange(E, dtype=np.float32) * np.float32(2.0 ** -22))[:, None]
+    dm = moe.MoeDims.of(T, d, E, k, 0, 64, 16)
+    idx, w, probs = _gate(dm, dev(x, True), dev(wg), None)
+    p, oidx, ow, margin = oracle.route(oracle.gate_logits(x, wg), np.zeros(E, np.float32), k)
+    assert oidx[0].tolist() == [7, 6, 5] and margin.min() > MARGIN_EXEMPT
+    assert np.array_equal(host(idx), oidx)
+    np.testing.assert_allclose(host(w), ow, atol=1e-6)
+    np.testing.assert_allclose(host(probs), p, atol=1e-7)
 
 
 def test_gate_bias_none_equals_zero_bias():

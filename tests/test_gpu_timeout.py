@@ -1,5 +1,5 @@
-"""Failure detection without a GPU fault: every wait inside the grouped GEMM is
-bounded.  With a wait budget of 1 ns the kernel's roles give up, record
+"""Failure detection without a GPU fault: every wait inside the grouped GEMM and
+the gate is bounded.  With a wait budget of 1 ns the kernel's roles give up, record
 MOE_ERR_DEVICE_TIMEOUT in the workspace status word, drain the copies and MMAs
 they already started and return; the host reads the status and the CUDA
 context stays usable.  Runs in a child process because the budget
@@ -34,9 +34,19 @@ y = torch.empty(E * rows, d, dtype=torch.bfloat16, device="cuda")
 moe.grouped_gemm_fwd(dm, ws, x, None, w1, w2, h, None, y)
 torch.cuda.synchronize()
 st = moe.moe_get_device_status(ws)
-print("status", st)
+print("gemm status", st)
 # the context still works: the status was cleared and a plain op runs
 assert moe.moe_get_device_status(ws) == 0
+# the gate's waits are bounded the same way
+dg = moe.MoeDims.of(1024, 4096, 128, 6, 0, 64, 128)
+wsg = torch.zeros(moe.moe_workspace_size(dg), dtype=torch.uint8, device="cuda")
+xg = bf(synth.normal_bf16(2, 1, (1024, 4096), 1.0))
+wg = torch.from_numpy(synth.normal_f32(2, 2, (128, 4096), 0.02)).cuda()
+idx = torch.empty(1024, 6, dtype=torch.int32, device="cuda")
+wt = torch.empty(1024, 6, dtype=torch.float32, device="cuda")
+moe.moe_gate_topk(dg, xg, wg, None, idx, wt, None, wsg)
+torch.cuda.synchronize()
+print("gate status", moe.moe_get_device_status(wsg))
 z = torch.arange(1000, device="cuda", dtype=torch.float32).sum().item()
 print("context ok", z == 499500.0)
 '''
@@ -48,5 +58,6 @@ def test_bounded_waits_report_timeout_and_keep_context():
     p = subprocess.run([sys.executable, "-c", f"ROOT = {ROOT!r}\n" + CHILD], env=env,
                        capture_output=True, text=True, timeout=300)
     assert p.returncode == 0, p.stdout + p.stderr
-    assert "status -4" in p.stdout, p.stdout
+    assert "gemm status -4" in p.stdout, p.stdout
+    assert "gate status -4" in p.stdout, p.stdout
     assert "context ok True" in p.stdout, p.stdout

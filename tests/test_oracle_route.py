@@ -161,3 +161,26 @@ def test_hand_derived_routing_fixture(case):
         assert math.isinf(margin[0])
     else:
         assert abs(margin[0] - m) < 1e-7  # bias is stored in f32
+
+
+def _fp32_bits_case(T=4, d=4096, E=8):
+    """x = +1, -1, +1, ... (bf16) and Wg = 1 + e * 2^-22 on the even columns, 1 on the odd
+    ones: the weights differ only below bf16's 8-bit significand."""
+    sign = np.where(np.arange(d) % 2 == 0, 1.0, -1.0).astype(np.float32)
+    x = np.tile((sign.view(np.uint32) >> 16).astype(np.uint16), (T, 1))
+    wg = np.ones((E, d), np.float32)
+    wg[:, 0::2] += (np.arange(E, dtype=np.float32) * np.float32(2.0 ** -22))[:, None]
+    return x, wg
+
+
+def test_gate_logits_keep_fp32_weight_bits():
+    # closed form: logit_e = (d / 2) * e * 2^-22 = e * 2^-11 exactly (FP32 gate of the pages,
+    # §Architecture "Mixture of Experts layer"); a bf16 copy of Wg would make all logits 0
+    x, wg = _fp32_bits_case()
+    logits = oracle.gate_logits(x, wg)
+    assert np.array_equal(logits, np.tile(np.arange(8) * 2.0 ** -11, (4, 1)))
+    wg_bf16 = (wg.view(np.uint32) + 0x8000 & 0xFFFF0000).view(np.float32)
+    assert np.all(oracle.gate_logits(x, wg_bf16) == 0.0)
+    _, idx, _, margin = oracle.route(logits, np.zeros(8, np.float32), 3)
+    assert idx.tolist() == [[7, 6, 5]] * 4
+    assert np.all(margin > 5e-5)
