@@ -52,6 +52,7 @@ constexpr int EPI_WARPS = 8;            // two per tensor-memory lane quarter
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;     // two 256-column FP32 accumulators
 constexpr int MAX_GROUPS = 264;  // E <= 256 routed + S <= 8 shared
+constexpr int M_BAND = 8;        // m-tiles per band of the FWD / DX tile order
 
 struct GemmArgs {
   int* status;
@@ -134,7 +135,13 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     const int p0 = __ldg(pre + lo);
     const int mt_g = __ldg(pre + lo + 1) - p0;
     const int local = tile - p0 * a.NT;
-    const int nt = local / mt_g, mt = local - nt * mt_g;
+    // n-tile-major inside bands of up to M_BAND m-tiles: the pairs running at one
+    // time share a B slice, and a band's A rows stay in L2 across all n-tiles
+    // (a shared group's 64 m-tiles would otherwise stream all of A once per n-tile)
+    const int b = local / (M_BAND * a.NT);
+    const int r = local - b * M_BAND * a.NT;
+    const int bm = min(M_BAND, mt_g - b * M_BAND);
+    const int nt = r / bm, mt = b * M_BAND + (r - nt * bm);
     t.m0 = mt * PM;
     t.n0 = nt * (MODE == MODE_FWD1 ? a.hn : 256);
     t.nkb = a.K / BK;
