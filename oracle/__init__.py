@@ -62,6 +62,8 @@ def _load():
         lib.oracle_round_bf16.argtypes = [dbl]
         lib.oracle_gate_logits.argtypes = [vp, vp, i64, i32, i32, vp]
         lib.oracle_route.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp]
+        lib.oracle_router_bwd.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp]
+        lib.oracle_bias_update.argtypes = [vp, i64, i32, i32, vp, ctypes.c_float, vp]
         lib.oracle_permute.restype = i64
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, i32, i64, vp, vp, vp, vp]
         for sfx in ("_bf16", "_f64"):
@@ -124,6 +126,29 @@ def route(logits: np.ndarray, bias: np.ndarray, k: int):
     margin = np.empty((T,), dtype=np.float64)
     _load().oracle_route(_p(logits), _p(bias), T, E, k, _p(probs), _p(idx), _p(w), _p(margin))
     return probs, idx, w, margin
+
+
+def router_bwd(x: np.ndarray, wg: np.ndarray, idx: np.ndarray, dw: np.ndarray):
+    """Gradient of the combine weights through the renormalisation and the softmax:
+    (dlogits [T,E], dx [T,d], dwg [E,d]), all FP64.  x: bf16 bits [T,d]; wg: f32 [E,d];
+    idx [T,k] the chosen experts; dw [T,k] = dL/dw."""
+    x, wg, idx, dw = _c(x, np.uint16), _c(wg, np.float32), _c(idx, np.int32), _c(dw, np.float64)
+    T, d = x.shape
+    E = wg.shape[0]
+    k = idx.shape[1]
+    dl = np.empty((T, E)); dx = np.empty((T, d)); dwg = np.empty((E, d))
+    _load().oracle_router_bwd(_p(x), _p(wg), _p(idx), _p(dw), T, d, E, k, _p(dl), _p(dx),
+                              _p(dwg))
+    return dl, dx, dwg
+
+
+def bias_update(idx: np.ndarray, E: int, bias: np.ndarray, gamma: float) -> np.ndarray:
+    """One aux-loss-free bias step: bias_e + gamma * sign(T k / E - load_e), FP64."""
+    idx, bias = _c(idx, np.int32), _c(bias, np.float32)
+    T, k = idx.shape
+    out = np.empty(E)
+    _load().oracle_bias_update(_p(idx), T, E, k, _p(bias), float(gamma), _p(out))
+    return out
 
 
 def permute(idx: np.ndarray, E: int, P: int, rows_cap: int):

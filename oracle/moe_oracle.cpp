@@ -196,6 +196,87 @@ void oracle_route(const double* logits, const float* bias, int64_t T, int E, int
   }
 }
 
+// Router backward: the gradient of the combine weights w[t, j] through the
+// renormalisation over the chosen set C and the softmax, then into the gate's
+// input and weights.  The selection (made on p + bias) is piecewise constant and
+// carries no gradient; the bias gets none.  With Z = sum_{j in C} p_j:
+//   w_j = p_j / Z        =>  dp_i = (dw_i - sum_j dw_j w_j) / Z   (i in C; 0 elsewhere)
+//   p = softmax(logit)   =>  dlogit_e = p_e (dp_e - sum_i p_i dp_i)
+//   logit = X Wg^T       =>  dX = dlogit Wg,   dWg = dlogit^T X
+// Logits and p are recomputed in FP64 from x and wg.  Any of the outputs may be null.
+void oracle_router_bwd(const uint16_t* x, const float* wg, const int32_t* idx, const double* dw,
+                       int64_t T, int d, int E, int k, double* dlogits, double* dx,
+                       double* dwg) {
+  std::vector<double> dl((size_t)T * E);
+#pragma omp parallel
+  {
+    std::vector<double> xt(d), p(E), dp(E);
+#pragma omp for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+      for (int c = 0; c < d; ++c) xt[c] = bf(x[t * d + c]);
+      double m = -INFINITY;
+      for (int e = 0; e < E; ++e) {
+        const float* w = wg + (size_t)e * d;
+        double s = 0.0;
+        for (int c = 0; c < d; ++c) s += xt[c] * (double)w[c];
+        p[e] = s;
+        m = std::max(m, s);
+      }
+      double z = 0.0;
+      for (int e = 0; e < E; ++e) {
+        p[e] = std::exp(p[e] - m);
+        z += p[e];
+      }
+      for (int e = 0; e < E; ++e) {
+        p[e] /= z;
+        dp[e] = 0.0;
+      }
+      double zc = 0.0, dot = 0.0;
+      for (int j = 0; j < k; ++j) zc += p[idx[t * k + j]];
+      for (int j = 0; j < k; ++j) dot += dw[t * k + j] * (p[idx[t * k + j]] / zc);
+      for (int j = 0; j < k; ++j) dp[idx[t * k + j]] = (dw[t * k + j] - dot) / zc;
+      double pdp = 0.0;
+      for (int e = 0; e < E; ++e) pdp += p[e] * dp[e];
+      for (int e = 0; e < E; ++e) dl[(size_t)t * E + e] = p[e] * (dp[e] - pdp);
+    }
+  }
+  if (dlogits) std::copy(dl.begin(), dl.end(), dlogits);
+  if (dx) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+      for (int c = 0; c < d; ++c) {
+        double s = 0.0;
+        for (int e = 0; e < E; ++e) s += dl[(size_t)t * E + e] * (double)wg[(size_t)e * d + c];
+        dx[t * d + c] = s;
+      }
+  }
+  if (dwg) {
+#pragma omp parallel for schedule(static)
+    for (int e = 0; e < E; ++e)
+      for (int c = 0; c < d; ++c) {
+        double s = 0.0;
+        for (int64_t t = 0; t < T; ++t) s += dl[(size_t)t * E + e] * bf(x[t * d + c]);
+        dwg[(size_t)e * d + c] = s;
+      }
+  }
+}
+
+// Aux-loss-free bias update, one step (the pages say the bias is adjusted during
+// training to keep the expert loads balanced; this is the plainest rule of that
+// kind): load_e = number of (token, pick) pairs routed to e in the batch, mean =
+// T k / E, bias_e += gamma * sign(mean - load_e) with sign(0) = 0.  The sum of two
+// f32 values is exact in double.
+void oracle_bias_update(const int32_t* idx, int64_t T, int E, int k, const float* bias,
+                        float gamma, double* out) {
+  std::vector<int64_t> load(E, 0);
+  for (int64_t i = 0; i < T * k; ++i) load[idx[i]] += 1;
+  for (int e = 0; e < E; ++e) {
+    const double diff = (double)T * k - (double)load[e] * E;  // E * (mean - load_e)
+    const double sgn = diff > 0 ? 1.0 : diff < 0 ? -1.0 : 0.0;
+    out[e] = (double)bias[e] + (double)gamma * sgn;
+  }
+}
+
 // Permutation into padded per-expert segments.
 //   c_e = #{(t, j) : idx[t, j] = e};  off_0 = 0, off_{e+1} = off_e + roundup(c_e, P)
 //   segment e lists its tokens in ascending order; pad rows hold -1.
