@@ -7,7 +7,8 @@ One step = one pass of the whole hot path over one batch:
   train (default): T=16384 tokens, d=4096, 128 routed experts top-6 + 2 shared,
                    I=1408, pad block 128; forward (gate, top-k, permute, grouped
                    SwiGLU GEMMs, combine) + backward (combine bwd, dX and dW
-                   grouped GEMMs, SwiGLU bwd, un-permute-sum).
+                   grouped GEMMs, SwiGLU bwd, un-permute-sum, router backward
+                   into dX and dWg) + the aux-loss-free bias step.
   layer:           T=8192, same layer, forward only.
   gemm_only:       the grouped GEMM forward alone (16 groups x 512 rows, d=4096,
                    I=1408): a small case for profiles, not the headline.
@@ -36,6 +37,11 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+
+# Update speed of the aux-loss-free bias step in the train step (the pages give no
+# value; 1e-3 per step is an illustrative choice, applied to a copy of the bias so
+# every timed step routes the same synthetic batch the same way).
+GAMMA = 1e-3
 
 METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of B200 BF16 peak), 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -327,13 +333,14 @@ def run_ours(args):
         if ev is None:
             layer.forward(b, xx, wg, bias, w1, w2, stream=s)
             if train:
-                layer.backward(b, xx, gg, w1, w2, stream=s)
+                layer.backward(b, xx, gg, w1, w2, stream=s, wg=wg, gamma=GAMMA, bias=bias)
             return
         # instrumented: events around each C-ABI call
         L = moe
         rec = lambda k: ev[k].append(torch.cuda.Event(enable_timing=True)) or ev[k][-1].record(s)
         rec("t0")
-        L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, b.ws, s)
+        L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, b.probs if train else None,
+                        b.ws, s)
         rec("gate")
         L.moe_permute_align(dims, b.topk_idx, xx, b.counts, b.offsets, b.sorted_ids, b.row_of,
                             b.x_perm, b.ws, s)
@@ -355,6 +362,11 @@ def run_ours(args):
             rec("dw1")
             L.moe_combine(dims, b.dxp, b.row_of, None, b.dx, s)
             rec("unpermute")
+            L.moe_router_bwd(dims, xx, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb, None, b.dx,
+                             b.dwg, 0, b.ws, s)
+            rec("router_bwd")
+            L.moe_bias_update(dims, b.counts, GAMMA, bias, b.bias_next, s)
+            rec("bias_step")
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -387,7 +399,8 @@ def run_ours(args):
     # ---- per-call breakdown (separate instrumented pass; not the headline)
     names = (["t0", "gate"] if gate_only else
              ["t0", "fwd"] if gemm_only else ["t0", "gate", "permute", "fwd", "combine"]) + (
-        ["combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute"] if train else [])
+        ["combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute", "router_bwd", "bias_step"]
+        if train else [])
     ev = {n: [] for n in names}
     nprof = max(3, min(args.steps, 20))
     with torch.cuda.stream(stream):
@@ -427,7 +440,8 @@ def run_ours(args):
         e2e_streams = [stream]
         e2e_note = "inputs H2D and results D2H every step, serialised with compute"
     else:
-        pipe = layer.HostPipeline(dims, w1, w2, wg, bias, train, device=dev)
+        pipe = layer.HostPipeline(dims, w1, w2, wg, bias, train, device=dev,
+                                  gamma=GAMMA if train else None)
         hx = [pinned(inp["x"])]
         hd = [pinned(inp["dout"])] if train else [None]
         ho = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -461,8 +475,11 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after timing: {moe.moe_status_string(status)}")
 
-    launches_per_step = (1 if gate_only else 2 if gemm_only else
-                         1 + 5 + 2 + 1 + ((2 + 4 + 1) if train else 0))
+    # kernels per step: gate 2 (weight split, gate), permute 5, forward GEMMs 2, combine 1;
+    # train adds combine backward 2, backward GEMMs 4, un-permute 1, router backward 5
+    # (weight split, dlogits, dX GEMM, dWg GEMM, split-K sum), bias step 1
+    launches_per_step = (2 if gate_only else 2 if gemm_only else
+                         2 + 5 + 2 + 1 + ((2 + 4 + 1 + 5 + 1) if train else 0))
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,

@@ -17,7 +17,8 @@ MOE_GEMM1, MOE_GEMM2 = 1, 2
 EXPORTS = (
     "moe_rows_routed", "moe_rows_total", "moe_workspace_size", "moe_gate_topk",
     "moe_permute_align", "moe_permute_align_static", "grouped_gemm_set_groups",
-    "grouped_gemm_fwd", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd", "moe_get_device_status",
+    "grouped_gemm_fwd", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw", "moe_combine",
+    "moe_combine_bwd", "moe_router_bwd", "moe_bias_update", "moe_get_device_status",
     "moe_status_string", "moe_last_cuda_error",
 )
 
@@ -72,6 +73,8 @@ def load():
         "grouped_gemm_bwd_dx": (i32, [D, vp, i32, vp, vp, vp, vp, vp, vp]),
         "grouped_gemm_bwd_dw": (i32, [D, vp, i32, vp, vp, vp, vp, vp, i32, vp]),
         "moe_combine": (i32, [D, vp, vp, vp, vp, vp]),
+        "moe_router_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+        "moe_bias_update": (i32, [D, vp, ctypes.c_float, vp, vp, vp]),
         "moe_combine_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_get_device_status": (i32, [vp, vp, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
@@ -182,6 +185,19 @@ def moe_combine(dims, y, row_of, topk_w, out, stream=None):
 def moe_combine_bwd(dims, ws, dout, y, row_of, topk_w, dy_routed, dw, stream=None):
     _ck(load().moe_combine_bwd(ctypes.byref(dims), _p(ws), _p(dout), _p(y), _p(row_of),
                                _p(topk_w), _p(dy_routed), _p(dw), _s(stream)), "moe_combine_bwd")
+
+
+def moe_router_bwd(dims, x, wg, probs, topk_idx, topk_w, dw, dlogits, dx, dwg, accumulate, ws,
+                   stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _ck(load().moe_router_bwd(ctypes.byref(dims), _p(x), _p(wg), _p(probs), _p(topk_idx),
+                              _p(topk_w), _p(dw), _p(dlogits), _p(dx), _p(dwg), int(accumulate),
+                              _p(ws), nbytes, _s(stream)), "moe_router_bwd")
+
+
+def moe_bias_update(dims, counts, gamma, bias_in, bias_out, stream=None):
+    _ck(load().moe_bias_update(ctypes.byref(dims), _p(counts), float(gamma), _p(bias_in),
+                               _p(bias_out), _s(stream)), "moe_bias_update")
 
 
 def moe_get_device_status(ws, stream=None) -> int:

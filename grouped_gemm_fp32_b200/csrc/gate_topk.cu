@@ -366,6 +366,17 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 
 }  // namespace
 
+int launch_split_wg(const moe_dims& dm, const float* wg, void* planes, void* stream) {
+  const int e_pad = (dm.E + 31) / 32 * 32;
+  const int64_t n4 = (int64_t)e_pad * dm.d / 4;
+  const int threads = 256;
+  int64_t blocks = (n4 + threads - 1) / threads;
+  if (blocks > 4096) blocks = 4096;
+  split_wg_kernel<<<(unsigned)blocks, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      wg, dm.E, e_pad, dm.d, reinterpret_cast<__nv_bfloat16*>(planes));
+  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const float* bias,
                      int32_t* idx, float* w, float* probs, void* ws, void* stream) {
   const int64_t T = dm.T;
@@ -377,12 +388,8 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
   const int e_pad = L.e_pad;
 
   {
-    const int64_t n4 = (int64_t)e_pad * dm.d / 4;
-    const int threads = 256;
-    int64_t blocks = (n4 + threads - 1) / threads;
-    if (blocks > 4096) blocks = 4096;
-    split_wg_kernel<<<(unsigned)blocks, threads, 0, st>>>(wg, dm.E, e_pad, dm.d, planes);
-    if (!cuda_ok(cudaGetLastError())) return MOE_ERR_CUDA;
+    const int rc = launch_split_wg(dm, wg, planes, stream);
+    if (rc != MOE_OK) return rc;
   }
 
   GateArgs a{};

@@ -71,6 +71,27 @@ int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const fl
   return launch_gate_topk(*dims, x, wg, bias, topk_idx, topk_w, probs, ws, stream);
 }
 
+int moe_router_bwd(const moe_dims* dims, const void* x, const float* wg, const float* probs,
+                   const int32_t* topk_idx, const float* topk_w, const float* dw, float* dlogits,
+                   void* dx, float* dwg, int accumulate, void* ws, size_t ws_bytes,
+                   void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (dims->E % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!ws || ws_bytes < ws_layout(*dims).total || !wg || !dwg) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!x || !probs || !topk_idx || !topk_w || !dw || !dx))
+    return MOE_ERR_INVALID_ARG;
+  return launch_router_bwd(*dims, x, wg, probs, topk_idx, topk_w, dw, dlogits, dx, dwg,
+                           accumulate ? 1 : 0, ws, stream);
+}
+
+int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
+                    const float* bias_in, float* bias_out, void* stream) {
+  if (!dims_ok(dims)) return MOE_ERR_INVALID_ARG;
+  if (!counts || !bias_in || !bias_out) return MOE_ERR_INVALID_ARG;
+  return launch_bias_update(*dims, counts, gamma, bias_in, bias_out, stream);
+}
+
 int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void* x,
                       int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* row_of,
                       void* x_perm, void* ws, size_t ws_bytes, void* stream) {

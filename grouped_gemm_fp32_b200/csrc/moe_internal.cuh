@@ -29,7 +29,7 @@ constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] ti
                                   // [3] routing valid, [4] bad expert id seen
 
 // Layer workspace: the routing tables first (`bytes` of them), then the
-// gate's split weights.
+// gate's split weights, then the router backward's scratch.
 struct WsLayout {
   size_t groups;        // GroupRec[G]
   size_t mtile_prefix;  // int32[G + 1]  prefix of ceil(rows_pad / 256) (pair tiles)
@@ -37,10 +37,28 @@ struct WsLayout {
   size_t chunk_hist;    // int32[nchunks * E]
   size_t bytes;         // end of the routing tables
   size_t gate_split;    // bf16[3][e_pad][d]  the gate weights as hi, mid, lo planes
+  size_t dl_planes;     // bf16[3][t_pad][e_pad]  dL/dlogit as hi, mid, lo planes
+  size_t gdw_part;      // f32[gdw_splits][e_pad][d]  split-K partial sums of dWg
   size_t total;         // whole workspace
   int nchunks;
   int e_pad;            // E rounded up to a multiple of 32
+  int t_pad;            // T rounded up to a multiple of 128
+  int gdw_splits;       // K splits of the dWg GEMM
 };
+
+// K splits of the dWg GEMM: as many work items as fit one wave on a B200's 148
+// SMs, at most 16 splits, and no split left empty.
+inline int gdw_splits_of(int e_pad, int d, int t_pad) {
+  const int tiles = ((e_pad + 127) / 128) * ((d + 255) / 256);
+  const int kb = 3 * (t_pad / 64);
+  if (kb == 0) return 1;
+  int s = 148 / tiles;
+  if (s < 1) s = 1;
+  if (s > 16) s = 16;
+  if (s > kb) s = kb;
+  const int per = (kb + s - 1) / s;
+  return (kb + per - 1) / per;
+}
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -61,8 +79,12 @@ inline WsLayout ws_layout(const moe_dims& dm) {
   off += sizeof(int32_t) * (size_t)L.nchunks * dm.E;
   L.bytes = align_up(off, 256);
   L.e_pad = (dm.E + 31) / 32 * 32;
+  L.t_pad = (int)((dm.T + 127) / 128 * 128);
+  L.gdw_splits = gdw_splits_of(L.e_pad, dm.d, L.t_pad);
   L.gate_split = align_up(L.bytes, 1024);
-  L.total = align_up(L.gate_split + (size_t)3 * L.e_pad * dm.d * 2, 256);
+  L.dl_planes = align_up(L.gate_split + (size_t)3 * L.e_pad * dm.d * 2, 1024);
+  L.gdw_part = align_up(L.dl_planes + (size_t)3 * L.t_pad * L.e_pad * 2, 1024);
+  L.total = align_up(L.gdw_part + (size_t)L.gdw_splits * L.e_pad * dm.d * 4, 256);
   return L;
 }
 
@@ -79,6 +101,17 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
                    void* stream);
 int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offsets, void* ws,
                       void* stream);
+int launch_split_wg(const moe_dims& dm, const float* wg, void* planes, void* stream);
+int launch_router_bwd(const moe_dims& dm, const void* x, const float* wg, const float* probs,
+                      const int32_t* idx, const float* w, const float* dw, float* dlogits,
+                      void* dx, float* dwg, int accumulate, void* ws, void* stream);
+int launch_bias_update(const moe_dims& dm, const int32_t* counts, float gamma,
+                       const float* bias_in, float* bias_out, void* stream);
+// Router-backward GEMMs (sgemm.cu); planes and partial sums live in the workspace.
+int launch_gate_dx(const moe_dims& dm, const void* dl_planes, const void* wg_planes, void* dx,
+                   int* status, void* stream);
+int launch_gate_dw(const moe_dims& dm, const void* dl_planes, const void* x, float* partial,
+                   int* status, void* stream);
 int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, const float* w,
                    void* out, void* stream);
 int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,

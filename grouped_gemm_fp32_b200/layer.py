@@ -11,8 +11,10 @@ and "Load balancing"; §3.2 "Efficient implementation of Grouped GEMM"):
     backward  moe_combine_bwd -> grouped_gemm_bwd_dx(GEMM2) -> grouped_gemm_bwd_dw(GEMM2)
               -> grouped_gemm_bwd_dx(GEMM1) -> grouped_gemm_bwd_dw(GEMM1)
               -> moe_combine(weights = NULL)  (un-permute-sum of the dX rows)
-The backward returns the gradient through the experts and the combine weights;
-the router's own gradient is not part of this path.
+              [-> moe_router_bwd (dlogits; gate term added into dX; dWg)]
+              [-> moe_bias_update (next step's selection bias)]
+The router backward runs when the gate weights are passed to ``backward``; the
+bias step when an update speed ``gamma`` is.
 """
 from __future__ import annotations
 
@@ -54,6 +56,9 @@ class MoEBuffers:
             self.dx = e(T, d)
             self.dw1 = e(G, 2 * I, d, dt=f32)
             self.dw2 = e(G, d, I, dt=f32)
+            self.probs = e(T, E, dt=f32)
+            self.dwg = e(E, d, dt=f32)
+            self.bias_next = e(E, dt=f32)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in vars(self).values()
@@ -63,14 +68,19 @@ class MoEBuffers:
 def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
     """out = MoE(x).  x [T, d] bf16, wg [E, d] f32, bias [E] f32, w1 [G, 2I, d], w2 [G, d, I].
 
-    ``routing=(topk_idx, topk_w)`` (device int32 / f32 [T, k]) replaces the gate's
-    choice, e.g. to run the experts on a routing decided elsewhere."""
+    ``routing=(topk_idx, topk_w[, probs])`` (device int32 / f32 [T, k], f32 [T, E])
+    replaces the gate's choice, e.g. to run the experts on a routing decided
+    elsewhere.  With train buffers the gate also saves its affinities (probs) for
+    the router backward."""
     dm = b.dims
+    probs = b.probs if b.train else None
     if routing is None:
-        L.moe_gate_topk(dm, x, wg, bias, b.topk_idx, b.topk_w, None, b.ws, stream)
+        L.moe_gate_topk(dm, x, wg, bias, b.topk_idx, b.topk_w, probs, b.ws, stream)
     else:
         b.topk_idx.copy_(routing[0])
         b.topk_w.copy_(routing[1])
+        if probs is not None and len(routing) > 2:
+            probs.copy_(routing[2])
     L.moe_permute_align(dm, b.topk_idx, x, b.counts, b.offsets, b.sorted_ids, b.row_of, b.x_perm,
                         b.ws, stream)
     L.grouped_gemm_fwd(dm, b.ws, b.x_perm, x, w1, w2, b.h, b.a1, b.y, stream)
@@ -78,9 +88,12 @@ def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
     return b.out
 
 
-def backward(b: MoEBuffers, x, dout, w1, w2, stream=None):
-    """Gradients after ``forward``: dx [T, d] (through the experts), dw1, dw2 (f32) and the
-    combine-weight gradient dw_comb [T, k]."""
+def backward(b: MoEBuffers, x, dout, w1, w2, stream=None, wg=None, gamma=None, bias=None):
+    """Gradients after ``forward``: dx [T, d], dw1, dw2 (f32) and the combine-weight
+    gradient dw_comb [T, k].  dx holds the gradient through the experts, plus the
+    router's (dlogit Wg) when ``wg`` is given; then ``b.dwg`` [E, d] f32 holds dL/dWg.
+    With ``gamma`` (and the step's ``bias``) ``b.bias_next`` receives the
+    aux-loss-free bias step."""
     if not b.train:
         raise ValueError("buffers were allocated without train=True")
     dm = b.dims
@@ -90,6 +103,11 @@ def backward(b: MoEBuffers, x, dout, w1, w2, stream=None):
     L.grouped_gemm_bwd_dx(dm, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, stream)
     L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x, b.dw1, 0, stream)
     L.moe_combine(dm, b.dxp, b.row_of, None, b.dx, stream)
+    if wg is not None:
+        L.moe_router_bwd(dm, x, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb, None, b.dx, b.dwg,
+                         0, b.ws, stream)
+    if gamma is not None:
+        L.moe_bias_update(dm, b.counts, gamma, bias, b.bias_next, stream)
     return b.dx, b.dw1, b.dw2, b.dw_comb
 
 
@@ -104,8 +122,9 @@ class HostPipeline:
     added.  All arithmetic runs in libmoe.so; torch provides memory and streams.
     """
 
-    def __init__(self, dims: L.MoeDims, w1, w2, wg, bias, train: bool, device="cuda"):
-        self.dims, self.train = dims, train
+    def __init__(self, dims: L.MoeDims, w1, w2, wg, bias, train: bool, device="cuda",
+                 gamma=None):
+        self.dims, self.train, self.gamma = dims, train, gamma
         self.w1, self.w2, self.wg, self.bias = w1, w2, wg, bias
         dev = torch.device(device)
         T, d = dims.T, dims.d
@@ -149,7 +168,8 @@ class HostPipeline:
                 s.wait_event(self.downloaded[j])  # results of step i-2 have left set j
                 forward(b, self.x[j], self.wg, self.bias, self.w1, self.w2, stream=s)
                 if self.train:
-                    backward(b, self.x[j], self.dout[j], self.w1, self.w2, stream=s)
+                    backward(b, self.x[j], self.dout[j], self.w1, self.w2, stream=s,
+                             wg=self.wg, gamma=self.gamma, bias=self.bias)
                 self.computed[j].record(s)
                 self.consumed[j].record(s)
             with torch.cuda.stream(self.down):

@@ -13,6 +13,8 @@
  *   5. weighted combine                                        (moe_combine)
  *   backward: combine bwd, dX and dW grouped GEMMs             (moe_combine_bwd,
  *             grouped_gemm_bwd_dx, grouped_gemm_bwd_dw, moe_combine)
+ *   router backward: dlogits, gate dX and dWg                  (moe_router_bwd)
+ *   aux-loss-free bias step                                    (moe_bias_update)
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -228,6 +230,47 @@ int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, cons
 int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, const void* y,
                     const int32_t* row_of, const float* topk_w, void* dy_routed, float* dw,
                     void* stream);
+
+/* Router backward: the gradient of the combine weights through their
+ * renormalisation over the chosen k and the softmax, into the gate's input and
+ * weights.
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts
+ * layer" (FP32 gate; the weights are the chosen experts' affinities) and "Load
+ * balancing" (the bias only decides the selection, so it gets no gradient; the
+ * selection itself is piecewise constant).  With Z = sum_{j chosen} p_j:
+ *   dp_j = (dw_j - sum_i dw_i w_i) / Z  (chosen j; 0 elsewhere)
+ *   dlogit_e = p_e (dp_e - sum_j p_j dp_j)
+ *   dx += dlogit Wg                      dwg (+)= dlogit^T x
+ *   x        [T, d] bf16             the gate's input
+ *   wg       [E, d] f32              gate weights
+ *   probs    [T, E] f32              softmax affinities (moe_gate_topk's probs)
+ *   topk_idx, topk_w [T, k]          the forward's choice and combine weights
+ *   dw       [T, k] f32              dL/dw (moe_combine_bwd's dw)
+ * Out:
+ *   dlogits  [T, E] f32              may be NULL
+ *   dx       [T, d] bf16             read-modify-write: the gate's term is added
+ *   dwg      [E, d] f32              written, or added to when accumulate != 0
+ *   ws / ws_bytes                    workspace of moe_workspace_size(dims) bytes;
+ *                                    the call overwrites its gate-weight planes and
+ *                                    scratch, not its routing tables
+ * Both GEMMs run on the tensor cores over exact three-term bf16 splits of the
+ * FP32 operands (dlogit, Wg), accumulating in FP32.  Requires E % 8 == 0,
+ * E <= 256, d % 64 == 0.  A bounded wait that runs out on the device sets
+ * MOE_ERR_DEVICE_TIMEOUT in the status word. */
+int moe_router_bwd(const moe_dims* dims, const void* x, const float* wg, const float* probs,
+                   const int32_t* topk_idx, const float* topk_w, const float* dw, float* dlogits,
+                   void* dx, float* dwg, int accumulate, void* ws, size_t ws_bytes, void* stream);
+
+/* Aux-loss-free bias step.
+ * Passage: dots.llm1 Technical Report, §Architecture "Load balancing" (the
+ * per-expert bias is adjusted during training to keep the loads balanced; the
+ * pages give no rule, this is the plainest one of that kind):
+ *   bias_out[e] = bias_in[e] + gamma * sign(T k / E - counts[e])   (sign(0) = 0)
+ *   counts [E] int32   the step's routed load per expert (moe_permute_align's counts)
+ * bias_in and bias_out may be the same buffer.  One FP32 addition per expert,
+ * correctly rounded. */
+int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
+                    const float* bias_in, float* bias_out, void* stream);
 
 /* Reads and clears the device status word of `ws` (synchronises `stream`).
  * *status_out receives MOE_OK or the first device error recorded. */

@@ -128,15 +128,18 @@ def route(logits: np.ndarray, bias: np.ndarray, k: int):
     return probs, idx, w, margin
 
 
-def router_bwd(x: np.ndarray, wg: np.ndarray, idx: np.ndarray, dw: np.ndarray):
+def router_bwd(x: np.ndarray, wg: np.ndarray, idx: np.ndarray, dw: np.ndarray,
+               want_dx: bool = True, want_dwg: bool = True):
     """Gradient of the combine weights through the renormalisation and the softmax:
-    (dlogits [T,E], dx [T,d], dwg [E,d]), all FP64.  x: bf16 bits [T,d]; wg: f32 [E,d];
-    idx [T,k] the chosen experts; dw [T,k] = dL/dw."""
+    (dlogits [T,E], dx [T,d], dwg [E,d]), all FP64 (dx / dwg None when not wanted).
+    x: bf16 bits [T,d]; wg: f32 [E,d]; idx [T,k] the chosen experts; dw [T,k] = dL/dw."""
     x, wg, idx, dw = _c(x, np.uint16), _c(wg, np.float32), _c(idx, np.int32), _c(dw, np.float64)
     T, d = x.shape
     E = wg.shape[0]
     k = idx.shape[1]
-    dl = np.empty((T, E)); dx = np.empty((T, d)); dwg = np.empty((E, d))
+    dl = np.empty((T, E))
+    dx = np.empty((T, d)) if want_dx else None
+    dwg = np.empty((E, d)) if want_dwg else None
     _load().oracle_router_bwd(_p(x), _p(wg), _p(idx), _p(dw), T, d, E, k, _p(dl), _p(dx),
                               _p(dwg))
     return dl, dx, dwg

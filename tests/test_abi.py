@@ -91,6 +91,17 @@ def test_validation_rejects_before_any_launch(lib):
     assert L.grouped_gemm_bwd_dx(ctypes.byref(ok64), p, 7, p, p, p, p, p, nul) == -1
     assert L.grouped_gemm_bwd_dw(ctypes.byref(ok64), p, 2, p, p, p, p, p, 5, nul) == -1
     assert L.moe_gate_topk(None, p, p, p, p, p, nul, p, 1 << 30, nul) == -1
+    # router backward: workspace, pointers, shapes; bias step: pointers
+    big = 1 << 40
+    assert L.moe_router_bwd(ctypes.byref(ok), p, p, p, p, p, p, nul, p, p, 0, nul, big, nul) == -1
+    assert L.moe_router_bwd(ctypes.byref(ok), p, p, p, p, p, p, nul, p, p, 0, p, 8, nul) == -1
+    assert L.moe_router_bwd(ctypes.byref(ok), nul, p, p, p, p, p, nul, p, p, 0, p, big, nul) == -1
+    assert L.moe_router_bwd(ctypes.byref(ok), p, p, p, p, p, p, nul, p, nul, 0, p, big, nul) == -1
+    e12 = lib.MoeDims.of(64, 128, 12, 2, 1, 64, 16)  # E % 8
+    assert L.moe_router_bwd(ctypes.byref(e12), p, p, p, p, p, p, nul, p, p, 0, p, big, nul) == -2
+    assert L.moe_bias_update(None, p, 1e-3, p, p, nul) == -1
+    assert L.moe_bias_update(ctypes.byref(ok), nul, 1e-3, p, p, nul) == -1
+    assert L.moe_bias_update(ctypes.byref(ok), p, 1e-3, p, nul, nul) == -1
 
 
 def test_status_strings(lib):
