@@ -6,7 +6,8 @@
 // experts that every token uses.
 //
 // HBM-bound; one warp per token, 16-byte vector accesses along the hidden
-// dimension, FP32 accumulation.
+// dimension, FP32 accumulation.  The backward keeps the token's upstream row in
+// registers for its k picks when d is 2048 or 4096.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -116,6 +117,48 @@ __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* 
   }
 }
 
+// Same, with the token's dOut row held in registers for all k picks: lane l owns
+// vectors l, l + 32, ... of the row (VPL = row_vec / 32 of them), and each pick's
+// Y row is loaded whole before it is used, so VPL loads are in flight per lane.
+template <int VPL>
+__global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
+                                       const int32_t* __restrict__ row_of,
+                                       const float* __restrict__ w, int64_t T, int k,
+                                       uint4* __restrict__ dy, float* __restrict__ dw) {
+  constexpr int row_vec = 32 * VPL;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  uint4 g[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) g[i] = dout[t * row_vec + lane + 32 * i];
+  for (int j = 0; j < k; ++j) {
+    const int64_t r = row_of[t * k + j];
+    const float wj = w[t * k + j];
+    uint4 yv[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) yv[i] = y[r * row_vec + lane + 32 * i];
+    float dot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      acc8(a, g[i], wj);
+      dy[r * row_vec + lane + 32 * i] = pack8(a);
+      const uint32_t gu[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
+      const uint32_t yu[4] = {yv[i].x, yv[i].y, yv[i].z, yv[i].w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        dot = fmaf(__uint_as_float(gu[p] << 16), __uint_as_float(yu[p] << 16), dot);
+        dot = fmaf(__uint_as_float(gu[p] & 0xFFFF0000u), __uint_as_float(yu[p] & 0xFFFF0000u),
+                   dot);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane == 0) dw[t * k + j] = dot;
+  }
+}
+
 }  // namespace
 
 int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream);
@@ -145,9 +188,17 @@ int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, con
   if (rc != MOE_OK || dm.T == 0) return rc;
   const int warps = 8;
   const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);
-  combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(
-      reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), row_of, w, dm.T,
-      dm.d / 8, dm.k, reinterpret_cast<uint4*>(dy), dw);
+  const uint4* dv = reinterpret_cast<const uint4*>(dout);
+  const uint4* yv = reinterpret_cast<const uint4*>(y);
+  uint4* dyv = reinterpret_cast<uint4*>(dy);
+  const int row_vec = dm.d / 8;
+  if (row_vec == 512)
+    combine_bwd_reg_kernel<16><<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
+  else if (row_vec == 256)
+    combine_bwd_reg_kernel<8><<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
+  else
+    combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, row_vec, dm.k, dyv,
+                                                      dw);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 

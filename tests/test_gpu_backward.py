@@ -36,8 +36,13 @@ def _run(wl, inp, routing=None):
     return b, dx, dw1, dw2, dwc
 
 
-def test_backward_small_full():
-    wl = SMALL
+SMALL_2048 = synth.Workload("small_train_2048", synth.Dims(T=200, d=2048, E=8, k=2, S=1, I=64,
+                                                         P=64),
+                            seed=12, w1_std=0.02, w2_std=0.05, wg_std=0.02, backward=True)
+
+
+@pytest.mark.parametrize("wl", [SMALL, SMALL_2048], ids=["d128", "d2048"])
+def test_backward_small_full(wl):
     inp = synth.make_inputs(wl)
     S = wl.dims.S
     p, oidx, ow, margin = oracle.route(oracle.gate_logits(inp["x"], inp["wg"]), inp["bias"],
