@@ -49,6 +49,7 @@ constexpr int MAX_STAGES = 6;
 constexpr int A_BYTES = BM * BK * 2;    // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of B (N/2 <= 128)
 constexpr int EPI_WARPS = 8;            // two per tensor-memory lane quarter
+constexpr int SLOT_BYTES = 32 * 128;    // an epilogue warp's staging slot: 32 rows x 128 B
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;     // two 256-column FP32 accumulators
 constexpr int MAX_GROUPS = 264;  // E <= 256 routed + S <= 8 shared
@@ -74,6 +75,7 @@ struct GemmArgs {
   int accumulate;
   uint32_t idesc;
   uint32_t idesc_narrow;  // N = 128 (modes whose B is N-major)
+  int staged;             // epilogue writes through shared memory + TMA stores
   uint64_t budget_ns;
 };
 
@@ -98,7 +100,7 @@ __host__ __device__ constexpr int stages_of() {
 template <int MODE>
 constexpr size_t smem_bytes() {
   return 1024 /* alignment slack */ + stages_of<MODE>() * (A_BYTES + B_BYTES) +
-         sizeof(SmemCtl) + 64;
+         EPI_WARPS * SLOT_BYTES + sizeof(SmemCtl) + 64;
 }
 
 struct TileInfo {
@@ -168,17 +170,61 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+// Eight 16-byte pieces of bf16: v[8 q .. 8 q + 7] -> piece q.
+__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
+  uint4 w;
+  w.x = pack_bf16(v[0], v[1]);
+  w.y = pack_bf16(v[2], v[3]);
+  w.z = pack_bf16(v[4], v[5]);
+  w.w = pack_bf16(v[6], v[7]);
+  return w;
+}
+
+// Staged stores.  An epilogue warp owns a 4 KB shared-memory slot for 32 rows x
+// 128 bytes in the 128-byte swizzled layout (16-byte piece j of row r sits at
+// j ^ (r % 8), so a warp's 16-byte writes cover all banks).  Thread `lane` writes
+// row `lane`; lane 0 then issues one TMA store -- or f32 add-reduction -- of the
+// 32-row box.  The slot is rewritten only after the previous store has read it.
+__device__ __forceinline__ void slot_acquire(int lane) {
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+}
+
+__device__ __forceinline__ void slot_put(uint8_t* slot, int lane, int j, uint4 v) {
+  *reinterpret_cast<uint4*>(slot + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+}
+
+template <bool REDUCE>
+__device__ __forceinline__ void slot_issue(uint8_t* slot, const CUtensorMap* map, int x, int y,
+                                           int lane) {
+  fence_proxy_async_smem();  // the generic-proxy writes become visible to the TMA unit
+  __syncwarp();
+  if (lane == 0) {
+    if (REDUCE)
+      tma_reduce_add_2d(map, slot, x, y);
+    else
+      tma_store_2d(map, slot, x, y);
+    bulk_commit();
+  }
+}
+
+template <bool REDUCE>
+__device__ __forceinline__ void staged_store(uint8_t* slot, const uint4 (&v)[8],
+                                             const CUtensorMap* map, int x, int y, int lane) {
+  slot_acquire(lane);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w = s4[q];
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  for (int j = 0; j < 8; ++j) slot_put(slot, lane, j, v[j]);
+  slot_issue<REDUCE>(slot, map, x, y, lane);
+}
+
+// bf16 of 32 accumulator words, as four 16-byte pieces
+__device__ __forceinline__ void pack_acc_bf16(const uint32_t (&r)[32], uint4 (&p)[4]) {
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      v[8 * q + 2 * p] = __uint_as_float(u[p] << 16);
-      v[8 * q + 2 * p + 1] = __uint_as_float(u[p] & 0xFFFF0000u);
-    }
+  for (int j = 0; j < 4; ++j) {
+    p[j].x = pack_bf16(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+    p[j].y = pack_bf16(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+    p[j].z = pack_bf16(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+    p[j].w = pack_bf16(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
   }
 }
 
@@ -187,6 +233,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ggemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                  const __grid_constant__ CUtensorMap tmC /* DX2: saved [G | U] */,
+                 const __grid_constant__ CUtensorMap tmO0 /* output (FWD1: H) */,
+                 const __grid_constant__ CUtensorMap tmO1 /* FWD1: saved A1 */,
                  const GemmArgs args) {
   constexpr bool A_MN = (MODE == MODE_DW2 || MODE == MODE_DW1);
   constexpr bool B_MN = (MODE != MODE_FWD1 && MODE != MODE_FWD2);
@@ -198,7 +246,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                              ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sB + STAGES * B_BYTES);
+  uint8_t* sSlots = sB + STAGES * B_BYTES;  // epilogue staging, one slot per epilogue warp
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sSlots + EPI_WARPS * SLOT_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -224,6 +273,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
     if (MODE == MODE_DX2) tma_prefetch_desc(&tmC);
+    if (args.staged) {
+      tma_prefetch_desc(&tmO0);
+      if (MODE == MODE_FWD1 && args.out2 != nullptr) tma_prefetch_desc(&tmO1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
@@ -427,127 +480,208 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const GroupRec gr = load_group(args, t.g);
       uint32_t r[32];
       float v[32];
+      uint8_t* slot = sSlots + (warp - 2) * SLOT_BYTES;
+      // this warp's 32 rows within its group: all real (staged TMA stores), none,
+      // or cut by the group's end (direct stores of the real rows)
+      const int rb = t.m0 + (int)rank * BM + q * 32;
       if constexpr (MODE == MODE_FWD1) {
         const int rloc = t.m0 + r_in_tile;
         const bool rv = rloc < gr.rows_pad;
+        const bool whole = rb + 32 <= gr.rows_pad;
         const int64_t orow = (int64_t)gr.out_row + rloc;
         __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0;
         __nv_bfloat16* A1 = reinterpret_cast<__nv_bfloat16*>(args.out2);
         const int cb = h * (args.hn >> 1), ce = cb + (args.hn >> 1);  // this warp's H columns
-        for (int c0 = cb; c0 < ce; c0 += 32) {
-          uint32_t u[32];
-          tmem_ld32_sync(taddr + c0, r);
-          tmem_ld32_sync(taddr + args.hn + c0, u);
-          if (c0 + 32 >= ce) release(acc);
-          if (rv) {
-            float hv[32];
+        if (args.staged && whole) {
+          // hn == 128: 64 H columns per warp, one 128-byte row each of H, then of the
+          // saved gate and up pre-activations (read from tensor memory again)
+          const int y = gr.out_row + rb;
+          slot_acquire(lane);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float g = __uint_as_float(r[i]), up = __uint_as_float(u[i]);
-              hv[i] = g / (1.0f + expf(-g)) * up;
-            }
-            store_bf16x32(H + c0, hv);
-            if (A1 != nullptr) {
-              __nv_bfloat16* a1r = A1 + orow * args.ld_out2 + t.n0 + c0;
+          for (int s2 = 0; s2 < 2; ++s2) {
+            uint32_t u[32];
+            tmem_ld32_sync(taddr + cb + 32 * s2, r);
+            tmem_ld32_sync(taddr + args.hn + cb + 32 * s2, u);
+            if (s2 == 1 && A1 == nullptr) release(acc);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-              store_bf16x32(a1r, v);
+            for (int j = 0; j < 4; ++j) {
+              float hv[8];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(u[i]);
-              store_bf16x32(a1r + args.I, v);
+              for (int i = 0; i < 8; ++i) {
+                const float g = __uint_as_float(r[8 * j + i]), up = __uint_as_float(u[8 * j + i]);
+                hv[i] = g / (1.0f + expf(-g)) * up;
+              }
+              slot_put(slot, lane, 4 * s2 + j, pack_bf16x8(hv));
             }
           }
+          slot_issue<false>(slot, &tmO0, t.n0 + cb, y, lane);
+          if (A1 != nullptr) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {  // gate columns, then up columns
+              slot_acquire(lane);
+#pragma unroll
+              for (int s2 = 0; s2 < 2; ++s2) {
+                uint4 pk[4];
+                tmem_ld32_sync(taddr + part * args.hn + cb + 32 * s2, r);
+                if (part == 1 && s2 == 1) release(acc);
+                pack_acc_bf16(r, pk);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) slot_put(slot, lane, 4 * s2 + j, pk[j]);
+              }
+              slot_issue<false>(slot, &tmO1, part * args.I + t.n0 + cb, y, lane);
+            }
+          }
+        } else {
+          for (int c0 = cb; c0 < ce; c0 += 32) {
+            uint32_t u[32];
+            tmem_ld32_sync(taddr + c0, r);
+            tmem_ld32_sync(taddr + args.hn + c0, u);
+            if (c0 + 32 >= ce) release(acc);
+            if (rv) {
+              float hv[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float g = __uint_as_float(r[i]), up = __uint_as_float(u[i]);
+                hv[i] = g / (1.0f + expf(-g)) * up;
+              }
+              store_bf16x32(H + c0, hv);
+              if (A1 != nullptr) {
+                __nv_bfloat16* a1r = A1 + orow * args.ld_out2 + t.n0 + c0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                store_bf16x32(a1r, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(u[i]);
+                store_bf16x32(a1r + args.I, v);
+              }
+            }
+          }
+          if (cb >= ce) release(acc);
         }
-        if (cb >= ce) release(acc);
       } else if constexpr (MODE == MODE_FWD2 || MODE == MODE_DX1) {
         const int rloc = t.m0 + r_in_tile;
         const bool rv = rloc < gr.rows_pad;
+        const bool whole = rb + 32 <= gr.rows_pad;
         const int64_t orow = (int64_t)gr.out_row + rloc;
         __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0;
-        const int cb = h * 128, ce = min(cb + 128, args.n_out - t.n0);
-        for (int c0 = cb; c0 < ce; c0 += 32) {
+        const int cb = h * 128, ce = min(cb + 128, args.n_out - t.n0);  // multiples of 64
+        for (int c0 = cb; c0 < ce; c0 += 64) {
+          uint32_t u[32];
           tmem_ld32_sync(taddr + c0, r);
-          if (c0 + 32 >= ce) release(acc);
-          if (rv) {
+          tmem_ld32_sync(taddr + c0 + 32, u);
+          if (c0 + 64 >= ce) release(acc);
+          if (args.staged && whole) {
+            uint4 pk[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[8 * j + i]);
+              pk[j] = pack_bf16x8(v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(u[8 * j + i]);
+              pk[4 + j] = pack_bf16x8(v);
+            }
+            staged_store<false>(slot, pk, &tmO0, t.n0 + c0, gr.out_row + rb, lane);
+          } else if (rv) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
             store_bf16x32(O + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(u[i]);
+            store_bf16x32(O + c0 + 32, v);
           }
         }
         if (cb >= ce) release(acc);
       } else if constexpr (MODE == MODE_DX2) {
         const int rloc = t.m0 + r_in_tile;
         const bool rv = rloc < gr.rows_pad;
+        const bool whole = rb + 32 <= gr.rows_pad;
         const int64_t orow = (int64_t)gr.out_row + rloc;
         const __nv_bfloat16* A1 =
             reinterpret_cast<const __nv_bfloat16*>(args.aux) + orow * args.ld_aux;
         __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out;
-        const int cb = h * 128, ce = min(cb + 128, args.I - t.n0);
-        for (int c0 = cb; c0 < ce; c0 += 32) {
+        const int cb = h * 128, ce = min(cb + 128, args.I - t.n0);  // multiples of 64
+        const bool staged = args.staged && whole;
+        for (int c0 = cb; c0 < ce; c0 += 64) {
           const int col = t.n0 + c0;
-          float gv[32], uv[32];
-          if (rv) {  // issue the saved-activation loads before waiting on tensor memory
-            load_bf16x32(A1 + col, gv);
-            load_bf16x32(A1 + args.I + col, uv);
-          }
-          tmem_ld32_sync(taddr + c0, r);
-          if (c0 + 32 >= ce) release(acc);
-          if (rv) {
-            float dg[32], du[32];
+          uint4 upk[8];  // staged: the du pieces wait here while dg goes out through the slot
+          if (staged) slot_acquire(lane);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float dh = __uint_as_float(r[i]);
-              const float g = gv[i];
-              const float s = 1.0f / (1.0f + expf(-g));
-              dg[i] = dh * uv[i] * s * (1.0f + g * (1.0f - s));
-              du[i] = dh * g * s;
+          for (int s2 = 0; s2 < 2; ++s2) {
+            const int cc = col + 32 * s2;
+            uint4 gq[4], uq[4];  // saved G and U of these 32 columns, bf16
+            if (rv) {  // issue the saved-activation loads before waiting on tensor memory
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                gq[j] = reinterpret_cast<const uint4*>(A1 + cc)[j];
+                uq[j] = reinterpret_cast<const uint4*>(A1 + args.I + cc)[j];
+              }
             }
-            store_bf16x32(dA + col, dg);
-            store_bf16x32(dA + args.I + col, du);
+            tmem_ld32_sync(taddr + c0 + 32 * s2, r);
+            if (s2 == 1 && c0 + 64 >= ce) release(acc);
+            if (rv) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {  // 8 columns at a time
+                float dg[8], du[8];
+                const uint32_t gw[4] = {gq[j].x, gq[j].y, gq[j].z, gq[j].w};
+                const uint32_t uw[4] = {uq[j].x, uq[j].y, uq[j].z, uq[j].w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float dh = __uint_as_float(r[8 * j + i]);
+                  const float g = __uint_as_float(i & 1 ? gw[i >> 1] & 0xFFFF0000u : gw[i >> 1] << 16);
+                  const float up =
+                      __uint_as_float(i & 1 ? uw[i >> 1] & 0xFFFF0000u : uw[i >> 1] << 16);
+                  const float sg = 1.0f / (1.0f + expf(-g));
+                  dg[i] = dh * up * sg * (1.0f + g * (1.0f - sg));
+                  du[i] = dh * g * sg;
+                }
+                const uint4 pg = pack_bf16x8(dg), pu = pack_bf16x8(du);
+                if (staged) {
+                  slot_put(slot, lane, 4 * s2 + j, pg);
+                  upk[4 * s2 + j] = pu;
+                } else {
+                  reinterpret_cast<uint4*>(dA + cc)[j] = pg;
+                  reinterpret_cast<uint4*>(dA + args.I + cc)[j] = pu;
+                }
+              }
+            }
+          }
+          if (staged) {
+            slot_issue<false>(slot, &tmO0, col, gr.out_row + rb, lane);
+            staged_store<false>(slot, upk, &tmO0, args.I + col, gr.out_row + rb, lane);
           }
         }
         if (cb >= ce) release(acc);
-      } else {  // DW2 / DW1: f32 output [G, m_out, n_out]
-        // 16-lane loads: 4 consecutive lanes hold 8 consecutive columns of one row,
-        // so every 8-byte store instruction writes 8 complete 32-byte row segments.
-        const int rb = t.m0 + (int)rank * BM + q * 32;  // this warp's 32 output rows
-        const bool wvalid = rb < args.m_out;             // m_out % 32 == 0: all or none
-        float* O = reinterpret_cast<float*>(args.out) + (int64_t)t.g * args.m_out * args.n_out;
+      } else {  // DW2 / DW1: f32 output [G, m_out, n_out], 32 columns (128 B) a store
+        const bool wvalid = rb < args.m_out;  // m_out % 32 == 0: all rows or none
+        const bool write = wvalid && !((t.nkb == 0) && args.accumulate);
         const int cb = h * 128, ce = min(cb + 128, args.n_out - t.n0);
-        const int rsub = lane >> 2, csub = 2 * (lane & 3);
-        for (int c0 = cb; c0 < ce; c0 += 64) {
+        const int y = t.g * args.m_out + rb;
+        for (int c0 = cb; c0 < ce; c0 += 32) {
+          if (t.nkb > 0) {
+            tmem_ld32_sync(taddr + c0, r);
+          } else {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            if (t.nkb > 0) {
-              tmem_ld16x256_x8_sync(taddr + ((uint32_t)(16 * half) << 16) + c0, r);
-            } else {
+            for (int i = 0; i < 32; ++i) r[i] = 0u;
+          }
+          if (c0 + 32 >= ce) release(acc);
+          if (write) {
+            uint4 pk[8];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = 0u;
-            }
-            if (half == 1 && c0 + 64 >= ce) release(acc);
-            if (wvalid && !((t.nkb == 0) && args.accumulate)) {
-              const int64_t row0 = rb + 16 * half + rsub;
-              float* p0 = O + row0 * args.n_out + t.n0 + c0 + csub;
-              float* p1 = p0 + 8 * (int64_t)args.n_out;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                float2 a = make_float2(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
-                float2 b = make_float2(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                float2* d0 = reinterpret_cast<float2*>(p0 + 8 * i);
-                float2* d1 = reinterpret_cast<float2*>(p1 + 8 * i);
-                if (args.accumulate) {
-                  const float2 o0 = *d0, o1 = *d1;
-                  a.x += o0.x; a.y += o0.y; b.x += o1.x; b.y += o1.y;
-                }
-                *d0 = a;
-                *d1 = b;
-              }
-            }
+            for (int j = 0; j < 8; ++j)
+              pk[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            if (args.accumulate)
+              staged_store<true>(slot, pk, &tmO0, t.n0 + c0, y, lane);
+            else
+              staged_store<false>(slot, pk, &tmO0, t.n0 + c0, y, lane);
           }
         }
         if (cb >= ce) release(acc);
       }
     }
+    // every staged store has finished (written to global memory) before the CTA can exit
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -567,7 +701,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
 template <int MODE>
 int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
-                const CUtensorMap& b1, const CUtensorMap& c, const GemmArgs& args,
+                const CUtensorMap& b1, const CUtensorMap& c, const CUtensorMap& o0,
+                const CUtensorMap& o1, const GemmArgs& args,
                 cudaStream_t st) {
   static int num_sms = 0;
   static bool attr_set = false;
@@ -594,7 +729,7 @@ int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
     cudaGetLastError();  // a failed query only leaves the default grid
     attr_set = true;
   }
-  ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmem, st>>>(a0, a1, b0, b1, c, args);
+  ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmem, st>>>(a0, a1, b0, b1, c, o0, o1, args);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -620,21 +755,25 @@ static EncodeTiledFn get_encode() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows, cols] (cols contiguous); box = 64 elements (128
-// bytes) of a row x box_rows rows, 128-byte swizzle.
-bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+// Row-major matrix [rows, cols] (cols contiguous) of bf16 (esz 2) or f32 (esz 4);
+// box = 128 bytes of a row x box_rows rows, 128-byte swizzle.
+static bool make_map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int esz,
+                        int box_rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc || base == nullptr) return false;
-  const int esz = 2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(cols * esz)};
   cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                   const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  return make_map_2d(m, base, rows, cols, 2, box_rows);
 }
 
 uint64_t wait_budget_ns() {
@@ -670,7 +809,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   a.accumulate = ops.accumulate;
   a.budget_ns = wait_budget_ns();
 
-  CUtensorMap m0{}, m1{}, n0{}, n1{}, c0{};
+  CUtensorMap m0{}, m1{}, n0{}, n1{}, c0{}, o0{}, o1{};
   bool ok = true;
   // a dummy map stands in for unused slots (never read by the kernel)
   auto same = [](CUtensorMap& dst, const CUtensorMap& src) { dst = src; };
@@ -692,7 +831,12 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, hn);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, a, st);
+      // staged stores need 64 H columns per epilogue warp
+      a.staged = hn == 128;
+      ok &= make_map_2d(&o0, ops.out, Rt, I, 2, 32);
+      if (ops.out2 != nullptr) ok &= make_map_2d(&o1, ops.out2, Rt, 2 * I, 2, 32); else same(o1, o0);
+      if (!ok) return MOE_ERR_CUDA;
+      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, o0, o1, a, st);
     }
     case MODE_FWD2: {
       a.K = I;
@@ -706,7 +850,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 128);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, a, st);
+      a.staged = 1;
+      if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
+      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, o0, o0, a, st);
     }
     case MODE_DX2: {
       a.K = d;
@@ -723,7 +869,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       same(n1, n0);
       ok &= make_map_bf16(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, a, st);
+      a.staged = 1;
+      if (!make_map_2d(&o0, ops.out, Rt, 2 * I, 2, 32)) return MOE_ERR_CUDA;
+      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, o0, o0, a, st);
     }
     case MODE_DX1: {
       a.K = 2 * I;
@@ -738,7 +886,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, a, st);
+      a.staged = 1;
+      if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
+      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, o0, o0, a, st);
     }
     case MODE_DW2: {  // dW2_g [d, I] = dY_g^T H_g
       a.m_out = d;
@@ -752,7 +902,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, Rt, I, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, a, st);
+      a.staged = 1;
+      if (!make_map_2d(&o0, ops.out, (int64_t)G * d, I, 4, 32)) return MOE_ERR_CUDA;
+      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, a, st);
     }
     case MODE_DW1: {  // dW1_g [2I, d] = dA_g^T X_g
       a.m_out = 2 * I;
@@ -766,7 +918,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, Rr, d, 64);
       if (dm.S > 0) ok &= make_map_bf16(&n1, ops.b1, T, d, 64); else same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, a, st);
+      a.staged = 1;
+      if (!make_map_2d(&o0, ops.out, (int64_t)G * 2 * I, d, 4, 32)) return MOE_ERR_CUDA;
+      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, o0, o0, a, st);
     }
   }
   return MOE_ERR_INVALID_ARG;
