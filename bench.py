@@ -10,6 +10,8 @@ One step = one pass of the whole hot path over one batch:
                    grouped GEMMs, SwiGLU bwd, un-permute-sum, router backward
                    into dX and dWg) + the aux-loss-free bias step.
   layer:           T=8192, same layer, forward only.
+  skewed:          layer with Zipf-shaped expert loads (8 empty experts, the
+                   hottest taking every token), forward only.
   gemm_only:       the grouped GEMM forward alone (16 groups x 512 rows, d=4096,
                    I=1408): a small case for profiles, not the headline.
   train_small:     train with E=16, T=2048 (same rows per expert): profiles.
@@ -53,7 +55,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="train",
-                    choices=["train", "layer", "gemm_only", "train_small", "gate_only"])
+                    choices=["train", "layer", "skewed", "gemm_only", "train_small", "gate_only"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
