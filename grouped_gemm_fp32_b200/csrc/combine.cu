@@ -192,10 +192,12 @@ int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, con
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* dyv = reinterpret_cast<uint4*>(dy);
   const int row_vec = dm.d / 8;
+  // the register-resident form uses ~170 registers a thread: 4-warp CTAs, three per SM
+  const unsigned blocks4 = (unsigned)((dm.T + 3) / 4);
   if (row_vec == 512)
-    combine_bwd_reg_kernel<16><<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
+    combine_bwd_reg_kernel<16><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
   else if (row_vec == 256)
-    combine_bwd_reg_kernel<8><<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
+    combine_bwd_reg_kernel<8><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
   else
     combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, row_vec, dm.k, dyv,
                                                       dw);

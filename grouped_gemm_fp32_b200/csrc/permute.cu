@@ -25,6 +25,8 @@
 namespace moe {
 namespace {
 
+constexpr int kPadSplit = 8;  // CTAs per group zeroing its pad rows
+
 constexpr int kScatterThreads = 256;
 
 __global__ void hist_kernel(const int32_t* __restrict__ idx, int64_t n, int E,
@@ -67,7 +69,19 @@ __global__ void groups_kernel(int32_t* __restrict__ hist, int nchunks, int E, in
   __syncthreads();
   int c = 0;
   if (tid < E) {
-    for (int ch = 0; ch < nchunks; ++ch) {
+    // exclusive scan of this expert's chunk counts, 16 independent loads at a time
+    int ch = 0;
+    for (; ch + 16 <= nchunks; ch += 16) {
+      int v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = hist[(int64_t)(ch + u) * E + tid];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        hist[(int64_t)(ch + u) * E + tid] = c;
+        c += v[u];
+      }
+    }
+    for (; ch < nchunks; ++ch) {
       const int v = hist[(int64_t)ch * E + tid];
       hist[(int64_t)ch * E + tid] = c;
       c += v;
@@ -229,7 +243,10 @@ __global__ void zero_pad_rows_kernel(const GroupRec* __restrict__ groups, int ro
   const int64_t r0 = (int64_t)g.out_row + g.rows, r1 = (int64_t)g.out_row + g.rows_pad;
   const int64_t n = (r1 - r0) * row_vec;
   const uint4 z = make_uint4(0, 0, 0, 0);
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) m[r0 * row_vec + i] = z;
+  // blockIdx.y splits one group's pad rows across several CTAs
+  for (int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.y * blockDim.x)
+    m[r0 * row_vec + i] = z;
 }
 
 }  // namespace
@@ -281,8 +298,8 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
     copy_rows_kernel_bigk<<<blocks, warps * 32, 0, st>>>(reinterpret_cast<const uint4*>(x), dm.T,
                                                          row_vec, dm.k, row_of,
                                                          reinterpret_cast<uint4*>(x_perm), status);
-  zero_pad_rows_kernel<<<dm.E, 256, 0, st>>>(reinterpret_cast<const GroupRec*>(wsb + L.groups),
-                                             row_vec, reinterpret_cast<uint4*>(x_perm));
+  zero_pad_rows_kernel<<<dim3(dm.E, kPadSplit), 256, 0, st>>>(
+      reinterpret_cast<const GroupRec*>(wsb + L.groups), row_vec, reinterpret_cast<uint4*>(x_perm));
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -303,7 +320,7 @@ int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offset
 int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream) {
   const WsLayout L = ws_layout(dm);
   const uint8_t* wsb = reinterpret_cast<const uint8_t*>(ws);
-  zero_pad_rows_kernel<<<dm.E, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  zero_pad_rows_kernel<<<dim3(dm.E, kPadSplit), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const GroupRec*>(wsb + L.groups), cols / 8, reinterpret_cast<uint4*>(m));
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
