@@ -16,6 +16,7 @@ One step = one pass of the whole hot path over one batch:
                    I=1408): a small case for profiles, not the headline.
   train_small:     train with E=16, T=2048 (same rows per expert): profiles.
   gate_only:       the gate + top-k alone on the layer shapes: profiles.
+  tiny:            T=64, d=128, E=8: host-side checks of the launch plumbing.
 Inputs are synthetic (seeded generator), resident in HBM for ``value``; the
 weights alone (4.5 GB) exceed L2, so no flush is needed between steps.
 
@@ -55,7 +56,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="train",
-                    choices=["train", "layer", "skewed", "gemm_only", "train_small", "gate_only"])
+                    choices=["train", "layer", "skewed", "gemm_only", "train_small", "gate_only",
+                             "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -85,6 +87,21 @@ def workload(name):
         return wl, synth.make_inputs(wl, with_weights=False)
     wl = synth.WORKLOADS[name]
     return wl, synth.make_inputs(wl, bias_override=fitted_bias(name))
+
+
+def rank_shard(wl, inp, rank):
+    """This rank's batch: its own tokens (X and the upstream gradient drawn from a
+    rank-dependent seed), the replicated weights, gate and bias unchanged.  Rank 0
+    keeps the workload's own batch."""
+    if rank == 0:
+        return inp
+    import synth
+    dm, seed = wl.dims, wl.seed + 7919 * rank
+    out = dict(inp)
+    out["x"] = synth.normal_bf16(seed, synth.SID_X, (dm.T, dm.d), wl.x_std)
+    if "dout" in inp:
+        out["dout"] = synth.normal_bf16(seed, synth.SID_DOUT, (dm.T, dm.d), 1.0)
+    return out
 
 
 def gemm_flops(dm, backward):
@@ -285,6 +302,7 @@ def run_ours(args):
     from grouped_gemm_fp32_b200 import layer
 
     wl, inp = workload(args.workload)
+    inp = rank_shard(wl, inp, rank)  # data parallel: each rank its own tokens
     dm = wl.dims
     dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
     train = wl.backward
