@@ -827,7 +827,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.ld_out2 = 2 * I;
       a.idesc = idesc_bf16_f32(PM, 2 * hn, false, false);
       ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
-      if (dm.S > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, hn);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
@@ -864,7 +864,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.idesc = idesc_bf16_f32(PM, 256, false, true);
       a.idesc_narrow = idesc_bf16_f32(PM, 128, false, true);
       ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
-      if (dm.S > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 64);
       same(n1, n0);
       ok &= make_map_bf16(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
@@ -898,7 +898,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.idesc = idesc_bf16_f32(PM, 256, true, true);
       a.idesc_narrow = idesc_bf16_f32(PM, 128, true, true);
       ok &= make_map_bf16(&m0, ops.a0, Rr, d, 64);
-      if (dm.S > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, 64); else same(m1, m0);
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, 64); else same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, Rt, I, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
@@ -916,7 +916,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&m0, ops.a0, Rt, 2 * I, 64);
       same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, Rr, d, 64);
-      if (dm.S > 0) ok &= make_map_bf16(&n1, ops.b1, T, d, 64); else same(n1, n0);
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&n1, ops.b1, T, d, 64); else same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * 2 * I, d, 4, 32)) return MOE_ERR_CUDA;

@@ -115,7 +115,7 @@ int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, c
                      const void* w1, const void* w2, void* h, void* a1, void* y, void* stream) {
   int rc = check_shape(dims, false);
   if (rc) return rc;
-  if (!ws || !x_perm || !w1 || !w2 || !h || !y || (dims->S > 0 && !x)) return MOE_ERR_INVALID_ARG;
+  if (!ws || !x_perm || !w1 || !w2 || !h || !y || (dims->S > 0 && dims->T > 0 && !x)) return MOE_ERR_INVALID_ARG;
   GemmOperands o{};
   o.a0 = x_perm;
   o.a1 = x;
@@ -142,7 +142,7 @@ int grouped_gemm_bwd_dx(const moe_dims* dims, const void* ws, int which, const v
   o.b0 = w;
   o.out = out;
   if (which == MOE_GEMM2) {
-    if (!a1 || (dims->S > 0 && !dy_shared)) return MOE_ERR_INVALID_ARG;
+    if (!a1 || (dims->S > 0 && dims->T > 0 && !dy_shared)) return MOE_ERR_INVALID_ARG;
     o.a1 = dy_shared;
     o.aux = a1;
     return launch_grouped_gemm(MODE_DX2, *dims, ws, o, stream);
@@ -164,12 +164,12 @@ int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const v
   o.out = dw;
   o.accumulate = accumulate;
   if (which == MOE_GEMM2) {
-    if (dims->S > 0 && !lhs_shared) return MOE_ERR_INVALID_ARG;
+    if (dims->S > 0 && dims->T > 0 && !lhs_shared) return MOE_ERR_INVALID_ARG;
     o.a1 = lhs_shared;
     return launch_grouped_gemm(MODE_DW2, *dims, ws, o, stream);
   }
   if (which == MOE_GEMM1) {
-    if (dims->S > 0 && !rhs_shared) return MOE_ERR_INVALID_ARG;
+    if (dims->S > 0 && dims->T > 0 && !rhs_shared) return MOE_ERR_INVALID_ARG;
     o.b1 = rhs_shared;
     return launch_grouped_gemm(MODE_DW1, *dims, ws, o, stream);
   }

@@ -173,7 +173,7 @@ int grouped_gemm_set_groups(const moe_dims* dims, const int32_t* counts, int32_t
  * and §3.2 (one tile = one expert's aligned segment).
  *   ws       workspace holding the group table
  *   x_perm   [Rr, d] bf16  A rows of the routed groups
- *   x        [T, d]  bf16  A rows of the shared groups (may be NULL when S = 0)
+ *   x        [T, d]  bf16  A rows of the shared groups (may be NULL when S = 0 or T = 0)
  *   w1 [G, 2I, d] bf16, w2 [G, d, I] bf16
  * Out (grouped row space, rows of each group up to its padded size):
  *   h  [Rt, I]  bf16  H = silu(A W1g^T) * (A W1u^T), from the FP32 accumulator
@@ -187,7 +187,7 @@ int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, c
  *   which = MOE_GEMM2: dH = dY W2, then the SwiGLU backward with the saved a1:
  *       dG = dH * U * s * (1 + G (1 - s)), s = sigmoid(G);  dU = dH * silu(G)
  *     dy_routed [Rr, d] bf16 (from moe_combine_bwd), dy_shared [T, d] bf16 (the
- *     upstream gradient itself; may be NULL when S = 0), w = w2, a1 [Rt, 2I]
+ *     upstream gradient itself; may be NULL when S = 0 or T = 0), w = w2, a1 [Rt, 2I]
  *     -> out = dA [Rt, 2I] bf16 ([dG | dU])
  *   which = MOE_GEMM1: dX_perm = dA W1
  *     dy_routed = dA [Rt, 2I] bf16, dy_shared ignored, w = w1, a1 ignored
