@@ -39,7 +39,7 @@ def _gemm_only_case(dims: synth.Dims, group_rows, seed, w1_std, w2_std, check_ro
     moe.grouped_gemm_set_groups(dm, counts, offsets, ws)
     Rt = moe.moe_rows_total(dm)
     h = torch.full((Rt, I), float("nan"), dtype=torch.bfloat16, device="cuda")
-    a1 = torch.empty(Rt, 2 * I, dtype=torch.bfloat16, device="cuda")
+    a1 = torch.full((Rt, 2 * I), float("nan"), dtype=torch.bfloat16, device="cuda")
     y = torch.full((Rt, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     moe.grouped_gemm_fwd(dm, ws, dev(x_np, True), None, dev(w1, True), dev(w2, True), h, a1, y)
     torch.cuda.synchronize()
@@ -57,6 +57,7 @@ def _gemm_only_case(dims: synth.Dims, group_rows, seed, w1_std, w2_std, check_ro
         assert_close(Y[R], yy, f"Y group {e}")
     # every padded row of every group was written (no NaN left inside a segment)
     assert np.all(np.isfinite(H[:off[-1]])) and np.all(np.isfinite(Y[:off[-1]]))
+    assert np.all(np.isfinite(A1[:off[-1]]))
 
 
 def test_grouped_gemm_alone_16x512():
