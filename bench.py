@@ -60,6 +60,8 @@ def parse():
                              "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the step as eager C-ABI calls instead of a replayed CUDA graph")
     return ap.parse_args()
 
 
@@ -396,6 +398,22 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(status)}")
 
+    # The layer step as a CUDA graph of the same C-ABI calls (captured after the
+    # warm-up, replayed in the timed loop); the eager step is timed beside it.
+    use_graph = not args.eager and not (gate_only or gemm_only)
+    graph = None
+    if use_graph:
+        graph = layer.GraphStep(b, x, wg, bias, w1, w2, dout=dout if train else None,
+                                gamma=GAMMA if train else None)
+
+    def timed_steps(n):
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                if graph is not None:
+                    graph.replay()
+                else:
+                    step(stream)
+
     # ---- timed region: device-resident inputs
     clk = ClockSampler(local)
     clk.start()
@@ -405,8 +423,8 @@ def run_ours(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(args.steps):
-            step(stream)
+    timed_steps(args.steps)
+    with torch.cuda.stream(stream):
         e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize(dev)
@@ -414,6 +432,17 @@ def run_ours(args):
     clocks = clk.stop()
     ms = e0.elapsed_time(e1) / args.steps
     ms = dist_max(ms, world, dev)
+    ms_eager = None
+    if graph is not None:  # the same steps as eager calls, for comparison
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                step(stream)
+            e1.record(stream)
+        e1.synchronize()
+        ms_eager = dist_max(e0.elapsed_time(e1) / args.steps, world, dev)
     tokens_per_s = world * dm.T / (ms / 1000.0)
 
     # ---- per-call breakdown (separate instrumented pass; not the headline)
@@ -509,6 +538,8 @@ def run_ours(args):
         "config": {"workload": describe(wl), "tokens_per_gpu": dm.T,
                    "global_batch_tokens": world * dm.T,
                    "parallelism": "replicas" if world > 1 else "single GPU",
+                   "step": "CUDA graph replay" if graph is not None else "eager C-ABI calls",
+                   "ms_per_step_eager": ms_eager,
                    "l2": "no flush: weights (4.5 GB) and activations exceed the 126 MB L2"},
         "roofline": {"bound": "tensor", "kernel": "ggemm_kernel (all grouped-GEMM launches)",
                      "achieved": gemm_tflops, "peak": sustained, "unit": "TFLOP/s",

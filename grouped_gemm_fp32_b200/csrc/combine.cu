@@ -49,8 +49,10 @@ __global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __res
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     if (j < k) {
-      rows[j] = (int64_t)row_of[t * k + j] * row_vec;
-      wt[j] = w ? w[t * k + j] : 1.0f;
+      const int32_t r = row_of[t * k + j];
+      const bool ok = r >= 0 && r < Rr;  // -1 (a pick without a row) or stale: skipped
+      rows[j] = ok ? (int64_t)r * row_vec : 0;
+      wt[j] = ok ? (w ? w[t * k + j] : 1.0f) : 0.0f;
     } else if (j < k + S) {
       rows[j] = (Rr + (int64_t)(j - k) * T + t) * row_vec;
       wt[j] = 1.0f;
@@ -80,6 +82,7 @@ __global__ void combine_kernel_any(const uint4* __restrict__ y, const int32_t* _
     float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k + S; ++j) {
       const int64_t r = j < k ? (int64_t)row_of[t * k + j] : Rr + (int64_t)(j - k) * T + t;
+      if (j < k && (r < 0 || r >= Rr)) continue;  // a pick without a row
       acc8(a, y[r * row_vec + c], j < k ? (w ? w[t * k + j] : 1.0f) : 1.0f);
     }
     out[t * row_vec + c] = pack8(a);
@@ -89,7 +92,8 @@ __global__ void combine_kernel_any(const uint4* __restrict__ y, const int32_t* _
 // dy[row_of[t, j]] = w[t, j] dout[t] (bf16);  dw[t, j] = <dout[t], y[row_of[t, j]]>
 __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                                    const int32_t* __restrict__ row_of, const float* __restrict__ w,
-                                   int64_t T, int row_vec, int k, uint4* __restrict__ dy,
+                                   int64_t T, int row_vec, int k, int64_t Rr,
+                                   uint4* __restrict__ dy,
                                    float* __restrict__ dw) {
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -97,6 +101,10 @@ __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* 
   for (int j = 0; j < k; ++j) {
     const int64_t r = row_of[t * k + j];
     const float wj = w[t * k + j];
+    if (r < 0 || r >= Rr) {  // a pick without a row: nothing to scatter, no gradient
+      if (lane == 0) dw[t * k + j] = 0.0f;
+      continue;
+    }
     float dot = 0.0f;
     for (int c = lane; c < row_vec; c += 32) {
       const uint4 g = dout[t * row_vec + c];
@@ -123,7 +131,7 @@ __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* 
 template <int VPL>
 __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                                        const int32_t* __restrict__ row_of,
-                                       const float* __restrict__ w, int64_t T, int k,
+                                       const float* __restrict__ w, int64_t T, int k, int64_t Rr,
                                        uint4* __restrict__ dy, float* __restrict__ dw) {
   constexpr int row_vec = 32 * VPL;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -135,6 +143,10 @@ __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uin
   for (int j = 0; j < k; ++j) {
     const int64_t r = row_of[t * k + j];
     const float wj = w[t * k + j];
+    if (r < 0 || r >= Rr) {  // a pick without a row: nothing to scatter, no gradient
+      if (lane == 0) dw[t * k + j] = 0.0f;
+      continue;
+    }
     uint4 yv[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) yv[i] = y[r * row_vec + lane + 32 * i];
@@ -188,6 +200,7 @@ int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, con
   if (rc != MOE_OK || dm.T == 0) return rc;
   const int warps = 8;
   const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);
+  const int64_t Rr = rows_routed(dm);
   const uint4* dv = reinterpret_cast<const uint4*>(dout);
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* dyv = reinterpret_cast<uint4*>(dy);
@@ -195,12 +208,14 @@ int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, con
   // the register-resident form uses ~170 registers a thread: 4-warp CTAs, three per SM
   const unsigned blocks4 = (unsigned)((dm.T + 3) / 4);
   if (row_vec == 512)
-    combine_bwd_reg_kernel<16><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
+    combine_bwd_reg_kernel<16><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, Rr, dyv,
+                                                        dw);
   else if (row_vec == 256)
-    combine_bwd_reg_kernel<8><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, dyv, dw);
+    combine_bwd_reg_kernel<8><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, Rr, dyv,
+                                                       dw);
   else
-    combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, row_vec, dm.k, dyv,
-                                                      dw);
+    combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, row_vec, dm.k, Rr,
+                                                      dyv, dw);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -112,27 +112,43 @@ __device__ __forceinline__ void route_tile(const float* L, int LS, int64_t t0, i
       const bool valid = q < per && e < E;
       p[q] = valid ? p[q] * inv : 0.0f;
       s[q] = valid ? p[q] + (bias ? bias[e] : 0.0f) : -INFINITY;
+      if (s[q] != s[q]) s[q] = -INFINITY;  // a NaN score ranks last (ties by index)
       if (valid && probs) probs[t * E + e] = p[q];
     }
     float psel = 0.0f;
+    // experts this lane may still pick (a bit per q); a pick clears its bit
+    uint32_t alive = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < per && lane + 32 * q < E) alive |= 1u << q;
     for (int j = 0; j < k; ++j) {
-      // lane-local best: larger s, then lower index (q ascending = index ascending)
+      // lane-local best: larger s, then lower index (q ascending = index ascending).  The
+      // first live expert is taken before any comparison and NaN scores rank as -inf,
+      // so even non-finite inputs yield k distinct, valid experts.
       float bs = -INFINITY, bp = 0.0f;
       int be = 0x7fffffff;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        if (s[q] > bs) { bs = s[q]; be = lane + 32 * q; bp = p[q]; }
+        if (((alive >> q) & 1u) && (be == 0x7fffffff || s[q] > bs)) {
+          bs = s[q];
+          be = lane + 32 * q;
+          bp = p[q];
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float os = __shfl_xor_sync(0xffffffffu, bs, o);
         const int oe = __shfl_xor_sync(0xffffffffu, be, o);
         const float op = __shfl_xor_sync(0xffffffffu, bp, o);
-        if (os > bs || (os == bs && oe < be)) { bs = os; be = oe; bp = op; }
+        if (oe != 0x7fffffff && (be == 0x7fffffff || os > bs || (os == bs && oe < be))) {
+          bs = os;
+          be = oe;
+          bp = op;
+        }
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (lane + 32 * q == be) s[q] = -INFINITY;  // remove the winner
+        if (lane + 32 * q == be) alive &= ~(1u << q);  // remove the winner
       psel += bp;
       if (lane == 0) {
         topk_idx[t * k + j] = be;

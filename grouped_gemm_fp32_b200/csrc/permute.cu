@@ -153,7 +153,14 @@ __global__ void __launch_bounds__(kScatterThreads)
                    const int* header) {
   __shared__ int32_t running[256];
   __shared__ int32_t wcnt[kScatterThreads / 32][256];
-  if (header[3] != 1) return;  // group table flagged the routing as invalid
+  if (header[3] != 1) {
+    // the group table flagged the routing as invalid: no pick gets a row, and
+    // row_of says so (-1), so no later call follows a stale index
+    const int64_t base = (int64_t)blockIdx.x * kChunk;
+    for (int i = threadIdx.x; i < kChunk; i += kScatterThreads)
+      if (base + i < n) row_of[base + i] = -1;
+    return;
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += kScatterThreads) running[e] = 0;
   for (int i = tid; i < (kScatterThreads / 32) * 256; i += kScatterThreads) (&wcnt[0][0])[i] = 0;

@@ -182,3 +182,37 @@ class HostPipeline:
     def synchronize(self):
         for st in (self.up, self.compute, self.down):
             st.synchronize()
+
+
+class GraphStep:
+    """One layer step -- forward, and with ``dout`` the backward (router backward
+    and bias step included when ``gamma`` is given) -- captured once as a CUDA
+    graph and replayed.  Every node is one of the same C-ABI calls as in eager
+    mode, on the captured stream; the graph keeps the buffers' addresses, so new
+    inputs are written into ``x`` / ``dout`` in place before ``replay``.
+
+    The step runs once eagerly before the capture: the library's first calls set
+    kernel attributes and look up driver entry points, which must not happen
+    inside a capture."""
+
+    def __init__(self, b: MoEBuffers, x, wg, bias, w1, w2, dout=None, gamma=None):
+        self.b = b
+        self.stream = torch.cuda.Stream(device=x.device)
+        args = (b, x, wg, bias, w1, w2, dout, gamma)
+        with torch.cuda.stream(self.stream):
+            self._step(self.stream, *args)
+        self.stream.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            self._step(self.stream, *args)
+        self.stream.synchronize()
+
+    @staticmethod
+    def _step(s, b, x, wg, bias, w1, w2, dout, gamma):
+        forward(b, x, wg, bias, w1, w2, stream=s)
+        if dout is not None:
+            backward(b, x, dout, w1, w2, stream=s, wg=wg, gamma=gamma,
+                     bias=bias if gamma is not None else None)
+
+    def replay(self):
+        self.graph.replay()

@@ -106,7 +106,9 @@ size_t moe_workspace_size(const moe_dims* dims);
  * The logits are FP32 sums of exact FP32 products: each FP32 weight is split
  * exactly into three bf16 terms (hi + mid + lo, exact to below 2^-24 |w|),
  * x is bf16, and the tensor cores accumulate the products in FP32.  p uses
- * expf.  Requires E % 8 == 0, E <= 256, d % 64 == 0.  A bounded wait that runs
+ * expf.  Non-finite inputs cannot make an invalid choice: a NaN score ranks
+ * last (ties by index), so every token still names k distinct experts in
+ * [0, E).  Requires E % 8 == 0, E <= 256, d % 64 == 0.  A bounded wait that runs
  * out on the device sets MOE_ERR_DEVICE_TIMEOUT in the status word and leaves
  * the outputs of the affected tokens unwritten. */
 int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const float* bias,
@@ -130,7 +132,9 @@ int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const fl
  *   ws / ws_bytes               workspace (group table written here)
  * Deterministic: the same input gives the same output bit for bit.  An expert
  * id outside [0, E) or off_E > Rr sets MOE_ERR_BAD_ROUTING in the device
- * status and leaves an empty group table. */
+ * status, leaves an empty group table and sets every row_of entry to -1, so
+ * the combine calls below add nothing for those picks instead of following a
+ * stale row. */
 int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void* x,
                       int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* row_of,
                       void* x_perm, void* ws, size_t ws_bytes, void* stream);
@@ -155,7 +159,8 @@ int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void*
  *     device, with that device current); make that first call before any stream
  *     capture.
  *   - Routing errors (expert id outside [0, E), padded rows above Rr) leave
- *     sorted_ids at -1 and x_perm unwritten; no device status is kept. */
+ *     sorted_ids and row_of at -1 and x_perm unwritten; no device status is
+ *     kept. */
 int moe_permute_align_static(const moe_dims* dims, const int32_t* topk_idx, const void* x,
                              int32_t* counts, int32_t* offsets, int32_t* sorted_ids,
                              int32_t* row_of, void* x_perm, void* stream);
@@ -216,7 +221,9 @@ int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const v
  *   y [Rt, d] bf16 (grouped row space), row_of [T, k], topk_w [T, k] f32
  *   out[t] = sum_j topk_w[t, j] * y[row_of[t, j]] + sum_s y[Rr + s*T + t]
  * accumulated in FP32, stored bf16 into out [T, d].  topk_w = NULL uses weight 1
- * for every routed row: the un-permute-sum that turns dX rows into dX. */
+ * for every routed row: the un-permute-sum that turns dX rows into dX.  A pick
+ * whose row_of is outside [0, Rr) (-1 after a refused permutation) adds
+ * nothing. */
 int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,
                 void* out, void* stream);
 
@@ -226,7 +233,8 @@ int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, cons
  *   dy_routed [Rr, d] bf16   dy[row_of[t, j]] = topk_w[t, j] * dout[t];
  *                            pad rows of every segment set to zero
  *   dw        [T, k]  f32    dw[t, j] = sum_c dout[t, c] * y[row_of[t, j], c]
- * The shared experts' dY is dout itself (no copy). */
+ * The shared experts' dY is dout itself (no copy).  A pick whose row_of is
+ * outside [0, Rr) scatters nothing and gets dw = 0. */
 int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, const void* y,
                     const int32_t* row_of, const float* topk_w, void* dy_routed, float* dw,
                     void* stream);

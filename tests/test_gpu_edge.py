@@ -59,3 +59,61 @@ def test_all_experts_chosen_and_eight_shared():
     _, gdx, gdwg = oracle.router_bwd(inp["x"], inp["wg"], idx, rdw)
     assert_close(host(b.dx), rdx + gdx, "dx")
     assert_close(host(b.dwg), gdwg, "dWg")
+
+
+def test_nan_tokens_still_get_valid_distinct_experts():
+    # non-finite hidden states make NaN scores; the gate must still name k distinct,
+    # valid experts for them (so nothing downstream indexes out of range), and the
+    # finite tokens must route as the oracle does
+    wl = synth.Workload("edge_nan", synth.Dims(T=256, d=128, E=16, k=4, S=1, I=64, P=64),
+                        seed=23, w1_std=0.05, w2_std=0.05, wg_std=0.05, backward=True)
+    inp = synth.make_inputs(wl)
+    bad = [3, 77, 200]
+    inp["x"][bad, 5] = 0x7FC0  # bf16 NaN
+    dm = dims_of(wl)
+    b = layer.MoEBuffers(dm, train=True)
+    x, w1, w2 = dev(inp["x"], True), dev(inp["w1"], True), dev(inp["w2"], True)
+    wg = dev(inp["wg"])
+    layer.forward(b, x, wg, dev(inp["bias"]), w1, w2)
+    layer.backward(b, x, dev(inp["dout"], True), w1, w2, wg=wg)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(b.ws) == 0
+    idx = host(b.topk_idx)
+    assert idx.min() >= 0 and idx.max() < 16
+    assert all(len(set(r)) == 4 for r in idx)
+    good = np.setdiff1d(np.arange(256), bad)
+    _, oidx, _, margin = oracle.route(oracle.gate_logits(inp["x"][good], inp["wg"]), inp["bias"], 4)
+    same = np.all(np.sort(idx[good], axis=1) == np.sort(oidx, axis=1), axis=1)
+    assert np.all(same | (margin < 1e-5))
+
+
+def test_invalid_routing_leaves_no_stale_rows():
+    # a caller's routing with an expert id out of range: the permutation is refused
+    # (status MOE_ERR_BAD_ROUTING), every pick is marked row -1, and the combine and
+    # its backward then add only the shared experts and give the picks no gradient
+    T, d, E, k, S = 64, 128, 8, 2, 1
+    dm = moe.MoeDims.of(T, d, E, k, S, 64, 16)
+    ws = torch.zeros(moe.moe_workspace_size(dm), dtype=torch.uint8, device="cuda")
+    idx = np.tile(np.array([[0, 1]], np.int32), (T, 1))
+    idx[9, 0] = 40
+    Rr, Rt = moe.moe_rows_routed(dm), moe.moe_rows_total(dm)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sorted_ids = torch.empty(Rr, dtype=torch.int32, device="cuda")
+    row_of = torch.full((T, k), 123456, dtype=torch.int32, device="cuda")  # stale garbage
+    x_perm = torch.zeros(Rr, d, dtype=torch.bfloat16, device="cuda")
+    x = dev(synth.normal_bf16(3, 1, (T, d), 1.0), True)
+    moe.moe_permute_align(dm, dev(idx), x, counts, offsets, sorted_ids, row_of, x_perm, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == -5
+    assert torch.all(row_of == -1)
+    y = dev(synth.normal_bf16(3, 2, (Rt, d), 1.0), True)
+    w = torch.full((T, k), 0.5, dtype=torch.float32, device="cuda")
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(dm, y, row_of, w, out)
+    dy = torch.zeros(Rr, d, dtype=torch.bfloat16, device="cuda")
+    dwc = torch.full((T, k), 9.0, dtype=torch.float32, device="cuda")
+    moe.moe_combine_bwd(dm, ws, x, y, row_of, w, dy, dwc)
+    torch.cuda.synchronize()
+    assert torch.equal(out, y[Rr:Rr + T])  # only the shared expert's rows
+    assert torch.all(dwc == 0) and torch.all(dy == 0)
