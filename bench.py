@@ -490,7 +490,7 @@ def run_ours(args):
         e2e_note = "inputs H2D and results D2H every step, serialised with compute"
     else:
         pipe = layer.HostPipeline(dims, w1, w2, wg, bias, train, device=dev,
-                                  gamma=GAMMA if train else None)
+                                  gamma=GAMMA if train else None, graphs=not args.eager)
         hx = [pinned(inp["x"])]
         hd = [pinned(inp["dout"])] if train else [None]
         ho = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]

@@ -123,13 +123,14 @@ class HostPipeline:
     """
 
     def __init__(self, dims: L.MoeDims, w1, w2, wg, bias, train: bool, device="cuda",
-                 gamma=None):
+                 gamma=None, graphs: bool = True):
         self.dims, self.train, self.gamma = dims, train, gamma
         self.w1, self.w2, self.wg, self.bias = w1, w2, wg, bias
         dev = torch.device(device)
         T, d = dims.T, dims.d
         self.bufs = [MoEBuffers(dims, device=dev, train=train) for _ in range(2)]
-        e = lambda: torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        # zero-filled: with graphs, one step runs on them before the capture
+        e = lambda: torch.zeros(T, d, dtype=torch.bfloat16, device=dev)
         self.x = [e(), e()]
         self.dout = [e(), e()] if train else [None, None]
         self.compute = torch.cuda.Stream(device=dev)
@@ -141,6 +142,12 @@ class HostPipeline:
         self.consumed = [torch.cuda.Event(), torch.cuda.Event()]
         for ev in self.downloaded + self.consumed:
             ev.record(self.compute)
+        # one captured step per buffer set (the graphs keep the sets' addresses)
+        self.graphs = None
+        if graphs:
+            self.graphs = [GraphStep(self.bufs[j], self.x[j], wg, bias, w1, w2,
+                                     dout=self.dout[j] if train else None,
+                                     gamma=gamma if train else None) for j in range(2)]
 
     def _upload(self, j, hx, hd):
         with torch.cuda.stream(self.up):
@@ -166,10 +173,13 @@ class HostPipeline:
             with torch.cuda.stream(s):
                 s.wait_event(self.uploaded[j])
                 s.wait_event(self.downloaded[j])  # results of step i-2 have left set j
-                forward(b, self.x[j], self.wg, self.bias, self.w1, self.w2, stream=s)
-                if self.train:
-                    backward(b, self.x[j], self.dout[j], self.w1, self.w2, stream=s,
-                             wg=self.wg, gamma=self.gamma, bias=self.bias)
+                if self.graphs is not None:
+                    self.graphs[j].replay()
+                else:
+                    forward(b, self.x[j], self.wg, self.bias, self.w1, self.w2, stream=s)
+                    if self.train:
+                        backward(b, self.x[j], self.dout[j], self.w1, self.w2, stream=s,
+                                 wg=self.wg, gamma=self.gamma, bias=self.bias)
                 self.computed[j].record(s)
                 self.consumed[j].record(s)
             with torch.cuda.stream(self.down):

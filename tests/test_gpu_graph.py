@@ -42,3 +42,31 @@ def test_graph_replay_matches_eager(case):
         assert moe.moe_get_device_status(b.ws) == 0
         for k in KEYS:
             assert torch.equal(getattr(b, k), ref[k]), k
+
+
+@pytest.mark.parametrize("graphs", [True, False], ids=["graphs", "eager"])
+def test_host_pipeline_matches_eager_steps(graphs):
+    # three different batches through the double-buffered host pipeline: every host
+    # output equals an eager forward/backward of that batch
+    wl = SMALL
+    inp = synth.make_inputs(wl)
+    dm = dims_of(wl)
+    w1, w2 = dev(inp["w1"], True), dev(inp["w2"], True)
+    wg, bias = dev(inp["wg"]), dev(inp["bias"])
+    xs = [synth.normal_bf16(40 + i, 1, (dm.T, dm.d), 1.0) for i in range(3)]
+    ds = [synth.normal_bf16(50 + i, 6, (dm.T, dm.d), 1.0) for i in range(3)]
+    pin = lambda a: torch.from_numpy(a).view(torch.bfloat16).pin_memory()
+    hx, hd = [pin(a) for a in xs], [pin(a) for a in ds]
+    ho = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    hdx = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    pipe = layer.HostPipeline(dm, w1, w2, wg, bias, True, gamma=1e-3, graphs=graphs)
+    pipe.run(hx, hd, ho, hdx, 3)
+    pipe.synchronize()
+    b = layer.MoEBuffers(dm, train=True)
+    for i in range(3):
+        x, dout = dev(xs[i], True), dev(ds[i], True)
+        layer.forward(b, x, wg, bias, w1, w2)
+        layer.backward(b, x, dout, w1, w2, wg=wg, gamma=1e-3, bias=bias)
+        torch.cuda.synchronize()
+        assert torch.equal(ho[i], b.out.cpu()), i
+        assert torch.equal(hdx[i], b.dx.cpu()), i
