@@ -117,3 +117,38 @@ def test_invalid_routing_leaves_no_stale_rows():
     torch.cuda.synchronize()
     assert torch.equal(out, y[Rr:Rr + T])  # only the shared expert's rows
     assert torch.all(dwc == 0) and torch.all(dy == 0)
+
+
+def test_256_experts_full_layer():
+    # E = 256 routed experts (the largest supported) + 2 shared: G = 258 groups, many of
+    # them short or empty; forward, backward and the router backward against the oracle
+    # with the oracle's routing injected
+    wl = synth.Workload("edge_e256", synth.Dims(T=1024, d=256, E=256, k=8, S=2, I=128, P=64),
+                        seed=25, w1_std=0.05, w2_std=0.05, wg_std=0.05, backward=True)
+    inp = synth.make_inputs(wl)
+    dm = dims_of(wl)
+    p, oidx, ow, _ = oracle.route(oracle.gate_logits(inp["x"], inp["wg"]), inp["bias"], 8)
+    b = layer.MoEBuffers(dm, train=True)
+    x, w1, w2 = dev(inp["x"], True), dev(inp["w1"], True), dev(inp["w2"], True)
+    wg = dev(inp["wg"])
+    out = layer.forward(b, x, wg, dev(inp["bias"]), w1, w2,
+                        routing=(dev(oidx), dev(ow.astype(np.float32)), dev(p.astype(np.float32))))
+    layer.backward(b, x, dev(inp["dout"], True), w1, w2, wg=wg)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(b.ws) == 0
+    assert host(b.counts).sum() == 1024 * 8  # no token dropped
+    toks = np.arange(0, 1024, 7)
+    ref = oracle.layer_fwd(inp["x"], oidx, ow, inp["w1"], inp["w2"], 2, tokens=toks)
+    assert_close(host(out)[toks], ref, "out")
+    rdx, rdw = oracle.layer_bwd(inp["x"], oidx, ow, inp["w1"], inp["w2"], inp["dout"], 2)
+    _, gdx, gdwg = oracle.router_bwd(inp["x"], inp["wg"], oidx, rdw)
+    assert_close(host(b.dx), rdx + gdx, "dx")
+    assert_close(host(b.dwg), gdwg, "dWg")
+    DW1, DW2 = host(b.dw1), host(b.dw2)
+    for g in (0, 97, 255, 256, 257):  # routed groups and both shared groups
+        r1, r2 = oracle.group_dw(inp["x"], oidx, ow, inp["w1"], inp["w2"], inp["dout"], 2, g)
+        if np.max(np.abs(r1)) == 0:
+            assert np.all(DW1[g] == 0) and np.all(DW2[g] == 0)
+            continue
+        assert_close(DW1[g], r1, f"dW1[{g}]")
+        assert_close(DW2[g], r2, f"dW2[{g}]")
