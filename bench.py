@@ -232,8 +232,8 @@ def barrier(world):
 # --------------------------------------------------------------- CPU (oracle) --
 def oracle_sample_step(wl, inp, ntok):
     """The oracle on the first ``ntok`` tokens of the workload: gate + route +
-    permute + expert forward (+ backward incl. every group's dW when the
-    workload trains).  Returns seconds."""
+    permute + expert forward (+ backward incl. every group's dW, the router
+    backward and the bias step when the workload trains).  Returns seconds."""
     import oracle
     dm = wl.dims
     x = inp["x"][:ntok]
@@ -244,17 +244,23 @@ def oracle_sample_step(wl, inp, ntok):
     oracle.layer_fwd(x, idx, w, inp["w1"], inp["w2"], dm.S)
     if wl.backward:
         dout = inp["dout"][:ntok]
-        oracle.layer_bwd(x, idx, w, inp["w1"], inp["w2"], dout, dm.S)
+        _, dw = oracle.layer_bwd(x, idx, w, inp["w1"], inp["w2"], dout, dm.S)
         used = set(np.unique(idx).tolist()) | set(range(dm.E, dm.E + dm.S))
         for g in sorted(used):
             oracle.group_dw(x, idx, w, inp["w1"], inp["w2"], dout, dm.S, g)
+        oracle.router_bwd(x, inp["wg"], idx, dw)
+        oracle.bias_update(idx, dm.E, inp["bias"], GAMMA)
     return time.perf_counter() - t0
 
 
-def cpu_baseline(wl, inp, ntok=64):
+def cpu_baseline(wl, inp, target_s=15.0):
+    """The oracle on a sample of the workload's tokens sized for about ``target_s``
+    seconds of host work (a 16-token probe sets the size)."""
     import oracle
     oracle.build()
     oracle_sample_step(wl, inp, 2)  # warm the library and the page cache
+    probe = oracle_sample_step(wl, inp, 16)
+    ntok = int(min(wl.dims.T, max(16, 16 * target_s / max(probe, 1e-6))))
     secs = oracle_sample_step(wl, inp, ntok)
     return {"value": ntok / secs, "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
