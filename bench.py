@@ -253,9 +253,10 @@ def oracle_sample_step(wl, inp, ntok):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(wl, inp, target_s=15.0):
-    """The oracle on a sample of the workload's tokens sized for about ``target_s``
-    seconds of host work (a 16-token probe sets the size)."""
+def cpu_baseline(wl, inp, target_s=20.0):
+    """The oracle on a sample of the workload's tokens sized from a 16-token probe
+    for ``target_s`` seconds of host work (the probe overstates the per-token
+    cost, so the sample itself takes less: about 10-15 s)."""
     import oracle
     oracle.build()
     oracle_sample_step(wl, inp, 2)  # warm the library and the page cache
@@ -265,7 +266,7 @@ def cpu_baseline(wl, inp, target_s=15.0):
     return {"value": ntok / secs, "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"first {ntok} tokens of the workload, full "
-                      f"{'forward+backward (all dW)' if wl.backward else 'forward'} in FP64, "
+                      f"{'forward+backward (all dW, router backward, bias step)' if wl.backward else 'forward'} in FP64, "
                       f"{secs:.1f} s; tokens/s scales linearly in tokens"}
 
 
