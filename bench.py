@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="time the step as eager C-ABI calls instead of a replayed CUDA graph")
+    ap.add_argument("--gather", action="store_true",
+                    help="the first GEMM and dW1 gather x rows through sorted_ids instead of "
+                         "reading the permuted copy x_perm")
     return ap.parse_args()
 
 
@@ -334,7 +337,7 @@ def run_ours(args):
             out = torch.empty(dm.T, dm.d, dtype=torch.bfloat16, device=dev)
         b = _GateBufs()
     else:
-        b = layer.MoEBuffers(dims, device=dev, train=train)
+        b = layer.MoEBuffers(dims, device=dev, train=train, gather=args.gather)
     if gemm_only:
         counts = torch.tensor(wl.group_rows, dtype=torch.int32, device=dev)
         moe.grouped_gemm_set_groups(dims, counts, b.offsets, b.ws)
@@ -374,7 +377,10 @@ def run_ours(args):
         L.moe_permute_align(dims, b.topk_idx, xx, b.counts, b.offsets, b.sorted_ids, b.row_of,
                             b.x_perm, b.ws, s)
         rec("permute")
-        L.grouped_gemm_fwd(dims, b.ws, b.x_perm, xx, w1, w2, b.h, b.a1, b.y, s)
+        if b.gather:
+            L.grouped_gemm_fwd_gather(dims, b.ws, b.sorted_ids, xx, w1, w2, b.h, b.a1, b.y, s)
+        else:
+            L.grouped_gemm_fwd(dims, b.ws, b.x_perm, xx, w1, w2, b.h, b.a1, b.y, s)
         rec("fwd")
         L.moe_combine(dims, b.y, b.row_of, b.topk_w, b.out, s)
         rec("combine")
@@ -387,7 +393,11 @@ def run_ours(args):
             rec("dw2")
             L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, s)
             rec("dx1")
-            L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, xx, b.dw1, 0, s)
+            if b.gather:
+                L.grouped_gemm_bwd_dw1_gather(dims, b.ws, b.sorted_ids, b.da, xx, b.dw1, 0, s)
+            else:
+                L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, xx, b.dw1,
+                                      0, s)
             rec("dw1")
             L.moe_combine(dims, b.dxp, b.row_of, None, b.dx, s)
             rec("unpermute")
@@ -497,7 +507,8 @@ def run_ours(args):
         e2e_note = "inputs H2D and results D2H every step, serialised with compute"
     else:
         pipe = layer.HostPipeline(dims, w1, w2, wg, bias, train, device=dev,
-                                  gamma=GAMMA if train else None, graphs=not args.eager)
+                                  gamma=GAMMA if train else None, graphs=not args.eager,
+                                  gather=args.gather)
         hx = [pinned(inp["x"])]
         hd = [pinned(inp["dout"])] if train else [None]
         ho = [torch.empty(dm.T, dm.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -532,11 +543,13 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after timing: {moe.moe_status_string(status)}")
 
-    # kernels per step: gate 2 (weight split, gate), permute 5, forward GEMMs 2, combine 1;
+    # kernels per step: gate 2 (weight split, gate), permute 3 (histogram, groups,
+    # scatter; + row copy and pad zeroing without gathering), forward GEMMs 2, combine 1;
     # train adds combine backward 2, backward GEMMs 4, un-permute 1, router backward 5
     # (weight split, dlogits, dX GEMM, dWg GEMM, split-K sum), bias step 1
+    permute_launches = 3 if args.gather else 5
     launches_per_step = (2 if gate_only else 2 if gemm_only else
-                         2 + 5 + 2 + 1 + ((2 + 4 + 1 + 5 + 1) if train else 0))
+                         2 + permute_launches + 2 + 1 + ((2 + 4 + 1 + 5 + 1) if train else 0))
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -546,6 +559,8 @@ def run_ours(args):
                    "global_batch_tokens": world * dm.T,
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "step": "CUDA graph replay" if graph is not None else "eager C-ABI calls",
+                   "x_rows": ("gathered from x by sorted_ids (tile::gather4)" if args.gather
+                              else "permuted copy x_perm"),
                    "ms_per_step_eager": ms_eager,
                    "l2": "no flush: weights (4.5 GB) and activations exceed the 126 MB L2"},
         "roofline": {"bound": "tensor", "kernel": "ggemm_kernel (all grouped-GEMM launches)",

@@ -7,7 +7,8 @@ caller-owned torch buffers (``grouped_gemm_fp32_b200.layer``).  There is no
 CPU or PyTorch fallback: without the built library every call raises.
 """
 from ._lib import (MOE_GEMM1, MOE_GEMM2, MoeDims, MoeError, grouped_gemm_bwd_dw,  # noqa: F401
-                   grouped_gemm_bwd_dx, grouped_gemm_fwd, grouped_gemm_set_groups, lib_path,
+                   grouped_gemm_bwd_dw1_gather, grouped_gemm_bwd_dx, grouped_gemm_fwd,
+                   grouped_gemm_fwd_gather, grouped_gemm_set_groups, lib_path,
                    load, moe_bias_update, moe_combine, moe_combine_bwd, moe_gate_topk,
                    moe_get_device_status, moe_last_cuda_error, moe_permute_align,
                    moe_permute_align_static, moe_router_bwd, moe_rows_routed, moe_rows_total,

@@ -17,7 +17,8 @@ MOE_GEMM1, MOE_GEMM2 = 1, 2
 EXPORTS = (
     "moe_rows_routed", "moe_rows_total", "moe_workspace_size", "moe_gate_topk",
     "moe_permute_align", "moe_permute_align_static", "grouped_gemm_set_groups",
-    "grouped_gemm_fwd", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw", "moe_combine",
+    "grouped_gemm_fwd", "grouped_gemm_fwd_gather", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw",
+    "grouped_gemm_bwd_dw1_gather", "moe_combine",
     "moe_combine_bwd", "moe_router_bwd", "moe_bias_update", "moe_get_device_status",
     "moe_status_string", "moe_last_cuda_error",
 )
@@ -70,7 +71,9 @@ def load():
         "moe_permute_align_static": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "grouped_gemm_set_groups": (i32, [D, vp, vp, vp, sz, vp]),
         "grouped_gemm_fwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "grouped_gemm_fwd_gather": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "grouped_gemm_bwd_dx": (i32, [D, vp, i32, vp, vp, vp, vp, vp, vp]),
+        "grouped_gemm_bwd_dw1_gather": (i32, [D, vp, vp, vp, vp, vp, i32, vp]),
         "grouped_gemm_bwd_dw": (i32, [D, vp, i32, vp, vp, vp, vp, vp, i32, vp]),
         "moe_combine": (i32, [D, vp, vp, vp, vp, vp]),
         "moe_router_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
@@ -164,6 +167,12 @@ def grouped_gemm_fwd(dims, ws, x_perm, x, w1, w2, h, a1, y, stream=None):
                                 _p(h), _p(a1), _p(y), _s(stream)), "grouped_gemm_fwd")
 
 
+def grouped_gemm_fwd_gather(dims, ws, sorted_ids, x, w1, w2, h, a1, y, stream=None):
+    _ck(load().grouped_gemm_fwd_gather(ctypes.byref(dims), _p(ws), _p(sorted_ids), _p(x), _p(w1),
+                                       _p(w2), _p(h), _p(a1), _p(y), _s(stream)),
+        "grouped_gemm_fwd_gather")
+
+
 def grouped_gemm_bwd_dx(dims, ws, which, dy_routed, dy_shared, w, a1, out, stream=None):
     _ck(load().grouped_gemm_bwd_dx(ctypes.byref(dims), _p(ws), int(which), _p(dy_routed),
                                    _p(dy_shared), _p(w), _p(a1), _p(out), _s(stream)),
@@ -175,6 +184,12 @@ def grouped_gemm_bwd_dw(dims, ws, which, lhs_routed, lhs_shared, rhs_routed, rhs
     _ck(load().grouped_gemm_bwd_dw(ctypes.byref(dims), _p(ws), int(which), _p(lhs_routed),
                                    _p(lhs_shared), _p(rhs_routed), _p(rhs_shared), _p(dw),
                                    int(accumulate), _s(stream)), "grouped_gemm_bwd_dw")
+
+
+def grouped_gemm_bwd_dw1_gather(dims, ws, sorted_ids, da, x, dw1, accumulate=0, stream=None):
+    _ck(load().grouped_gemm_bwd_dw1_gather(ctypes.byref(dims), _p(ws), _p(sorted_ids), _p(da),
+                                           _p(x), _p(dw1), int(accumulate), _s(stream)),
+        "grouped_gemm_bwd_dw1_gather")
 
 
 def moe_combine(dims, y, row_of, topk_w, out, stream=None):

@@ -34,6 +34,7 @@
 
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 
 #include "moe_internal.cuh"
 #include "sm100.cuh"
@@ -77,6 +78,8 @@ struct GemmArgs {
   uint32_t idesc_narrow;  // N = 128 (modes whose B is N-major)
   int staged;             // epilogue writes through shared memory + TMA stores
   uint64_t budget_ns;
+  const int32_t* gather_ids;  // FWD1 / DW1: token of each routed row, or null
+  int gather_T;               // rows of the gathered tensor x
 };
 
 // full[] and tempty[] are used in the leader CTA only (both CTAs' producers and
@@ -111,6 +114,29 @@ struct TileInfo {
 __device__ __forceinline__ GroupRec load_group(const GemmArgs& a, int g) {
   const int4 v = __ldg(reinterpret_cast<const int4*>(a.groups) + g);
   return GroupRec{v.x, v.y, v.z, v.w};
+}
+
+// Gathered x rows.  Every row a gather copies must lie inside x, so rows that
+// hold no token -- pad rows (id -1), rows past the group's padded end, and ids
+// outside [0, T) -- read the group's first token instead.  Their products are
+// never used: pad rows' forward results are not read, and their upstream
+// gradients are zero in the backward, so they add nothing to dW.
+__device__ __forceinline__ int gather_first(const GemmArgs& a, const GroupRec& gr) {
+  const int id = __ldg(a.gather_ids + gr.a_row);
+  return (id >= 0 && id < a.gather_T) ? id : 0;
+}
+
+// Tokens of the group's rows local .. local + 3.
+__device__ __forceinline__ int4 gather_rows4(const GemmArgs& a, const GroupRec& gr, int local,
+                                             int first) {
+  int v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int r = local + j;
+    const int id = r < gr.rows_pad ? __ldg(a.gather_ids + gr.a_row + r) : -1;
+    v[j] = (id >= 0 && id < a.gather_T) ? id : first;
+  }
+  return make_int4(v[0], v[1], v[2], v[3]);
 }
 
 template <int MODE>
@@ -302,7 +328,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0) {
+    // Lane 0 waits for free stages, arms the leader's full barrier and issues the
+    // tile copies.  With gathered x rows (FWD1's routed A, DW1's routed B) all 32
+    // lanes issue four-row gathers of the same stage as well.
+    constexpr bool CAN_GATHER = (MODE == MODE_FWD1 || MODE == MODE_DW1);
+    // one loop, compiled twice: WIDE (all lanes, gathers) and lane 0 alone
+    auto produce = [&](auto wide_tag) {
+      constexpr bool WIDE = decltype(wide_tag)::value;
       int stage = 0;
       uint32_t phase = 0, issued = 0, lastpar = 0;
       const int roff = (int)rank * BM;                       // this CTA's 128 rows of A
@@ -311,30 +343,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const TileInfo t = decode_tile<MODE>(tile, args);
         const GroupRec gr = load_group(args, t.g);
         const bool shared = t.g >= args.E;
+        const bool gat = WIDE && !shared;
         // this CTA's half of B: N/2 columns from n0 + rank * N/2, in 64-column chunks
         const int bchunks = t.nw / 128;
-        const int boff = (int)rank * (t.nw / 2);
+        [[maybe_unused]] const int boff = (int)rank * (t.nw / 2);
         const uint32_t b_bytes = (MODE == MODE_FWD1) ? (uint32_t)(args.hn * BK * 2)
                                  : B_MN ? (uint32_t)(bchunks * 8192) : (uint32_t)B_BYTES;
         const uint32_t pair_bytes = 2 * (A_BYTES + b_bytes);  // both CTAs' copies
+        int first = 0;
+        int4 rows4 = make_int4(0, 0, 0, 0);  // the four x rows this lane gathers
+        if (gat) {
+          first = gather_first(args, gr);
+          // FWD1: rows 4 lane .. 4 lane + 3 of this CTA's 128, fixed over the K loop;
+          // DW1: rows 4 (lane % 16) .. of the first K block (then one block ahead)
+          rows4 = gather_rows4(args, gr, MODE == MODE_FWD1 ? t.m0 + roff + 4 * lane
+                                                           : 4 * (lane & 15), first);
+        }
         for (int kb = 0; kb < t.nkb; ++kb) {
-          if (!mbar_wait(&ctl->empty[stage], phase ^ 1, abort_flag, args.status,
-                         MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
-            abort_pair();
+          int got = 1;
+          if (lane == 0)
+            got = mbar_wait(&ctl->empty[stage], phase ^ 1, abort_flag, args.status,
+                            MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
+          if constexpr (WIDE) got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            if (lane == 0) abort_pair();
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&ctl->full[stage], pair_bytes);
+          if (leader && lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], pair_bytes);
           const uint32_t fb = map_to_rank(&ctl->full[stage], 0);
           uint8_t* a_dst = sA + stage * A_BYTES;
           uint8_t* b_dst = sB + stage * B_BYTES;
           const int k0 = kb * BK;
           if constexpr (MODE == MODE_FWD1) {
             // A: rows m0 + roff; B: the leader stages the gate rows, the peer the up rows
-            tma_load_2d_pair(a_dst, shared ? &tmA1 : &tmA0, fb, k0,
-                             (shared ? 0 : gr.a_row) + t.m0 + roff);
-            tma_load_2d_pair(b_dst, &tmB0, fb, k0,
-                             t.g * args.b_group_rows + t.n0 + (leader ? 0 : args.I));
+            if (gat)
+              tma_gather4_pair(a_dst + lane * 512, &tmA0, fb, k0, rows4.x, rows4.y, rows4.z,
+                               rows4.w);
+            if (lane == 0) {
+              if (!gat)
+                tma_load_2d_pair(a_dst, shared ? &tmA1 : &tmA0, fb, k0,
+                                 (shared ? 0 : gr.a_row) + t.m0 + roff);
+              tma_load_2d_pair(b_dst, &tmB0, fb, k0,
+                               t.g * args.b_group_rows + t.n0 + (leader ? 0 : args.I));
+            }
           } else if constexpr (MODE == MODE_FWD2) {
             tma_load_2d_pair(a_dst, &tmA0, fb, k0, gr.out_row + t.m0 + roff);
             tma_load_2d_pair(b_dst, &tmB0, fb, k0, t.g * args.b_group_rows + t.n0 + roff);
@@ -374,11 +426,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               mb = shared ? &tmB1 : &tmB0;
               brow = shared ? 0 : gr.a_row;
             }
+            if (lane == 0) {
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-              tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
-            for (int c = 0; c < bchunks; ++c)
-              tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + boff + c * 64, brow + k0);
+              for (int c = 0; c < 2; ++c)
+                tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
+              if (!gat)
+                for (int c = 0; c < bchunks; ++c)
+                  tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + boff + c * 64, brow + k0);
+            }
+            if constexpr (MODE == MODE_DW1) {
+              if (gat) {
+                // lanes 0..15: 64-column chunk 0, lanes 16..31: chunk 1; lane i % 16
+                // brings K rows 4 i .. 4 i + 3 of this block
+                const int c = lane >> 4;
+                if (c < bchunks)
+                  tma_gather4_pair(b_dst + c * 8192 + (lane & 15) * 512, mb, fb,
+                                   t.n0 + boff + c * 64, rows4.x, rows4.y, rows4.z, rows4.w);
+                if (kb + 1 < t.nkb) rows4 = gather_rows4(args, gr, k0 + BK + 4 * (lane & 15), first);
+              }
+            }
           }
           issued |= 1u << stage;
           lastpar = (lastpar & ~(1u << stage)) | (phase << stage);
@@ -390,13 +456,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
       // The leader's full barriers count both CTAs' copies: once they have
       // completed, every copy either CTA started has landed.
-      if (leader)
+      if (leader && lane == 0)
         for (int s = 0; s < STAGES; ++s)
           if (issued & (1u << s)) {
             volatile int never = 0;
             mbar_wait(&ctl->full[s], (lastpar >> s) & 1u, &never, args.status,
                       MOE_ERR_DEVICE_TIMEOUT, drain_budget);
           }
+    };
+    if (CAN_GATHER && args.gather_ids != nullptr) {
+      if constexpr (CAN_GATHER) produce(std::true_type{});
+    } else if (lane == 0) {
+      produce(std::false_type{});
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer (leader) --
@@ -826,10 +897,17 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.ld_out = I;
       a.ld_out2 = 2 * I;
       a.idesc = idesc_bf16_f32(PM, 2 * hn, false, false);
-      ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
-      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, hn);
       same(n1, n0);
+      if (ops.gather_ids != nullptr) {
+        // routed A rows gathered from x, one-row boxes (four rows a copy)
+        a.gather_ids = ops.gather_ids;
+        a.gather_T = (int)T;
+        if (T > 0) ok &= make_map_bf16(&m0, ops.a1, T, d, 1); else same(m0, n0);
+      } else {
+        ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
+      }
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
       if (!ok) return MOE_ERR_CUDA;
       // staged stores need 64 H columns per epilogue warp
       a.staged = hn == 128;
@@ -915,7 +993,14 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.idesc_narrow = idesc_bf16_f32(PM, 128, true, true);
       ok &= make_map_bf16(&m0, ops.a0, Rt, 2 * I, 64);
       same(m1, m0);
-      ok &= make_map_bf16(&n0, ops.b0, Rr, d, 64);
+      if (ops.gather_ids != nullptr) {
+        // routed x rows (the reduction's K rows) gathered, four a copy
+        a.gather_ids = ops.gather_ids;
+        a.gather_T = (int)T;
+        if (T > 0) ok &= make_map_bf16(&n0, ops.b1, T, d, 1); else same(n0, m0);
+      } else {
+        ok &= make_map_bf16(&n0, ops.b0, Rr, d, 64);
+      }
       if (dm.S > 0 && T > 0) ok &= make_map_bf16(&n1, ops.b1, T, d, 64); else same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;

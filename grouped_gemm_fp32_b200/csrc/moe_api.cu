@@ -98,7 +98,7 @@ int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void*
   int rc = check_shape(dims, false);
   if (rc) return rc;
   if (!counts || !offsets || !sorted_ids || !ws_ok(dims, ws, ws_bytes)) return MOE_ERR_INVALID_ARG;
-  if (dims->T > 0 && (!topk_idx || !x || !row_of || !x_perm)) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!topk_idx || !row_of || (x_perm && !x))) return MOE_ERR_INVALID_ARG;
   return launch_permute(*dims, topk_idx, x, counts, offsets, sorted_ids, row_of, x_perm, ws,
                         stream);
 }
@@ -111,24 +111,41 @@ int grouped_gemm_set_groups(const moe_dims* dims, const int32_t* counts, int32_t
   return launch_set_groups(*dims, counts, offsets, ws, stream);
 }
 
-int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, const void* x,
-                     const void* w1, const void* w2, void* h, void* a1, void* y, void* stream) {
-  int rc = check_shape(dims, false);
-  if (rc) return rc;
-  if (!ws || !x_perm || !w1 || !w2 || !h || !y || (dims->S > 0 && dims->T > 0 && !x)) return MOE_ERR_INVALID_ARG;
+// FWD1 then FWD2; routed A rows from x_perm, or gathered from x by sorted_ids.
+static int gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm,
+                    const int32_t* sorted_ids, const void* x, const void* w1, const void* w2,
+                    void* h, void* a1, void* y, void* stream) {
   GemmOperands o{};
   o.a0 = x_perm;
   o.a1 = x;
   o.b0 = w1;
   o.out = h;
   o.out2 = a1;
-  rc = launch_grouped_gemm(MODE_FWD1, *dims, ws, o, stream);
+  o.gather_ids = sorted_ids;
+  int rc = launch_grouped_gemm(MODE_FWD1, *dims, ws, o, stream);
   if (rc) return rc;
   GemmOperands o2{};
   o2.a0 = h;
   o2.b0 = w2;
   o2.out = y;
   return launch_grouped_gemm(MODE_FWD2, *dims, ws, o2, stream);
+}
+
+int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, const void* x,
+                     const void* w1, const void* w2, void* h, void* a1, void* y, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!ws || !x_perm || !w1 || !w2 || !h || !y || (dims->S > 0 && dims->T > 0 && !x)) return MOE_ERR_INVALID_ARG;
+  return gemm_fwd(dims, ws, x_perm, nullptr, x, w1, w2, h, a1, y, stream);
+}
+
+int grouped_gemm_fwd_gather(const moe_dims* dims, const void* ws, const int32_t* sorted_ids,
+                            const void* x, const void* w1, const void* w2, void* h, void* a1,
+                            void* y, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!ws || !sorted_ids || !w1 || !w2 || !h || !y || (dims->T > 0 && !x)) return MOE_ERR_INVALID_ARG;
+  return gemm_fwd(dims, ws, nullptr, sorted_ids, x, w1, w2, h, a1, y, stream);
 }
 
 int grouped_gemm_bwd_dx(const moe_dims* dims, const void* ws, int which, const void* dy_routed,
@@ -174,6 +191,23 @@ int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const v
     return launch_grouped_gemm(MODE_DW1, *dims, ws, o, stream);
   }
   return MOE_ERR_INVALID_ARG;
+}
+
+int grouped_gemm_bwd_dw1_gather(const moe_dims* dims, const void* ws, const int32_t* sorted_ids,
+                                const void* da, const void* x, float* dw1, int accumulate,
+                                void* stream) {
+  int rc = check_shape(dims, true);
+  if (rc) return rc;
+  if (!ws || !sorted_ids || !da || !dw1 || (dims->T > 0 && !x) ||
+      (accumulate != 0 && accumulate != 1))
+    return MOE_ERR_INVALID_ARG;
+  GemmOperands o{};
+  o.a0 = da;
+  o.b1 = x;
+  o.out = dw1;
+  o.accumulate = accumulate;
+  o.gather_ids = sorted_ids;
+  return launch_grouped_gemm(MODE_DW1, *dims, ws, o, stream);
 }
 
 int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,

@@ -129,6 +129,9 @@ struct GemmOperands {
   void* out2;       // FWD1: saved pre-activations (nullable)
   const void* aux;  // DX2: saved pre-activations
   int accumulate;
+  // FWD1 / DW1: when set, the routed groups' x rows are gathered from a1 (x)
+  // through these token ids (sorted_ids [Rr]) instead of read from a permuted copy
+  const int32_t* gather_ids;
 };
 
 // Tensor map of a row-major bf16 matrix [rows, cols] (cols contiguous): box of

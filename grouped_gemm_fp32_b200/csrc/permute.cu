@@ -17,6 +17,8 @@
 //                warp counts) and writes sorted_ids and row_of.
 //   4. copy:     one warp per token reads x[t] once and writes its k rows.
 //   5. pad rows of x_perm are zeroed.
+// Steps 4 and 5 are skipped when no x_perm is asked for: the grouped GEMMs can
+// gather the x rows themselves through sorted_ids.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -294,6 +296,8 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
   if (n == 0) return MOE_OK;
   scatter_kernel<<<L.nchunks, kScatterThreads, 0, st>>>(idx, n, dm.k, dm.E, hist, offsets,
                                                         sorted_ids, row_of, status);
+  if (x_perm == nullptr)  // routing tables only: the GEMMs gather x rows themselves
+    return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
   const int row_vec = dm.d / 8;
   const int warps = 8;
   const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);

@@ -66,7 +66,7 @@ extern "C" int moe_permute_align_static(const moe_dims* dims, const int32_t* top
   // the scratch this call needs must fit the fixed array
   if (ws_layout(*dims).bytes > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!counts || !offsets || !sorted_ids) return MOE_ERR_INVALID_ARG;
-  if (dims->T > 0 && (!topk_idx || !x || !row_of || !x_perm)) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!topk_idx || !row_of || (x_perm && !x))) return MOE_ERR_INVALID_ARG;
   int rc = MOE_OK;
   void* ws = scratch_for_current_device(&rc);
   if (rc != MOE_OK) return rc;

@@ -7,9 +7,9 @@ libmoe.so.
 
 Layer (dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
 and "Load balancing"; §3.2 "Efficient implementation of Grouped GEMM"):
-    forward   moe_gate_topk -> moe_permute_align -> grouped_gemm_fwd -> moe_combine
+    forward   moe_gate_topk -> moe_permute_align -> grouped_gemm_fwd[_gather] -> moe_combine
     backward  moe_combine_bwd -> grouped_gemm_bwd_dx(GEMM2) -> grouped_gemm_bwd_dw(GEMM2)
-              -> grouped_gemm_bwd_dx(GEMM1) -> grouped_gemm_bwd_dw(GEMM1)
+              -> grouped_gemm_bwd_dx(GEMM1) -> grouped_gemm_bwd_dw(GEMM1) [or _dw1_gather]
               -> moe_combine(weights = NULL)  (un-permute-sum of the dX rows)
               [-> moe_router_bwd (dlogits; gate term added into dX; dWg)]
               [-> moe_bias_update (next step's selection bias)]
@@ -24,9 +24,16 @@ from . import _lib as L
 
 
 class MoEBuffers:
-    def __init__(self, dims: L.MoeDims, device="cuda", train: bool = False):
+    def __init__(self, dims: L.MoeDims, device="cuda", train: bool = False,
+                 gather: bool = False):
+        """``gather``: the first GEMM (and dW1) read the routed x rows straight from x
+        through ``sorted_ids`` (grouped_gemm_fwd_gather / grouped_gemm_bwd_dw1_gather)
+        and no x_perm [Rr, d] is allocated; otherwise (the default, faster on B200:
+        the row copy costs less than the four-row gather copies) they read the
+        permuted copy ``x_perm`` that moe_permute_align writes."""
         self.dims = dims
         self.train = train
+        self.gather = gather
         T, d, E, k, S, I = dims.T, dims.d, dims.E, dims.k, dims.S, dims.I
         G = E + S
         self.Rr = L.moe_rows_routed(dims)
@@ -43,7 +50,7 @@ class MoEBuffers:
         self.offsets = e(E + 1, dt=i32)
         self.sorted_ids = e(self.Rr, dt=i32)
         self.row_of = e(T, k, dt=i32)
-        self.x_perm = e(self.Rr, d)
+        self.x_perm = None if gather else e(self.Rr, d)
         self.h = e(self.Rt, I)
         self.a1 = e(self.Rt, 2 * I) if train else None
         self.y = e(self.Rt, d)
@@ -83,7 +90,10 @@ def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
             probs.copy_(routing[2])
     L.moe_permute_align(dm, b.topk_idx, x, b.counts, b.offsets, b.sorted_ids, b.row_of, b.x_perm,
                         b.ws, stream)
-    L.grouped_gemm_fwd(dm, b.ws, b.x_perm, x, w1, w2, b.h, b.a1, b.y, stream)
+    if b.gather:
+        L.grouped_gemm_fwd_gather(dm, b.ws, b.sorted_ids, x, w1, w2, b.h, b.a1, b.y, stream)
+    else:
+        L.grouped_gemm_fwd(dm, b.ws, b.x_perm, x, w1, w2, b.h, b.a1, b.y, stream)
     L.moe_combine(dm, b.y, b.row_of, b.topk_w, b.out, stream)
     return b.out
 
@@ -101,7 +111,10 @@ def backward(b: MoEBuffers, x, dout, w1, w2, stream=None, wg=None, gamma=None, b
     L.grouped_gemm_bwd_dx(dm, b.ws, L.MOE_GEMM2, b.dy, dout, w2, b.a1, b.da, stream)
     L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM2, b.dy, dout, b.h, None, b.dw2, 0, stream)
     L.grouped_gemm_bwd_dx(dm, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, stream)
-    L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x, b.dw1, 0, stream)
+    if b.gather:
+        L.grouped_gemm_bwd_dw1_gather(dm, b.ws, b.sorted_ids, b.da, x, b.dw1, 0, stream)
+    else:
+        L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x, b.dw1, 0, stream)
     L.moe_combine(dm, b.dxp, b.row_of, None, b.dx, stream)
     if wg is not None:
         L.moe_router_bwd(dm, x, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb, None, b.dx, b.dwg,
@@ -123,12 +136,12 @@ class HostPipeline:
     """
 
     def __init__(self, dims: L.MoeDims, w1, w2, wg, bias, train: bool, device="cuda",
-                 gamma=None, graphs: bool = True):
+                 gamma=None, graphs: bool = True, gather: bool = False):
         self.dims, self.train, self.gamma = dims, train, gamma
         self.w1, self.w2, self.wg, self.bias = w1, w2, wg, bias
         dev = torch.device(device)
         T, d = dims.T, dims.d
-        self.bufs = [MoEBuffers(dims, device=dev, train=train) for _ in range(2)]
+        self.bufs = [MoEBuffers(dims, device=dev, train=train, gather=gather) for _ in range(2)]
         # zero-filled: with graphs, one step runs on them before the capture
         e = lambda: torch.zeros(T, d, dtype=torch.bfloat16, device=dev)
         self.x = [e(), e()]

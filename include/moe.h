@@ -128,7 +128,10 @@ int moe_gate_topk(const moe_dims* dims, const void* x, const float* wg, const fl
  *                               segment), -1 on pad rows and rows >= off_E
  *   row_of     [T, k]   int32   routed row of (t, j)
  *   x_perm     [Rr, d]  bf16    x_perm[row_of[t, j]] = x[t]; pad rows zero;
- *                               rows >= off_E are not written
+ *                               rows >= off_E are not written.  May be NULL
+ *                               (then x may be NULL too): only the routing
+ *                               tables are written, for the *_gather GEMMs
+ *                               below, which read x rows through sorted_ids
  *   ws / ws_bytes               workspace (group table written here)
  * Deterministic: the same input gives the same output bit for bit.  An expert
  * id outside [0, E) or off_E > Rr sets MOE_ERR_BAD_ROUTING in the device
@@ -188,6 +191,23 @@ int grouped_gemm_set_groups(const moe_dims* dims, const int32_t* counts, int32_t
 int grouped_gemm_fwd(const moe_dims* dims, const void* ws, const void* x_perm, const void* x,
                      const void* w1, const void* w2, void* h, void* a1, void* y, void* stream);
 
+/* grouped_gemm_fwd with the routed groups' A rows gathered from x itself: row
+ * r of routed group e is x[sorted_ids[off_e + r]], loaded four rows at a time
+ * by tile::gather4 tensor copies, so no permuted copy x_perm is written or
+ * read.  (Passage: §3.2, as above; the row order inside a segment is the one
+ * moe_permute_align gives.)
+ *   sorted_ids [Rr] int32 (device), as written by moe_permute_align
+ *   x          [T, d] bf16 (may be NULL only when T = 0)
+ *   other arguments and outputs as in grouped_gemm_fwd.
+ * Rows holding no token (pad rows, id -1) and ids outside [0, T) read the
+ * group's first token instead of zeros: their h / a1 / y rows hold that
+ * token's values (pad-row contents are unspecified; nothing reads them, and
+ * with zero upstream gradients on pad rows they add nothing to dW).  No row
+ * outside x is ever read. */
+int grouped_gemm_fwd_gather(const moe_dims* dims, const void* ws, const int32_t* sorted_ids,
+                            const void* x, const void* w1, const void* w2, void* h, void* a1,
+                            void* y, void* stream);
+
 /* Backward data-gradient grouped GEMMs.
  *   which = MOE_GEMM2: dH = dY W2, then the SwiGLU backward with the saved a1:
  *       dG = dH * U * s * (1 + G (1 - s)), s = sigmoid(G);  dU = dH * silu(G)
@@ -214,6 +234,17 @@ int grouped_gemm_bwd_dx(const moe_dims* dims, const void* ws, int which, const v
 int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const void* lhs_routed,
                         const void* lhs_shared, const void* rhs_routed, const void* rhs_shared,
                         float* dw, int accumulate, void* stream);
+
+/* dW1_g = dA_g^T X_g (grouped_gemm_bwd_dw with which = MOE_GEMM1) with the
+ * routed groups' x rows gathered from x by sorted_ids as in
+ * grouped_gemm_fwd_gather; no x_perm.
+ *   sorted_ids [Rr] int32, da [Rt, 2I] bf16, x [T, d] bf16 (NULL only when T = 0)
+ *   -> dw1 [G, 2I, d] f32; accumulate as in grouped_gemm_bwd_dw.
+ * Pad rows of da must be zero (moe_combine_bwd zeroes the pad rows of dY, and
+ * the SwiGLU backward keeps them zero), since their x rows are a real token's. */
+int grouped_gemm_bwd_dw1_gather(const moe_dims* dims, const void* ws, const int32_t* sorted_ids,
+                                const void* da, const void* x, float* dw1, int accumulate,
+                                void* stream);
 
 /* Weighted combine (un-permute).
  * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"

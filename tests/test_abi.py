@@ -91,6 +91,16 @@ def test_validation_rejects_before_any_launch(lib):
     assert L.grouped_gemm_bwd_dx(ctypes.byref(ok64), p, 7, p, p, p, p, p, nul) == -1
     assert L.grouped_gemm_bwd_dw(ctypes.byref(ok64), p, 2, p, p, p, p, p, 5, nul) == -1
     assert L.moe_gate_topk(None, p, p, p, p, p, nul, p, 1 << 30, nul) == -1
+    # gathered-row GEMMs: sorted_ids and x are required (T > 0), dW1 needs P % 64
+    assert L.grouped_gemm_fwd_gather(ctypes.byref(ok), p, nul, p, p, p, p, nul, p, nul) == -1
+    assert L.grouped_gemm_fwd_gather(ctypes.byref(ok), p, p, nul, p, p, p, nul, p, nul) == -1
+    assert L.grouped_gemm_fwd_gather(ctypes.byref(ok), nul, p, p, p, p, p, nul, p, nul) == -1
+    assert L.grouped_gemm_bwd_dw1_gather(ctypes.byref(ok), p, p, p, p, p, 0, nul) == -2
+    assert L.grouped_gemm_bwd_dw1_gather(ctypes.byref(ok64), p, nul, p, p, p, 0, nul) == -1
+    assert L.grouped_gemm_bwd_dw1_gather(ctypes.byref(ok64), p, p, p, nul, p, 0, nul) == -1
+    assert L.grouped_gemm_bwd_dw1_gather(ctypes.byref(ok64), p, p, p, p, p, 5, nul) == -1
+    # permute without x_perm: x is optional then, but not when x_perm is given
+    assert L.moe_permute_align(ctypes.byref(ok), p, nul, p, p, p, p, p, p, 8, nul) == -1  # small ws
     # router backward: workspace, pointers, shapes; bias step: pointers
     big = 1 << 40
     assert L.moe_router_bwd(ctypes.byref(ok), p, p, p, p, p, p, nul, p, p, 0, nul, big, nul) == -1

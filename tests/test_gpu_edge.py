@@ -1,5 +1,6 @@
 """Edge cases of the whole layer through the C ABI: an empty batch, and the
-shape limits (k = E, S = 8 shared experts), against the oracle.
+shape limits (k = E, S = 8 shared experts), against the oracle; the layer-level
+cases run with x_perm and with x rows gathered through sorted_ids.
 
 Passages: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
 (routed top-k plus always-on shared experts) and "Load balancing" (no token
@@ -18,9 +19,10 @@ from grouped_gemm_fp32_b200 import layer
 pytestmark = pytest.mark.gpu
 
 
-def test_empty_batch_runs_every_call():
+@pytest.mark.parametrize("gather", [False, True])
+def test_empty_batch_runs_every_call(gather):
     dm = moe.MoeDims.of(0, 128, 8, 2, 1, 64, 64)
-    b = layer.MoEBuffers(dm, train=True)
+    b = layer.MoEBuffers(dm, train=True, gather=gather)
     x = torch.empty(0, 128, dtype=torch.bfloat16, device="cuda")
     wg = torch.ones(8, 128, device="cuda")
     bias = torch.zeros(8, device="cuda")
@@ -36,13 +38,14 @@ def test_empty_batch_runs_every_call():
     assert torch.equal(b.bias_next, bias)  # load 0 == mean load 0: sign 0, no step
 
 
-def test_all_experts_chosen_and_eight_shared():
+@pytest.mark.parametrize("gather", [False, True])
+def test_all_experts_chosen_and_eight_shared(gather):
     # k = E: every token uses every routed expert (w = p); S = 8 shared experts (G = 16)
     wl = synth.Workload("edge_kE_S8", synth.Dims(T=200, d=128, E=8, k=8, S=8, I=64, P=64),
                         seed=21, w1_std=0.05, w2_std=0.05, wg_std=0.05, backward=True)
     inp = synth.make_inputs(wl)
     dm = dims_of(wl)
-    b = layer.MoEBuffers(dm, train=True)
+    b = layer.MoEBuffers(dm, train=True, gather=gather)
     x, w1, w2 = dev(inp["x"], True), dev(inp["w1"], True), dev(inp["w2"], True)
     wg = dev(inp["wg"])
     out = layer.forward(b, x, wg, dev(inp["bias"]), w1, w2)
@@ -61,7 +64,8 @@ def test_all_experts_chosen_and_eight_shared():
     assert_close(host(b.dwg), gdwg, "dWg")
 
 
-def test_nan_tokens_still_get_valid_distinct_experts():
+@pytest.mark.parametrize("gather", [False, True])
+def test_nan_tokens_still_get_valid_distinct_experts(gather):
     # non-finite hidden states make NaN scores; the gate must still name k distinct,
     # valid experts for them (so nothing downstream indexes out of range), and the
     # finite tokens must route as the oracle does
@@ -71,7 +75,7 @@ def test_nan_tokens_still_get_valid_distinct_experts():
     bad = [3, 77, 200]
     inp["x"][bad, 5] = 0x7FC0  # bf16 NaN
     dm = dims_of(wl)
-    b = layer.MoEBuffers(dm, train=True)
+    b = layer.MoEBuffers(dm, train=True, gather=gather)
     x, w1, w2 = dev(inp["x"], True), dev(inp["w1"], True), dev(inp["w2"], True)
     wg = dev(inp["wg"])
     layer.forward(b, x, wg, dev(inp["bias"]), w1, w2)
@@ -119,7 +123,8 @@ def test_invalid_routing_leaves_no_stale_rows():
     assert torch.all(dwc == 0) and torch.all(dy == 0)
 
 
-def test_256_experts_full_layer():
+@pytest.mark.parametrize("gather", [False, True])
+def test_256_experts_full_layer(gather):
     # E = 256 routed experts (the largest supported) + 2 shared: G = 258 groups, many of
     # them short or empty; forward, backward and the router backward against the oracle
     # with the oracle's routing injected
@@ -128,7 +133,7 @@ def test_256_experts_full_layer():
     inp = synth.make_inputs(wl)
     dm = dims_of(wl)
     p, oidx, ow, _ = oracle.route(oracle.gate_logits(inp["x"], inp["wg"]), inp["bias"], 8)
-    b = layer.MoEBuffers(dm, train=True)
+    b = layer.MoEBuffers(dm, train=True, gather=gather)
     x, w1, w2 = dev(inp["x"], True), dev(inp["w1"], True), dev(inp["w2"], True)
     wg = dev(inp["wg"])
     out = layer.forward(b, x, wg, dev(inp["bias"]), w1, w2,

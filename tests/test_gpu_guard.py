@@ -53,7 +53,8 @@ def _guard_buffers(b: layer.MoEBuffers, g: Guarded):
     (77, 128, 16, 4, 2, 128, 16, False),    # pad block 16 < the 128-row MMA tile
     (1000, 256, 32, 6, 1, 192, 64, True),   # I = 192: a narrow last N tile in the dX/dW GEMMs
 ])
-def test_no_write_outside_any_buffer(T, d, E, k, S, I, P, train):
+@pytest.mark.parametrize("gather", [False, True])
+def test_no_write_outside_any_buffer(T, d, E, k, S, I, P, train, gather):
     wl = synth.Workload("guard", synth.Dims(T=T, d=d, E=E, k=k, S=S, I=I, P=P), seed=T + E,
                         w1_std=0.05, w2_std=0.05, wg_std=0.05, backward=train)
     inp = synth.make_inputs(wl)
@@ -61,7 +62,7 @@ def test_no_write_outside_any_buffer(T, d, E, k, S, I, P, train):
     bias[1] = -1.0  # expert 1 empty
     dm = dims_of(wl)
     g = Guarded()
-    b = layer.MoEBuffers(dm, train=train)
+    b = layer.MoEBuffers(dm, train=train, gather=gather)
     _guard_buffers(b, g)
     x = g.wrap(dev(inp["x"], True))
     w1, w2 = g.wrap(dev(inp["w1"], True)), g.wrap(dev(inp["w2"], True))
