@@ -19,6 +19,14 @@ function cites the passage of the dots.llm1 Technical Report it follows:
   two-layer SwiGLU experts, 6 routed + 2 shared per token.
 * ``layer_bwd`` / ``group_dw``   -- the exact gradient of ``layer_fwd``
   (bf16 storage points treated as the identity).
+* ``router_bwd``   -- the gradient of the combine weights (the chosen experts'
+  affinities, §"Mixture of Experts layer") through the renormalisation and
+  the softmax, into the gate's input and weights.
+* ``bias_update``  -- §"Load balancing": the bias is adjusted during training
+  to keep the loads balanced (sign step towards the mean load).
+* ``seq_balance``  -- §"Load balancing": the sequence-wise balance loss the
+  pages add without a formula, read as the one in the report they cite for
+  their method (DeepSeek-V3), with softmax affinities; value and gradient.
 
 Pins (what this oracle is checked against, other than itself) live in
 ``tests/test_oracle_*.py``.  Parity of every function here is pinned.
@@ -62,7 +70,9 @@ def _load():
         lib.oracle_round_bf16.argtypes = [dbl]
         lib.oracle_gate_logits.argtypes = [vp, vp, i64, i32, i32, vp]
         lib.oracle_route.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp]
-        lib.oracle_router_bwd.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp]
+        lib.oracle_router_bwd.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp]
+        lib.oracle_seq_balance.restype = dbl
+        lib.oracle_seq_balance.argtypes = [vp, vp, i64, i32, i32, i64, dbl, vp]
         lib.oracle_bias_update.argtypes = [vp, i64, i32, i32, vp, ctypes.c_float, vp]
         lib.oracle_permute.restype = i64
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, i32, i64, vp, vp, vp, vp]
@@ -129,20 +139,36 @@ def route(logits: np.ndarray, bias: np.ndarray, k: int):
 
 
 def router_bwd(x: np.ndarray, wg: np.ndarray, idx: np.ndarray, dw: np.ndarray,
-               want_dx: bool = True, want_dwg: bool = True):
+               want_dx: bool = True, want_dwg: bool = True, dl_extra=None):
     """Gradient of the combine weights through the renormalisation and the softmax:
     (dlogits [T,E], dx [T,d], dwg [E,d]), all FP64 (dx / dwg None when not wanted).
-    x: bf16 bits [T,d]; wg: f32 [E,d]; idx [T,k] the chosen experts; dw [T,k] = dL/dw."""
+    x: bf16 bits [T,d]; wg: f32 [E,d]; idx [T,k] the chosen experts; dw [T,k] = dL/dw.
+    dl_extra [T,E] (optional): a further dL/dlogit term (``seq_balance``'s) added to
+    dlogits before dx and dwg are formed."""
     x, wg, idx, dw = _c(x, np.uint16), _c(wg, np.float32), _c(idx, np.int32), _c(dw, np.float64)
     T, d = x.shape
     E = wg.shape[0]
     k = idx.shape[1]
+    extra = None if dl_extra is None else _c(dl_extra, np.float64)
     dl = np.empty((T, E))
     dx = np.empty((T, d)) if want_dx else None
     dwg = np.empty((E, d)) if want_dwg else None
-    _load().oracle_router_bwd(_p(x), _p(wg), _p(idx), _p(dw), T, d, E, k, _p(dl), _p(dx),
-                              _p(dwg))
+    _load().oracle_router_bwd(_p(x), _p(wg), _p(idx), _p(dw), T, d, E, k, _p(extra), _p(dl),
+                              _p(dx), _p(dwg))
     return dl, dx, dwg
+
+
+def seq_balance(logits: np.ndarray, idx: np.ndarray, seq_len: int, alpha: float,
+                want_grad: bool = True):
+    """Sequence-wise balance loss (mean over the batch's sequences of seq_len
+    tokens) and its gradient dL/dlogit [T,E] (FP64; None when not wanted)."""
+    logits, idx = _c(logits, np.float64), _c(idx, np.int32)
+    T, E = logits.shape
+    k = idx.shape[1]
+    dl = np.empty((T, E)) if want_grad else None
+    loss = _load().oracle_seq_balance(_p(logits), _p(idx), T, E, k, int(seq_len), float(alpha),
+                                      _p(dl))
+    return float(loss), dl
 
 
 def bias_update(idx: np.ndarray, E: int, bias: np.ndarray, gamma: float) -> np.ndarray:

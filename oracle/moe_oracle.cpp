@@ -204,9 +204,11 @@ void oracle_route(const double* logits, const float* bias, int64_t T, int E, int
 //   p = softmax(logit)   =>  dlogit_e = p_e (dp_e - sum_i p_i dp_i)
 //   logit = X Wg^T       =>  dX = dlogit Wg,   dWg = dlogit^T X
 // Logits and p are recomputed in FP64 from x and wg.  Any of the outputs may be null.
+// dl_extra [T, E] (nullable) is a further dL/dlogit term (the sequence-wise balance
+// loss's) added before dX and dWg are formed.
 void oracle_router_bwd(const uint16_t* x, const float* wg, const int32_t* idx, const double* dw,
-                       int64_t T, int d, int E, int k, double* dlogits, double* dx,
-                       double* dwg) {
+                       int64_t T, int d, int E, int k, const double* dl_extra, double* dlogits,
+                       double* dx, double* dwg) {
   std::vector<double> dl((size_t)T * E);
 #pragma omp parallel
   {
@@ -240,6 +242,8 @@ void oracle_router_bwd(const uint16_t* x, const float* wg, const int32_t* idx, c
       for (int e = 0; e < E; ++e) dl[(size_t)t * E + e] = p[e] * (dp[e] - pdp);
     }
   }
+  if (dl_extra)
+    for (size_t i = 0; i < dl.size(); ++i) dl[i] += dl_extra[i];
   if (dlogits) std::copy(dl.begin(), dl.end(), dlogits);
   if (dx) {
 #pragma omp parallel for schedule(static)
@@ -259,6 +263,69 @@ void oracle_router_bwd(const uint16_t* x, const float* wg, const int32_t* idx, c
         dwg[(size_t)e * d + c] = s;
       }
   }
+}
+
+// Sequence-wise balance loss and its gradient with respect to the logits.
+// The pages add a sequence-wise balance loss to the aux-loss-free method without
+// stating it; the method they cite (the DeepSeek-V3 report) defines one, taken
+// here with this layer's softmax affinities.  The batch's T tokens form
+// sequences of L tokens (the last one may be shorter); for sequence s with L_s
+// tokens:
+//   p_t   = softmax(logit_t),   q_t = p_t / sum_e p_t,e      (normalised affinities)
+//   f_s,i = E / (k L_s) * #{(t in s, j) : idx[t, j] = i}     (load fraction, x E)
+//   P_s,i = (1 / L_s) * sum_{t in s} q_t,i                   (mean affinity)
+//   loss  = (1 / n_seq) * sum_s alpha * sum_i f_s,i P_s,i     (mean over sequences)
+// The selection is piecewise constant, so the gradient runs through P only:
+//   dloss/dq_t,i = alpha f_s,i / (n_seq L_s)
+//   dloss/dp_t,j = sum_i dloss/dq_t,i (delta_ij / z - p_t,i / z^2),  z = sum_e p_t,e
+//   dloss/dlogit_t,e = p_t,e (dloss/dp_t,e - sum_j p_t,j dloss/dp_t,j)
+// Returns the loss; dlogits [T, E] may be null.
+double oracle_seq_balance(const double* logits, const int32_t* idx, int64_t T, int E, int k,
+                          int64_t L, double alpha, double* dlogits) {
+  if (T <= 0 || L <= 0) return 0.0;
+  const int64_t nseq = (T + L - 1) / L;
+  std::vector<double> p((size_t)T * E), q((size_t)T * E), z(T);
+  for (int64_t t = 0; t < T; ++t) {
+    const double* lg = logits + t * E;
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e) m = std::max(m, lg[e]);
+    double sum = 0.0;
+    for (int e = 0; e < E; ++e) sum += (p[t * E + e] = std::exp(lg[e] - m));
+    for (int e = 0; e < E; ++e) p[t * E + e] /= sum;
+    z[t] = 0.0;
+    for (int e = 0; e < E; ++e) z[t] += p[t * E + e];
+    for (int e = 0; e < E; ++e) q[t * E + e] = p[t * E + e] / z[t];
+  }
+  double loss = 0.0;
+  std::vector<double> f(E), P(E), g(E), dp(E);
+  for (int64_t s = 0; s < nseq; ++s) {
+    const int64_t t0 = s * L, t1 = std::min(T, t0 + L), Ls = t1 - t0;
+    std::fill(f.begin(), f.end(), 0.0);
+    std::fill(P.begin(), P.end(), 0.0);
+    for (int64_t t = t0; t < t1; ++t) {
+      for (int j = 0; j < k; ++j) f[idx[t * k + j]] += 1.0;
+      for (int e = 0; e < E; ++e) P[e] += q[t * E + e];
+    }
+    double ls = 0.0;
+    for (int e = 0; e < E; ++e) {
+      f[e] *= (double)E / ((double)k * (double)Ls);
+      P[e] /= (double)Ls;
+      ls += f[e] * P[e];
+    }
+    loss += alpha * ls / (double)nseq;
+    if (!dlogits) continue;
+    for (int e = 0; e < E; ++e) g[e] = alpha * f[e] / ((double)nseq * (double)Ls);
+    for (int64_t t = t0; t < t1; ++t) {
+      const double* pt = p.data() + t * E;
+      double gp = 0.0;
+      for (int i = 0; i < E; ++i) gp += g[i] * pt[i];
+      for (int j = 0; j < E; ++j) dp[j] = g[j] / z[t] - gp / (z[t] * z[t]);
+      double pdp = 0.0;
+      for (int e = 0; e < E; ++e) pdp += pt[e] * dp[e];
+      for (int e = 0; e < E; ++e) dlogits[t * E + e] = pt[e] * (dp[e] - pdp);
+    }
+  }
+  return loss;
 }
 
 // Aux-loss-free bias update, one step (the pages say the bias is adjusted during
