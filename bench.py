@@ -45,6 +45,10 @@ sys.path.insert(0, ROOT)
 # value; 1e-3 per step is an illustrative choice, applied to a copy of the bias so
 # every timed step routes the same synthetic batch the same way).
 GAMMA = 1e-3
+# Sequence-wise balance loss of the train step: (alpha, tokens per sequence).  The
+# pages give no alpha (a small illustrative value here); 8192 tokens is the
+# pre-training sequence length they state.
+SEQ_BALANCE = (1e-4, 8192)
 
 METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of B200 BF16 peak), 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -251,7 +255,8 @@ def oracle_sample_step(wl, inp, ntok):
         used = set(np.unique(idx).tolist()) | set(range(dm.E, dm.E + dm.S))
         for g in sorted(used):
             oracle.group_dw(x, idx, w, inp["w1"], inp["w2"], dout, dm.S, g)
-        oracle.router_bwd(x, inp["wg"], idx, dw)
+        _, dl_bal = oracle.seq_balance(lg, idx, SEQ_BALANCE[1], SEQ_BALANCE[0])
+        oracle.router_bwd(x, inp["wg"], idx, dw, dl_extra=dl_bal)
         oracle.bias_update(idx, dm.E, inp["bias"], GAMMA)
     return time.perf_counter() - t0
 
@@ -363,7 +368,8 @@ def run_ours(args):
                 ev["fwd"][-1].record(s)
             return
         if ev is None:
-            layer.forward(b, xx, wg, bias, w1, w2, stream=s)
+            layer.forward(b, xx, wg, bias, w1, w2, stream=s,
+                          seq_balance=SEQ_BALANCE if train else None)
             if train:
                 layer.backward(b, xx, gg, w1, w2, stream=s, wg=wg, gamma=GAMMA, bias=bias)
             return
@@ -385,6 +391,10 @@ def run_ours(args):
         L.moe_combine(dims, b.y, b.row_of, b.topk_w, b.out, s)
         rec("combine")
         if train:
+            L.moe_seq_balance_loss(dims, SEQ_BALANCE[1], SEQ_BALANCE[0], b.topk_idx, b.probs,
+                                   b.bal_loss, b.bal_grad, b.ws, s)
+            rec("seq_balance")
+        if train:
             L.moe_combine_bwd(dims, b.ws, gg, b.y, b.row_of, b.topk_w, b.dy, b.dw_comb, s)
             rec("combine_bwd")
             L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM2, b.dy, gg, w2, b.a1, b.da, s)
@@ -401,8 +411,8 @@ def run_ours(args):
             rec("dw1")
             L.moe_combine(dims, b.dxp, b.row_of, None, b.dx, s)
             rec("unpermute")
-            L.moe_router_bwd(dims, xx, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb, None, b.dx,
-                             b.dwg, 0, b.ws, s)
+            L.moe_router_bwd_seqbal(dims, xx, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb,
+                                    b.bal_grad, SEQ_BALANCE[1], None, b.dx, b.dwg, 0, b.ws, s)
             rec("router_bwd")
             L.moe_bias_update(dims, b.counts, GAMMA, bias, b.bias_next, s)
             rec("bias_step")
@@ -421,7 +431,8 @@ def run_ours(args):
     graph = None
     if use_graph:
         graph = layer.GraphStep(b, x, wg, bias, w1, w2, dout=dout if train else None,
-                                gamma=GAMMA if train else None)
+                                gamma=GAMMA if train else None,
+                                seq_balance=SEQ_BALANCE if train else None)
 
     def timed_steps(n):
         with torch.cuda.stream(stream):
@@ -465,7 +476,8 @@ def run_ours(args):
     # ---- per-call breakdown (separate instrumented pass; not the headline)
     names = (["t0", "gate"] if gate_only else
              ["t0", "fwd"] if gemm_only else ["t0", "gate", "permute", "fwd", "combine"]) + (
-        ["combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute", "router_bwd", "bias_step"]
+        ["seq_balance", "combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute", "router_bwd",
+         "bias_step"]
         if train else [])
     ev = {n: [] for n in names}
     nprof = max(3, min(args.steps, 20))
@@ -508,6 +520,7 @@ def run_ours(args):
     else:
         pipe = layer.HostPipeline(dims, w1, w2, wg, bias, train, device=dev,
                                   gamma=GAMMA if train else None, graphs=not args.eager,
+                                  seq_balance=SEQ_BALANCE if train else None,
                                   gather=args.gather)
         hx = [pinned(inp["x"])]
         hd = [pinned(inp["dout"])] if train else [None]
@@ -545,11 +558,12 @@ def run_ours(args):
 
     # kernels per step: gate 2 (weight split, gate), permute 3 (histogram, groups,
     # scatter; + row copy and pad zeroing without gathering), forward GEMMs 2, combine 1;
-    # train adds combine backward 2, backward GEMMs 4, un-permute 1, router backward 5
-    # (weight split, dlogits, dX GEMM, dWg GEMM, split-K sum), bias step 1
+    # train adds the balance loss 2 (chunk sums, finish), combine backward 2, backward
+    # GEMMs 4, un-permute 1, router backward 5 (weight split, dlogits, dX GEMM, dWg GEMM,
+    # split-K sum), bias step 1
     permute_launches = 3 if args.gather else 5
     launches_per_step = (2 if gate_only else 2 if gemm_only else
-                         2 + permute_launches + 2 + 1 + ((2 + 4 + 1 + 5 + 1) if train else 0))
+                         2 + permute_launches + 2 + 1 + ((2 + 2 + 4 + 1 + 5 + 1) if train else 0))
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -561,6 +575,8 @@ def run_ours(args):
                    "step": "CUDA graph replay" if graph is not None else "eager C-ABI calls",
                    "x_rows": ("gathered from x by sorted_ids (tile::gather4)" if args.gather
                               else "permuted copy x_perm"),
+                   "seq_balance": ({"alpha": SEQ_BALANCE[0], "seq_len": SEQ_BALANCE[1]}
+                                   if train else None),
                    "ms_per_step_eager": ms_eager,
                    "l2": "no flush: weights (4.5 GB) and activations exceed the 126 MB L2"},
         "roofline": {"bound": "tensor", "kernel": "ggemm_kernel (all grouped-GEMM launches)",

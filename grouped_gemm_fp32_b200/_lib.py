@@ -19,7 +19,8 @@ EXPORTS = (
     "moe_permute_align", "moe_permute_align_static", "grouped_gemm_set_groups",
     "grouped_gemm_fwd", "grouped_gemm_fwd_gather", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw",
     "grouped_gemm_bwd_dw1_gather", "moe_combine",
-    "moe_combine_bwd", "moe_router_bwd", "moe_bias_update", "moe_get_device_status",
+    "moe_combine_bwd", "moe_router_bwd", "moe_router_bwd_seqbal", "moe_seq_balance_loss",
+    "moe_bias_update", "moe_get_device_status",
     "moe_status_string", "moe_last_cuda_error",
 )
 
@@ -77,6 +78,9 @@ def load():
         "grouped_gemm_bwd_dw": (i32, [D, vp, i32, vp, vp, vp, vp, vp, i32, vp]),
         "moe_combine": (i32, [D, vp, vp, vp, vp, vp]),
         "moe_router_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+        "moe_router_bwd_seqbal": (i32, [D, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, i32, vp,
+                                        sz, vp]),
+        "moe_seq_balance_loss": (i32, [D, i64, ctypes.c_float, vp, vp, vp, vp, vp, sz, vp]),
         "moe_bias_update": (i32, [D, vp, ctypes.c_float, vp, vp, vp]),
         "moe_combine_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_get_device_status": (i32, [vp, vp, vp]),
@@ -208,6 +212,22 @@ def moe_router_bwd(dims, x, wg, probs, topk_idx, topk_w, dw, dlogits, dx, dwg, a
     _ck(load().moe_router_bwd(ctypes.byref(dims), _p(x), _p(wg), _p(probs), _p(topk_idx),
                               _p(topk_w), _p(dw), _p(dlogits), _p(dx), _p(dwg), int(accumulate),
                               _p(ws), nbytes, _s(stream)), "moe_router_bwd")
+
+
+def moe_router_bwd_seqbal(dims, x, wg, probs, topk_idx, topk_w, dw, seq_grad, seq_len, dlogits,
+                          dx, dwg, accumulate, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _ck(load().moe_router_bwd_seqbal(ctypes.byref(dims), _p(x), _p(wg), _p(probs), _p(topk_idx),
+                                     _p(topk_w), _p(dw), _p(seq_grad), int(seq_len),
+                                     _p(dlogits), _p(dx), _p(dwg), int(accumulate), _p(ws),
+                                     nbytes, _s(stream)), "moe_router_bwd_seqbal")
+
+
+def moe_seq_balance_loss(dims, seq_len, alpha, topk_idx, probs, loss, seq_grad, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _ck(load().moe_seq_balance_loss(ctypes.byref(dims), int(seq_len), float(alpha),
+                                    _p(topk_idx), _p(probs), _p(loss), _p(seq_grad), _p(ws),
+                                    nbytes, _s(stream)), "moe_seq_balance_loss")
 
 
 def moe_bias_update(dims, counts, gamma, bias_in, bias_out, stream=None):

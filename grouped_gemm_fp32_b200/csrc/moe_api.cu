@@ -81,8 +81,35 @@ int moe_router_bwd(const moe_dims* dims, const void* x, const float* wg, const f
   if (!ws || ws_bytes < ws_layout(*dims).total || !wg || !dwg) return MOE_ERR_INVALID_ARG;
   if (dims->T > 0 && (!x || !probs || !topk_idx || !topk_w || !dw || !dx))
     return MOE_ERR_INVALID_ARG;
-  return launch_router_bwd(*dims, x, wg, probs, topk_idx, topk_w, dw, dlogits, dx, dwg,
-                           accumulate ? 1 : 0, ws, stream);
+  return launch_router_bwd(*dims, x, wg, probs, topk_idx, topk_w, dw, nullptr, 1, dlogits, dx,
+                           dwg, accumulate ? 1 : 0, ws, stream);
+}
+
+int moe_router_bwd_seqbal(const moe_dims* dims, const void* x, const float* wg,
+                          const float* probs, const int32_t* topk_idx, const float* topk_w,
+                          const float* dw, const float* seq_grad, int64_t seq_len,
+                          float* dlogits, void* dx, float* dwg, int accumulate, void* ws,
+                          size_t ws_bytes, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (dims->E % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!ws || ws_bytes < ws_layout(*dims).total || !wg || !dwg) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!x || !probs || !topk_idx || !topk_w || !dw || !dx || !seq_grad ||
+                      seq_len < kSeqMin))
+    return MOE_ERR_INVALID_ARG;
+  return launch_router_bwd(*dims, x, wg, probs, topk_idx, topk_w, dw, seq_grad, seq_len,
+                           dlogits, dx, dwg, accumulate ? 1 : 0, ws, stream);
+}
+
+int moe_seq_balance_loss(const moe_dims* dims, int64_t seq_len, float alpha,
+                         const int32_t* topk_idx, const float* probs, float* loss,
+                         float* seq_grad, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (seq_len < kSeqMin) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!ws || ws_bytes < ws_layout(*dims).total || !loss) return MOE_ERR_INVALID_ARG;
+  if (dims->T > 0 && (!topk_idx || !probs || !seq_grad)) return MOE_ERR_INVALID_ARG;
+  return launch_seq_balance(*dims, seq_len, alpha, topk_idx, probs, loss, seq_grad, ws, stream);
 }
 
 int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,

@@ -39,12 +39,19 @@ struct WsLayout {
   size_t gate_split;    // bf16[3][e_pad][d]  the gate weights as hi, mid, lo planes
   size_t dl_planes;     // bf16[3][t_pad][e_pad]  dL/dlogit as hi, mid, lo planes
   size_t gdw_part;      // f32[gdw_splits][e_pad][d]  split-K partial sums of dWg
+  size_t seqbal;        // sequence-wise balance loss: f32[sb_chunks][E] affinity sums,
+                        // then int32[sb_chunks][E] pick counts
   size_t total;         // whole workspace
   int nchunks;
   int e_pad;            // E rounded up to a multiple of 32
   int t_pad;            // T rounded up to a multiple of 128
   int gdw_splits;       // K splits of the dWg GEMM
+  int sb_chunks;        // token chunks (of <= kSeqChunk, inside one sequence) the
+                        // balance loss can need: sequences of >= kSeqMin tokens
 };
+
+constexpr int kSeqChunk = 64;  // tokens per chunk of the balance loss's column sums
+constexpr int kSeqMin = 128;   // shortest sequence the balance loss accepts
 
 // K splits of the dWg GEMM: as many work items as fit one wave on a B200's 148
 // SMs, at most 16 splits, and no split left empty.
@@ -84,7 +91,11 @@ inline WsLayout ws_layout(const moe_dims& dm) {
   L.gate_split = align_up(L.bytes, 1024);
   L.dl_planes = align_up(L.gate_split + (size_t)3 * L.e_pad * dm.d * 2, 1024);
   L.gdw_part = align_up(L.dl_planes + (size_t)3 * L.t_pad * L.e_pad * 2, 1024);
-  L.total = align_up(L.gdw_part + (size_t)L.gdw_splits * L.e_pad * dm.d * 4, 256);
+  // chunks of sequences of L >= kSeqMin >= kSeqChunk tokens:
+  // sum_s ceil(L_s / kSeqChunk) <= T / kSeqChunk + n_seq <= 2 ceil(T / kSeqChunk)
+  L.sb_chunks = (int)(2 * ((dm.T + kSeqChunk - 1) / kSeqChunk)) + 1;
+  L.seqbal = align_up(L.gdw_part + (size_t)L.gdw_splits * L.e_pad * dm.d * 4, 256);
+  L.total = align_up(L.seqbal + (size_t)L.sb_chunks * dm.E * 8, 256);
   return L;
 }
 
@@ -103,10 +114,13 @@ int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offset
                       void* stream);
 int launch_split_wg(const moe_dims& dm, const float* wg, void* planes, void* stream);
 int launch_router_bwd(const moe_dims& dm, const void* x, const float* wg, const float* probs,
-                      const int32_t* idx, const float* w, const float* dw, float* dlogits,
-                      void* dx, float* dwg, int accumulate, void* ws, void* stream);
+                      const int32_t* idx, const float* w, const float* dw,
+                      const float* seq_grad, int64_t seq_len, float* dlogits, void* dx,
+                      float* dwg, int accumulate, void* ws, void* stream);
 int launch_bias_update(const moe_dims& dm, const int32_t* counts, float gamma,
                        const float* bias_in, float* bias_out, void* stream);
+int launch_seq_balance(const moe_dims& dm, int64_t seq_len, float alpha, const int32_t* idx,
+                       const float* probs, float* loss, float* seq_grad, void* ws, void* stream);
 // Router-backward GEMMs (sgemm.cu); planes and partial sums live in the workspace.
 int launch_gate_dx(const moe_dims& dm, const void* dl_planes, const void* wg_planes, void* dx,
                    int* status, void* stream);

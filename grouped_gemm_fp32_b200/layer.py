@@ -11,7 +11,8 @@ and "Load balancing"; §3.2 "Efficient implementation of Grouped GEMM"):
     backward  moe_combine_bwd -> grouped_gemm_bwd_dx(GEMM2) -> grouped_gemm_bwd_dw(GEMM2)
               -> grouped_gemm_bwd_dx(GEMM1) -> grouped_gemm_bwd_dw(GEMM1) [or _dw1_gather]
               -> moe_combine(weights = NULL)  (un-permute-sum of the dX rows)
-              [-> moe_router_bwd (dlogits; gate term added into dX; dWg)]
+              [-> moe_router_bwd (dlogits; gate term added into dX; dWg), or
+                  moe_router_bwd_seqbal after forward's moe_seq_balance_loss]
               [-> moe_bias_update (next step's selection bias)]
 The router backward runs when the gate weights are passed to ``backward``; the
 bias step when an update speed ``gamma`` is.
@@ -66,19 +67,26 @@ class MoEBuffers:
             self.probs = e(T, E, dt=f32)
             self.dwg = e(E, d, dt=f32)
             self.bias_next = e(E, dt=f32)
+            # sequence-wise balance loss: its value and dL/dp per sequence (sequences
+            # of >= 128 tokens, so at most ceil(T / 128) of them)
+            self.bal_loss = torch.zeros(1, dtype=f32, device=dev)
+            self.bal_grad = e(max(1, -(-T // 128)), E, dt=f32)
+            self.bal_seq_len = None
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in vars(self).values()
                    if isinstance(t, torch.Tensor))
 
 
-def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
+def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None, seq_balance=None):
     """out = MoE(x).  x [T, d] bf16, wg [E, d] f32, bias [E] f32, w1 [G, 2I, d], w2 [G, d, I].
 
     ``routing=(topk_idx, topk_w[, probs])`` (device int32 / f32 [T, k], f32 [T, E])
     replaces the gate's choice, e.g. to run the experts on a routing decided
     elsewhere.  With train buffers the gate also saves its affinities (probs) for
-    the router backward."""
+    the router backward.  ``seq_balance=(alpha, seq_len)`` (train buffers) also
+    computes the sequence-wise balance loss into ``b.bal_loss``; ``backward``
+    then adds its gradient to the router's."""
     dm = b.dims
     probs = b.probs if b.train else None
     if routing is None:
@@ -95,6 +103,13 @@ def forward(b: MoEBuffers, x, wg, bias, w1, w2, stream=None, routing=None):
     else:
         L.grouped_gemm_fwd(dm, b.ws, b.x_perm, x, w1, w2, b.h, b.a1, b.y, stream)
     L.moe_combine(dm, b.y, b.row_of, b.topk_w, b.out, stream)
+    if b.train:
+        b.bal_seq_len = None
+        if seq_balance is not None:
+            alpha, seq_len = seq_balance
+            L.moe_seq_balance_loss(dm, seq_len, alpha, b.topk_idx, b.probs, b.bal_loss,
+                                   b.bal_grad, b.ws, stream)
+            b.bal_seq_len = int(seq_len)
     return b.out
 
 
@@ -117,8 +132,12 @@ def backward(b: MoEBuffers, x, dout, w1, w2, stream=None, wg=None, gamma=None, b
         L.grouped_gemm_bwd_dw(dm, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x, b.dw1, 0, stream)
     L.moe_combine(dm, b.dxp, b.row_of, None, b.dx, stream)
     if wg is not None:
-        L.moe_router_bwd(dm, x, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb, None, b.dx, b.dwg,
-                         0, b.ws, stream)
+        if b.bal_seq_len is not None:
+            L.moe_router_bwd_seqbal(dm, x, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb,
+                                    b.bal_grad, b.bal_seq_len, None, b.dx, b.dwg, 0, b.ws, stream)
+        else:
+            L.moe_router_bwd(dm, x, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb, None, b.dx,
+                             b.dwg, 0, b.ws, stream)
     if gamma is not None:
         L.moe_bias_update(dm, b.counts, gamma, bias, b.bias_next, stream)
     return b.dx, b.dw1, b.dw2, b.dw_comb
@@ -136,8 +155,9 @@ class HostPipeline:
     """
 
     def __init__(self, dims: L.MoeDims, w1, w2, wg, bias, train: bool, device="cuda",
-                 gamma=None, graphs: bool = True, gather: bool = False):
+                 gamma=None, graphs: bool = True, gather: bool = False, seq_balance=None):
         self.dims, self.train, self.gamma = dims, train, gamma
+        self.seq_balance = seq_balance if train else None
         self.w1, self.w2, self.wg, self.bias = w1, w2, wg, bias
         dev = torch.device(device)
         T, d = dims.T, dims.d
@@ -160,7 +180,8 @@ class HostPipeline:
         if graphs:
             self.graphs = [GraphStep(self.bufs[j], self.x[j], wg, bias, w1, w2,
                                      dout=self.dout[j] if train else None,
-                                     gamma=gamma if train else None) for j in range(2)]
+                                     gamma=gamma if train else None,
+                                     seq_balance=self.seq_balance) for j in range(2)]
 
     def _upload(self, j, hx, hd):
         with torch.cuda.stream(self.up):
@@ -189,7 +210,8 @@ class HostPipeline:
                 if self.graphs is not None:
                     self.graphs[j].replay()
                 else:
-                    forward(b, self.x[j], self.wg, self.bias, self.w1, self.w2, stream=s)
+                    forward(b, self.x[j], self.wg, self.bias, self.w1, self.w2, stream=s,
+                            seq_balance=self.seq_balance)
                     if self.train:
                         backward(b, self.x[j], self.dout[j], self.w1, self.w2, stream=s,
                                  wg=self.wg, gamma=self.gamma, bias=self.bias)
@@ -209,7 +231,8 @@ class HostPipeline:
 
 class GraphStep:
     """One layer step -- forward, and with ``dout`` the backward (router backward
-    and bias step included when ``gamma`` is given) -- captured once as a CUDA
+    and bias step included when ``gamma`` is given, the sequence-wise balance loss
+    when ``seq_balance=(alpha, seq_len)`` is) -- captured once as a CUDA
     graph and replayed.  Every node is one of the same C-ABI calls as in eager
     mode, on the captured stream; the graph keeps the buffers' addresses, so new
     inputs are written into ``x`` / ``dout`` in place before ``replay``.
@@ -218,10 +241,11 @@ class GraphStep:
     kernel attributes and look up driver entry points, which must not happen
     inside a capture."""
 
-    def __init__(self, b: MoEBuffers, x, wg, bias, w1, w2, dout=None, gamma=None):
+    def __init__(self, b: MoEBuffers, x, wg, bias, w1, w2, dout=None, gamma=None,
+                 seq_balance=None):
         self.b = b
         self.stream = torch.cuda.Stream(device=x.device)
-        args = (b, x, wg, bias, w1, w2, dout, gamma)
+        args = (b, x, wg, bias, w1, w2, dout, gamma, seq_balance)
         with torch.cuda.stream(self.stream):
             self._step(self.stream, *args)
         self.stream.synchronize()
@@ -231,8 +255,9 @@ class GraphStep:
         self.stream.synchronize()
 
     @staticmethod
-    def _step(s, b, x, wg, bias, w1, w2, dout, gamma):
-        forward(b, x, wg, bias, w1, w2, stream=s)
+    def _step(s, b, x, wg, bias, w1, w2, dout, gamma, seq_balance):
+        forward(b, x, wg, bias, w1, w2, stream=s,
+                seq_balance=seq_balance if dout is not None else None)
         if dout is not None:
             backward(b, x, dout, w1, w2, stream=s, wg=wg, gamma=gamma,
                      bias=bias if gamma is not None else None)

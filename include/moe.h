@@ -14,6 +14,8 @@
  *   backward: combine bwd, dX and dW grouped GEMMs             (moe_combine_bwd,
  *             grouped_gemm_bwd_dx, grouped_gemm_bwd_dw, moe_combine)
  *   router backward: dlogits, gate dX and dWg                  (moe_router_bwd)
+ *   sequence-wise balance loss and its router gradient         (moe_seq_balance_loss,
+ *                                                               moe_router_bwd_seqbal)
  *   aux-loss-free bias step                                    (moe_bias_update)
  *
  * Conventions for every call:
@@ -299,6 +301,42 @@ int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, cons
 int moe_router_bwd(const moe_dims* dims, const void* x, const float* wg, const float* probs,
                    const int32_t* topk_idx, const float* topk_w, const float* dw, float* dlogits,
                    void* dx, float* dwg, int accumulate, void* ws, size_t ws_bytes, void* stream);
+
+/* Sequence-wise balance loss and the gradient it sends into the router.
+ * Passage: dots.llm1 Technical Report, §Architecture "Load balancing": besides
+ * the aux-loss-free bias, a sequence-wise balance loss keeps a single sequence
+ * from extreme imbalance.  The pages give no formula; this is the one of the
+ * report they cite for their method (DeepSeek-V3), with this layer's softmax
+ * affinities and the batch's loss the mean over its sequences.  The T tokens
+ * form sequences of seq_len tokens (the last may be shorter); for sequence s
+ * with L_s tokens and expert e:
+ *   f[s, e] = E / (k L_s) * #{(t in s, j) : topk_idx[t, j] = e}
+ *   P[s, e] = (1 / L_s) * sum_{t in s} probs[t, e]       (probs sum to 1 per token)
+ *   loss    = alpha / n_seq * sum_s sum_e f[s, e] P[s, e]
+ *   seq_grad[s, e] = alpha f[s, e] / (n_seq L_s) = dloss / dprobs[t, e], t in s
+ * (the picks are piecewise constant: the gradient runs through P only).
+ *   topk_idx [T, k] int32, probs [T, E] f32   (moe_gate_topk's outputs)
+ * Out:
+ *   loss     [1] f32 (device)
+ *   seq_grad [ceil(T / seq_len), E] f32      for moe_router_bwd_seqbal
+ *   ws / ws_bytes                            workspace of moe_workspace_size(dims)
+ *                                            bytes (its balance-loss scratch is used)
+ * Requires seq_len >= 128 (MOE_ERR_UNSUPPORTED_SHAPE otherwise).  FP32, in a
+ * fixed order: the same inputs give the same bits.  T = 0 gives loss 0. */
+int moe_seq_balance_loss(const moe_dims* dims, int64_t seq_len, float alpha,
+                         const int32_t* topk_idx, const float* probs, float* loss,
+                         float* seq_grad, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_router_bwd with the sequence-wise balance loss's gradient included: for a
+ * token t of sequence s = t / seq_len, dp[e] += seq_grad[s, e] for every expert
+ * before the softmax backward, so dlogits, the gate's dx term and dwg carry
+ * both losses.  seq_grad and seq_len as written and used by
+ * moe_seq_balance_loss (seq_len >= 128); other arguments as in moe_router_bwd. */
+int moe_router_bwd_seqbal(const moe_dims* dims, const void* x, const float* wg,
+                          const float* probs, const int32_t* topk_idx, const float* topk_w,
+                          const float* dw, const float* seq_grad, int64_t seq_len,
+                          float* dlogits, void* dx, float* dwg, int accumulate, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /* Aux-loss-free bias step.
  * Passage: dots.llm1 Technical Report, §Architecture "Load balancing" (the

@@ -109,6 +109,16 @@ def test_validation_rejects_before_any_launch(lib):
     assert L.moe_router_bwd(ctypes.byref(ok), p, p, p, p, p, p, nul, p, nul, 0, p, big, nul) == -1
     e12 = lib.MoeDims.of(64, 128, 12, 2, 1, 64, 16)  # E % 8
     assert L.moe_router_bwd(ctypes.byref(e12), p, p, p, p, p, p, nul, p, p, 0, p, big, nul) == -2
+    # sequence-wise balance loss: seq_len >= 128, loss / seq_grad / workspace required
+    f32 = ctypes.c_float(1e-4)
+    assert L.moe_seq_balance_loss(ctypes.byref(ok), 64, f32, p, p, p, p, p, big, nul) == -2
+    assert L.moe_seq_balance_loss(ctypes.byref(ok), 128, f32, p, p, nul, p, p, big, nul) == -1
+    assert L.moe_seq_balance_loss(ctypes.byref(ok), 128, f32, p, p, p, nul, p, big, nul) == -1
+    assert L.moe_seq_balance_loss(ctypes.byref(ok), 128, f32, p, p, p, p, p, 8, nul) == -1
+    assert L.moe_router_bwd_seqbal(ctypes.byref(ok), p, p, p, p, p, p, nul, 128, nul, p, p, 0,
+                                   p, big, nul) == -1
+    assert L.moe_router_bwd_seqbal(ctypes.byref(ok), p, p, p, p, p, p, p, 100, nul, p, p, 0,
+                                   p, big, nul) == -1
     assert L.moe_bias_update(None, p, 1e-3, p, p, nul) == -1
     assert L.moe_bias_update(ctypes.byref(ok), nul, 1e-3, p, p, nul) == -1
     assert L.moe_bias_update(ctypes.byref(ok), p, 1e-3, p, nul, nul) == -1

@@ -24,23 +24,25 @@ def test_graph_replay_matches_eager(case):
     else:
         wl, inp = synth.WORKLOADS["train"], workload_inputs("train")
     dm = dims_of(wl)
+    sb = (1e-2, 128) if case == "small" else (1e-4, 8192)  # with the balance loss
     x, w1, w2 = dev(inp["x"], True), dev(inp["w1"], True), dev(inp["w2"], True)
     wg, bias, dout = dev(inp["wg"]), dev(inp["bias"]), dev(inp["dout"], True)
     eager = layer.MoEBuffers(dm, train=True)
-    layer.forward(eager, x, wg, bias, w1, w2)
+    layer.forward(eager, x, wg, bias, w1, w2, seq_balance=sb)
     layer.backward(eager, x, dout, w1, w2, wg=wg, gamma=1e-3, bias=bias)
     torch.cuda.synchronize()
-    ref = {k: getattr(eager, k).clone() for k in KEYS}
+    keys = KEYS + ("bal_loss",)
+    ref = {k: getattr(eager, k).clone() for k in keys}
     del eager
     b = layer.MoEBuffers(dm, train=True)
-    g = layer.GraphStep(b, x, wg, bias, w1, w2, dout=dout, gamma=1e-3)
+    g = layer.GraphStep(b, x, wg, bias, w1, w2, dout=dout, gamma=1e-3, seq_balance=sb)
     for _ in range(2):  # replays after the capture step rewrite every output
-        for k in KEYS:
+        for k in keys:
             getattr(b, k).zero_()
         g.replay()
         torch.cuda.synchronize()
         assert moe.moe_get_device_status(b.ws) == 0
-        for k in KEYS:
+        for k in keys:
             assert torch.equal(getattr(b, k), ref[k]), k
 
 
