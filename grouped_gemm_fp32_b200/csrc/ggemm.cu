@@ -76,6 +76,9 @@ struct GemmArgs {
   int accumulate;
   uint32_t idesc;
   uint32_t idesc_narrow;  // N = 128 (modes whose B is N-major)
+  uint32_t idesc_h;         // half tiles: the pair's M = 128 (64 rows per CTA)
+  uint32_t idesc_h_narrow;  // half tile with N = 128
+  int half_ok;              // FWD / DX modes: a group's last 128 rows run as a half tile
   int staged;             // epilogue writes through shared memory + TMA stores
   uint64_t budget_ns;
   const int32_t* gather_ids;  // FWD1 / DW1: token of each routed row, or null
@@ -108,7 +111,9 @@ constexpr size_t smem_bytes() {
 
 struct TileInfo {
   int g, m0, n0, nkb;
-  int nw;  // N of this tile's MMA: 256, or 128 for a last tile with <= 128 columns left
+  int nw;    // N of this tile's MMA: 256, or 128 for a last tile with <= 128 columns left
+  int half;  // 1: at most 128 rows of the group are left, the pair runs M = 128
+             // (64 rows per CTA) instead of computing 128 rows past the group's end
 };
 
 __device__ __forceinline__ GroupRec load_group(const GemmArgs& a, int g) {
@@ -151,6 +156,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     t.n0 = nt * 256;
     t.nkb = (load_group(a, t.g).rows_pad + BK - 1) / BK;  // the tail block reads zeros past the end
     t.nw = (a.n_out - t.n0 > 128) ? 256 : 128;
+    t.half = 0;
   } else {
     // largest g with prefix[g] * NT <= tile  (the prefix is non-decreasing)
     const int* pre = a.mtile_prefix;
@@ -174,6 +180,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     t.n0 = nt * (MODE == MODE_FWD1 ? a.hn : 256);
     t.nkb = a.K / BK;
     t.nw = (MODE == MODE_DX2 || MODE == MODE_DX1) && (a.n_out - t.n0 <= 128) ? 128 : 256;
+    t.half = a.half_ok && load_group(a, lo).rows_pad - t.m0 <= BM;
   }
   return t;
 }
@@ -261,6 +268,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                  const __grid_constant__ CUtensorMap tmC /* DX2: saved [G | U] */,
                  const __grid_constant__ CUtensorMap tmO0 /* output (FWD1: H) */,
                  const __grid_constant__ CUtensorMap tmO1 /* FWD1: saved A1 */,
+                 const __grid_constant__ CUtensorMap tmA0h /* half tiles: 64-row A boxes */,
+                 const __grid_constant__ CUtensorMap tmA1h,
+                 const __grid_constant__ CUtensorMap tmBh /* FWD1 half tiles: 64-row B boxes */,
                  const GemmArgs args) {
   constexpr bool A_MN = (MODE == MODE_DW2 || MODE == MODE_DW1);
   constexpr bool B_MN = (MODE != MODE_FWD1 && MODE != MODE_FWD2);
@@ -337,11 +347,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       constexpr bool WIDE = decltype(wide_tag)::value;
       int stage = 0;
       uint32_t phase = 0, issued = 0, lastpar = 0;
-      const int roff = (int)rank * BM;                       // this CTA's 128 rows of A
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<MODE>(tile, args);
         const GroupRec gr = load_group(args, t.g);
+        const int roff = (int)rank * (t.half ? BM / 2 : BM);  // this CTA's rows of A
         const bool shared = t.g >= args.E;
         const bool gat = WIDE && !shared;
         // this CTA's half of B: N/2 columns from n0 + rank * N/2, in 64-column chunks
@@ -349,7 +359,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         [[maybe_unused]] const int boff = (int)rank * (t.nw / 2);
         const uint32_t b_bytes = (MODE == MODE_FWD1) ? (uint32_t)(args.hn * BK * 2)
                                  : B_MN ? (uint32_t)(bchunks * 8192) : (uint32_t)B_BYTES;
-        const uint32_t pair_bytes = 2 * (A_BYTES + b_bytes);  // both CTAs' copies
+        const uint32_t a_bytes = t.half ? A_BYTES / 2 : A_BYTES;
+        const uint32_t pair_bytes = 2 * (a_bytes + b_bytes);  // both CTAs' copies
         int first = 0;
         int4 rows4 = make_int4(0, 0, 0, 0);  // the four x rows this lane gathers
         if (gat) {
@@ -376,20 +387,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           uint8_t* b_dst = sB + stage * B_BYTES;
           const int k0 = kb * BK;
           if constexpr (MODE == MODE_FWD1) {
-            // A: rows m0 + roff; B: the leader stages the gate rows, the peer the up rows
-            if (gat)
+            // A: rows m0 + roff; B: the leader stages the gate rows, the peer the up
+            // rows -- in a half tile each CTA stages 64 gate rows and the matching 64
+            // up rows, so a row's gate and up sums land in the same tensor-memory lane
+            if (gat && (!t.half || lane < 16))
               tma_gather4_pair(a_dst + lane * 512, &tmA0, fb, k0, rows4.x, rows4.y, rows4.z,
                                rows4.w);
             if (lane == 0) {
               if (!gat)
-                tma_load_2d_pair(a_dst, shared ? &tmA1 : &tmA0, fb, k0,
-                                 (shared ? 0 : gr.a_row) + t.m0 + roff);
-              tma_load_2d_pair(b_dst, &tmB0, fb, k0,
-                               t.g * args.b_group_rows + t.n0 + (leader ? 0 : args.I));
+                tma_load_2d_pair(a_dst,
+                                 t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0),
+                                 fb, k0, (shared ? 0 : gr.a_row) + t.m0 + roff);
+              const int brow = t.g * args.b_group_rows + t.n0;
+              if (t.half) {
+                tma_load_2d_pair(b_dst, &tmBh, fb, k0, brow + (int)rank * 64);
+                tma_load_2d_pair(b_dst + 8192, &tmBh, fb, k0, brow + args.I + (int)rank * 64);
+              } else {
+                tma_load_2d_pair(b_dst, &tmB0, fb, k0, brow + (leader ? 0 : args.I));
+              }
             }
           } else if constexpr (MODE == MODE_FWD2) {
-            tma_load_2d_pair(a_dst, &tmA0, fb, k0, gr.out_row + t.m0 + roff);
-            tma_load_2d_pair(b_dst, &tmB0, fb, k0, t.g * args.b_group_rows + t.n0 + roff);
+            tma_load_2d_pair(a_dst, t.half ? &tmA0h : &tmA0, fb, k0, gr.out_row + t.m0 + roff);
+            tma_load_2d_pair(b_dst, &tmB0, fb, k0,
+                             t.g * args.b_group_rows + t.n0 + (int)rank * 128);
           } else if constexpr (MODE == MODE_DX2 || MODE == MODE_DX1) {
             if constexpr (MODE == MODE_DX2) {
               // the epilogue of this tile reads the saved [G | U] of its rows: start
@@ -403,10 +423,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     tma_prefetch_l2_2d(&tmC, args.I + t.n0 + c * 64, y);
                   }
               }
-              tma_load_2d_pair(a_dst, shared ? &tmA1 : &tmA0, fb, k0,
-                               (shared ? 0 : gr.a_row) + t.m0 + roff);
+              tma_load_2d_pair(a_dst,
+                               t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0),
+                               fb, k0, (shared ? 0 : gr.a_row) + t.m0 + roff);
             } else {
-              tma_load_2d_pair(a_dst, &tmA0, fb, k0, gr.out_row + t.m0 + roff);
+              tma_load_2d_pair(a_dst, t.half ? &tmA0h : &tmA0, fb, k0, gr.out_row + t.m0 + roff);
             }
             const int brow = t.g * args.b_group_rows + k0;
             for (int c = 0; c < bchunks; ++c)
@@ -487,7 +508,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
-        const uint32_t idesc = t.nw == 256 ? args.idesc : args.idesc_narrow;
+        const uint32_t idesc = t.half ? (t.nw == 256 ? args.idesc_h : args.idesc_h_narrow)
+                                      : (t.nw == 256 ? args.idesc : args.idesc_narrow);
         for (int kb = 0; kb < t.nkb; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, abort_flag, args.status,
                          MOE_ERR_DEVICE_TIMEOUT, args.budget_ns)) {
@@ -523,10 +545,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue --
     // Warps 2..9: warp w reads tensor-memory lanes [32q, 32q + 32), q = w % 4,
-    // and the half h of the accumulator's columns.
+    // and the half h of the accumulator's columns.  A full tile gives this CTA the
+    // tile's rows rank * 128 + [0, 128), quarter q holding rows 32q..; a half tile
+    // (M = 128) gives it rows rank * 64 + [0, 64) with quarters q and q + 2 on the
+    // same 32 rows (q % 2): q < 2 the first N/2 columns, q >= 2 the last N/2, both
+    // in tensor-memory columns [0, N/2).
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
-    const int r_in_tile = (int)rank * BM + q * 32 + lane;  // row within the 256-row pair tile
     const uint32_t tempty_leader[2] = {map_to_rank(&ctl->tempty[0], 0),
                                        map_to_rank(&ctl->tempty[1], 0)};
     // hand the accumulator back to the leader's MMA thread once this warp's last
@@ -554,16 +579,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint8_t* slot = sSlots + (warp - 2) * SLOT_BYTES;
       // this warp's 32 rows within its group: all real (staged TMA stores), none,
       // or cut by the group's end (direct stores of the real rows)
-      const int rb = t.m0 + (int)rank * BM + q * 32;
+      const int qr = t.half ? (q & 1) : q;
+      const int r_in_tile = (int)rank * (t.half ? BM / 2 : BM) + qr * 32 + lane;  // row in the tile
+      const int rb = t.m0 + (int)rank * (t.half ? BM / 2 : BM) + qr * 32;
       if constexpr (MODE == MODE_FWD1) {
         const int rloc = t.m0 + r_in_tile;
         const bool rv = rloc < gr.rows_pad;
         const bool whole = rb + 32 <= gr.rows_pad;
         const int64_t orow = (int64_t)gr.out_row + rloc;
-        __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0;
+        // this warp's H columns [cb, ce), counted from H column n0 + hc0; a column's gate
+        // sum sits at tensor-memory column c, its up sum at c + uofs (a half tile: one
+        // warp per quarter takes all 64 of the quarter's H columns)
+        const int hc0 = t.half ? 64 * (q >> 1) : 0;
+        const int uofs = t.half ? 64 : args.hn;
+        const int cb = t.half ? 0 : h * (args.hn >> 1);
+        const int ce = t.half ? (h == 0 ? 64 : 0) : cb + (args.hn >> 1);
+        __nv_bfloat16* H =
+            reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0 + hc0;
         __nv_bfloat16* A1 = reinterpret_cast<__nv_bfloat16*>(args.out2);
-        const int cb = h * (args.hn >> 1), ce = cb + (args.hn >> 1);  // this warp's H columns
-        if (args.staged && whole) {
+        if (args.staged && whole && cb < ce) {
           // hn == 128: 64 H columns per warp, one 128-byte row each of H, then of the
           // saved gate and up pre-activations (read from tensor memory again)
           const int y = gr.out_row + rb;
@@ -572,7 +606,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           for (int s2 = 0; s2 < 2; ++s2) {
             uint32_t u[32];
             tmem_ld32_sync(taddr + cb + 32 * s2, r);
-            tmem_ld32_sync(taddr + args.hn + cb + 32 * s2, u);
+            tmem_ld32_sync(taddr + uofs + cb + 32 * s2, u);
             if (s2 == 1 && A1 == nullptr) release(acc);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -585,7 +619,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               slot_put(slot, lane, 4 * s2 + j, pack_bf16x8(hv));
             }
           }
-          slot_issue<false>(slot, &tmO0, t.n0 + cb, y, lane);
+          slot_issue<false>(slot, &tmO0, t.n0 + hc0 + cb, y, lane);
           if (A1 != nullptr) {
 #pragma unroll
             for (int part = 0; part < 2; ++part) {  // gate columns, then up columns
@@ -593,20 +627,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int s2 = 0; s2 < 2; ++s2) {
                 uint4 pk[4];
-                tmem_ld32_sync(taddr + part * args.hn + cb + 32 * s2, r);
+                tmem_ld32_sync(taddr + part * uofs + cb + 32 * s2, r);
                 if (part == 1 && s2 == 1) release(acc);
                 pack_acc_bf16(r, pk);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) slot_put(slot, lane, 4 * s2 + j, pk[j]);
               }
-              slot_issue<false>(slot, &tmO1, part * args.I + t.n0 + cb, y, lane);
+              slot_issue<false>(slot, &tmO1, part * args.I + t.n0 + hc0 + cb, y, lane);
             }
           }
         } else {
           for (int c0 = cb; c0 < ce; c0 += 32) {
             uint32_t u[32];
             tmem_ld32_sync(taddr + c0, r);
-            tmem_ld32_sync(taddr + args.hn + c0, u);
+            tmem_ld32_sync(taddr + uofs + c0, u);
             if (c0 + 32 >= ce) release(acc);
             if (rv) {
               float hv[32];
@@ -617,7 +651,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               }
               store_bf16x32(H + c0, hv);
               if (A1 != nullptr) {
-                __nv_bfloat16* a1r = A1 + orow * args.ld_out2 + t.n0 + c0;
+                __nv_bfloat16* a1r = A1 + orow * args.ld_out2 + t.n0 + hc0 + c0;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
                 store_bf16x32(a1r, v);
@@ -634,8 +668,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const bool rv = rloc < gr.rows_pad;
         const bool whole = rb + 32 <= gr.rows_pad;
         const int64_t orow = (int64_t)gr.out_row + rloc;
-        __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0;
-        const int cb = h * 128, ce = min(cb + 128, args.n_out - t.n0);  // multiples of 64
+        // logical column of this quarter's tensor-memory column 0, and this warp's
+        // tensor-memory columns [cb, ce) (multiples of 64)
+        const int coff = t.half ? (t.nw >> 1) * (q >> 1) : 0;
+        const int cb = t.half ? h * 64 : h * 128;
+        const int ce = t.half ? min(min(cb + 64, t.nw >> 1), args.n_out - t.n0 - coff)
+                              : min(cb + 128, args.n_out - t.n0);
+        __nv_bfloat16* O =
+            reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out + t.n0 + coff;
         for (int c0 = cb; c0 < ce; c0 += 64) {
           uint32_t u[32];
           tmem_ld32_sync(taddr + c0, r);
@@ -652,7 +692,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(u[8 * j + i]);
               pk[4 + j] = pack_bf16x8(v);
             }
-            staged_store<false>(slot, pk, &tmO0, t.n0 + c0, gr.out_row + rb, lane);
+            staged_store<false>(slot, pk, &tmO0, t.n0 + coff + c0, gr.out_row + rb, lane);
           } else if (rv) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -671,10 +711,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const __nv_bfloat16* A1 =
             reinterpret_cast<const __nv_bfloat16*>(args.aux) + orow * args.ld_aux;
         __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(args.out) + orow * args.ld_out;
-        const int cb = h * 128, ce = min(cb + 128, args.I - t.n0);  // multiples of 64
+        const int coff = t.half ? (t.nw >> 1) * (q >> 1) : 0;  // as in FWD2 / DX1
+        const int cb = t.half ? h * 64 : h * 128;
+        const int ce = t.half ? min(min(cb + 64, t.nw >> 1), args.I - t.n0 - coff)
+                              : min(cb + 128, args.I - t.n0);
         const bool staged = args.staged && whole;
         for (int c0 = cb; c0 < ce; c0 += 64) {
-          const int col = t.n0 + c0;
+          const int col = t.n0 + coff + c0;
           uint4 upk[8];  // staged: the du pieces wait here while dg goes out through the slot
           if (staged) slot_acquire(lane);
 #pragma unroll
@@ -773,8 +816,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 template <int MODE>
 int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
                 const CUtensorMap& b1, const CUtensorMap& c, const CUtensorMap& o0,
-                const CUtensorMap& o1, const GemmArgs& args,
-                cudaStream_t st) {
+                const CUtensorMap& o1, const CUtensorMap& a0h, const CUtensorMap& a1h,
+                const CUtensorMap& bh, const GemmArgs& args, cudaStream_t st) {
   static int num_sms = 0;
   static bool attr_set = false;
   constexpr size_t kSmem = smem_bytes<MODE>();
@@ -800,7 +843,8 @@ int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
     cudaGetLastError();  // a failed query only leaves the default grid
     attr_set = true;
   }
-  ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmem, st>>>(a0, a1, b0, b1, c, o0, o1, args);
+  ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmem, st>>>(a0, a1, b0, b1, c, o0, o1, a0h, a1h,
+                                                          bh, args);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -881,6 +925,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   a.budget_ns = wait_budget_ns();
 
   CUtensorMap m0{}, m1{}, n0{}, n1{}, c0{}, o0{}, o1{};
+  CUtensorMap mh0{}, mh1{}, nh{};  // half tiles: 64-row boxes of A (and of B in FWD1)
   bool ok = true;
   // a dummy map stands in for unused slots (never read by the kernel)
   auto same = [](CUtensorMap& dst, const CUtensorMap& src) { dst = src; };
@@ -908,13 +953,21 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
         ok &= make_map_bf16(&m0, ops.a0, Rr, d, BM);
       }
       if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
+      // a group's last <= 128 rows run as a half tile (M = 128), whose B rows are
+      // staged as 64 gate + 64 up rows per CTA: needs hn == 128
+      a.half_ok = hn == 128;
+      a.idesc_h = idesc_bf16_f32(BM, 2 * hn, false, false);
+      if (ops.gather_ids == nullptr) ok &= make_map_bf16(&mh0, ops.a0, Rr, d, BM / 2);
+      else same(mh0, m0);
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&mh1, ops.a1, T, d, BM / 2); else same(mh1, mh0);
+      ok &= make_map_bf16(&nh, ops.b0, (int64_t)G * 2 * I, d, BM / 2);
       if (!ok) return MOE_ERR_CUDA;
       // staged stores need 64 H columns per epilogue warp
       a.staged = hn == 128;
       ok &= make_map_2d(&o0, ops.out, Rt, I, 2, 32);
       if (ops.out2 != nullptr) ok &= make_map_2d(&o1, ops.out2, Rt, 2 * I, 2, 32); else same(o1, o0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, o0, o1, a, st);
+      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, o0, o1, mh0, mh1, nh, a, st);
     }
     case MODE_FWD2: {
       a.K = I;
@@ -927,10 +980,15 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 128);
       same(n1, n0);
+      a.half_ok = 1;
+      a.idesc_h = idesc_bf16_f32(BM, 256, false, false);
+      ok &= make_map_bf16(&mh0, ops.a0, Rt, I, BM / 2);
+      same(mh1, mh0);
+      same(nh, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, o0, o0, a, st);
+      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, a, st);
     }
     case MODE_DX2: {
       a.K = d;
@@ -946,10 +1004,16 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 64);
       same(n1, n0);
       ok &= make_map_bf16(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
+      a.half_ok = 1;
+      a.idesc_h = idesc_bf16_f32(BM, 256, false, true);
+      a.idesc_h_narrow = idesc_bf16_f32(BM, 128, false, true);
+      ok &= make_map_bf16(&mh0, ops.a0, Rr, d, BM / 2);
+      if (dm.S > 0 && T > 0) ok &= make_map_bf16(&mh1, ops.a1, T, d, BM / 2); else same(mh1, mh0);
+      same(nh, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, 2 * I, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, o0, o0, a, st);
+      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, o0, o0, mh0, mh1, nh, a, st);
     }
     case MODE_DX1: {
       a.K = 2 * I;
@@ -963,10 +1027,16 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * 2 * I, d, 64);
       same(n1, n0);
+      a.half_ok = 1;
+      a.idesc_h = idesc_bf16_f32(BM, 256, false, true);
+      a.idesc_h_narrow = idesc_bf16_f32(BM, 128, false, true);
+      ok &= make_map_bf16(&mh0, ops.a0, Rt, 2 * I, BM / 2);
+      same(mh1, mh0);
+      same(nh, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, o0, o0, a, st);
+      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, a, st);
     }
     case MODE_DW2: {  // dW2_g [d, I] = dY_g^T H_g
       a.m_out = d;
@@ -982,7 +1052,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * d, I, 4, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, a, st);
+      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, a, st);
     }
     case MODE_DW1: {  // dW1_g [2I, d] = dA_g^T X_g
       a.m_out = 2 * I;
@@ -1005,7 +1075,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * 2 * I, d, 4, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, o0, o0, a, st);
+      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, a, st);
     }
   }
   return MOE_ERR_INVALID_ARG;
