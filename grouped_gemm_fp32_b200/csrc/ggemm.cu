@@ -19,7 +19,11 @@
 //                 32-lane quarter, each on half the columns): tcgen05.ld, fused
 //                 SwiGLU / SwiGLU-backward, bf16 or f32 stores
 // with two 256-column FP32 accumulators in tensor memory per CTA so the
-// epilogue of one tile overlaps the MMAs of the next.
+// epilogue of one tile overlaps the MMAs of the next.  Segments are padded to
+// 128-row blocks, so a group's last m-tile may hold only 128 rows: it runs as a
+// half tile (the paired MMA with M = 128, 64 rows per CTA), whose accumulator
+// puts the first N/2 columns of the CTA's rows in lanes 0-63 and the last N/2
+// in lanes 64-127 of tensor-memory columns [0, N/2).
 //
 // Six GEMMs of the expert FFN share this kernel (A is M x K, B is N x K):
 //   FWD1  A = x rows (K-major)     B = W1 gate|up rows (K-major)  -> SwiGLU -> H (+ A1)
