@@ -28,11 +28,13 @@ def test_empty_batch_runs_every_call(gather):
     bias = torch.zeros(8, device="cuda")
     w1 = torch.ones(9, 128, 128, dtype=torch.bfloat16, device="cuda")
     w2 = torch.ones(9, 128, 64, dtype=torch.bfloat16, device="cuda")
-    out = layer.forward(b, x, wg, bias, w1, w2)
+    b.bal_loss.fill_(5.0)
+    out = layer.forward(b, x, wg, bias, w1, w2, seq_balance=(1e-2, 128))
     layer.backward(b, x, x, w1, w2, wg=wg, gamma=1e-3, bias=bias)
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(b.ws) == 0
     assert out.shape == (0, 128)
+    assert float(b.bal_loss.item()) == 0.0  # no sequence: loss 0
     assert torch.all(b.counts == 0)
     assert torch.all(b.dw1 == 0) and torch.all(b.dw2 == 0) and torch.all(b.dwg == 0)
     assert torch.equal(b.bias_next, bias)  # load 0 == mean load 0: sign 0, no step

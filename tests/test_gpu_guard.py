@@ -67,10 +67,12 @@ def test_no_write_outside_any_buffer(T, d, E, k, S, I, P, train, gather):
     x = g.wrap(dev(inp["x"], True))
     w1, w2 = g.wrap(dev(inp["w1"], True)), g.wrap(dev(inp["w2"], True))
     wg, bias_t = g.wrap(dev(inp["wg"])), g.wrap(dev(bias))
-    layer.forward(b, x, wg, bias_t, w1, w2)
+    # train steps include the sequence-wise balance loss (sequences of 128 tokens)
+    layer.forward(b, x, wg, bias_t, w1, w2, seq_balance=(1e-2, 128) if train else None)
     if train:
         dout = g.wrap(dev(inp["dout"], True))
         layer.backward(b, x, dout, w1, w2, wg=wg, gamma=1e-3, bias=bias_t)
+        assert b.bal_seq_len == 128
     torch.cuda.synchronize()
     assert moe.moe_get_device_status(b.ws) == 0
     assert int(b.counts[1].item()) == 0
