@@ -36,11 +36,24 @@ __device__ __forceinline__ uint4 pack8(const float* a) {
   return r;
 }
 
+// Eight accumulated columns to the output: bf16 (one 16-byte vector) or, F32,
+// the FP32 sums themselves (two).  Both take the same sums in the same order.
+template <bool F32>
+__device__ __forceinline__ void store8(void* out, int64_t i, const float* a) {
+  if constexpr (F32) {
+    float4* o = reinterpret_cast<float4*>(out) + 2 * i;
+    o[0] = make_float4(a[0], a[1], a[2], a[3]);
+    o[1] = make_float4(a[4], a[5], a[6], a[7]);
+  } else {
+    reinterpret_cast<uint4*>(out)[i] = pack8(a);
+  }
+}
+
 // out[t] = sum_j w[t, j] y[row_of[t, j]] + sum_s y[Rr + s T + t]
-template <int KMAX>
+template <int KMAX, bool F32>
 __global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
                                const float* __restrict__ w, int64_t T, int row_vec, int k, int S,
-                               int64_t Rr, uint4* __restrict__ out) {
+                               int64_t Rr, void* __restrict__ out) {
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -67,14 +80,15 @@ __global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __res
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)
       if (j < k + S) acc8(a, v[j], wt[j]);
-    out[t * row_vec + c] = pack8(a);
+    store8<F32>(out, t * row_vec + c, a);
   }
 }
 
 // Generic fallback (any k + S): rows gathered on the fly.
+template <bool F32>
 __global__ void combine_kernel_any(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
                                    const float* __restrict__ w, int64_t T, int row_vec, int k,
-                                   int S, int64_t Rr, uint4* __restrict__ out) {
+                                   int S, int64_t Rr, void* __restrict__ out) {
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -85,7 +99,7 @@ __global__ void combine_kernel_any(const uint4* __restrict__ y, const int32_t* _
       if (j < k && (r < 0 || r >= Rr)) continue;  // a pick without a row
       acc8(a, y[r * row_vec + c], j < k ? (w ? w[t * k + j] : 1.0f) : 1.0f);
     }
-    out[t * row_vec + c] = pack8(a);
+    store8<F32>(out, t * row_vec + c, a);
   }
 }
 
@@ -176,7 +190,7 @@ __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uin
 int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream);
 
 int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, const float* w,
-                   void* out, void* stream) {
+                   void* out, bool f32_out, void* stream) {
   if (dm.T == 0) return MOE_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int warps = 8;
@@ -184,12 +198,21 @@ int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, con
   const int row_vec = dm.d / 8;
   const int64_t Rr = rows_routed(dm);
   const uint4* yv = reinterpret_cast<const uint4*>(y);
-  uint4* o = reinterpret_cast<uint4*>(out);
-  if (dm.k + dm.S <= 8)
-    combine_kernel<8><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k, dm.S, Rr, o);
-  else
-    combine_kernel_any<<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k, dm.S, Rr,
-                                                      o);
+  if (dm.k + dm.S <= 8) {
+    if (f32_out)
+      combine_kernel<8, true><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
+                                                            dm.S, Rr, out);
+    else
+      combine_kernel<8, false><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
+                                                             dm.S, Rr, out);
+  } else {
+    if (f32_out)
+      combine_kernel_any<true><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
+                                                             dm.S, Rr, out);
+    else
+      combine_kernel_any<false><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
+                                                              dm.S, Rr, out);
+  }
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -242,7 +242,15 @@ int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, cons
   int rc = check_shape(dims, false);
   if (rc) return rc;
   if (dims->T > 0 && (!y || !row_of || !out)) return MOE_ERR_INVALID_ARG;
-  return launch_combine(*dims, y, row_of, topk_w, out, stream);
+  return launch_combine(*dims, y, row_of, topk_w, out, false, stream);
+}
+
+int moe_combine_f32(const moe_dims* dims, const void* y, const int32_t* row_of,
+                    const float* topk_w, float* out, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (dims->T > 0 && (!y || !row_of || !out)) return MOE_ERR_INVALID_ARG;
+  return launch_combine(*dims, y, row_of, topk_w, out, true, stream);
 }
 
 int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, const void* y,

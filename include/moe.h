@@ -260,6 +260,13 @@ int grouped_gemm_bwd_dw1_gather(const moe_dims* dims, const void* ws, const int3
 int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,
                 void* out, void* stream);
 
+/* moe_combine with the FP32 sums stored as they are, out [T, d] f32, without the
+ * final bf16 rounding (the same sums in the same order: rounding this output to
+ * bf16 gives moe_combine's bits).  For callers that keep the layer output, or
+ * dX before the router's term is added, in FP32. */
+int moe_combine_f32(const moe_dims* dims, const void* y, const int32_t* row_of,
+                    const float* topk_w, float* out, void* stream);
+
 /* Backward of the weighted combine.
  *   dout [T, d] bf16, y [Rt, d] bf16 (forward output rows), row_of, topk_w
  * Out:

@@ -80,6 +80,8 @@ def test_validation_rejects_before_any_launch(lib):
                 lib.MoeDims.of(64, 128, 8, 9, 1, 64, 16),    # k > E
                 lib.MoeDims.of(64, 128, 8, 2, 1, 64, 12)):   # P % 8
         assert L.moe_combine(ctypes.byref(bad), p, p, p, p, nul) == -2
+        assert L.moe_combine_f32(ctypes.byref(bad), p, p, p, p, nul) == -2
+    assert L.moe_combine_f32(ctypes.byref(ok), p, p, p, nul, nul) == -1
     # backward needs P % 64 == 0
     assert L.grouped_gemm_bwd_dx(ctypes.byref(ok), p, 1, p, p, p, p, p, nul) == -2
     # null pointers / bad enum / small workspace

@@ -137,3 +137,29 @@ def test_combine_unpermute_identity():
     moe.moe_combine(dm, x_perm, row_of, dev(np.ones((T, k), np.float32)), out)
     torch.cuda.synchronize()
     assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), x_np)
+
+
+@pytest.mark.parametrize("weighted", [True, False], ids=["combine", "unpermute_sum"])
+def test_combine_f32_is_the_unrounded_combine(weighted):
+    # moe_combine_f32 keeps the FP32 sums moe_combine rounds: rounding them to bf16
+    # gives moe_combine's bits, on the full layer workload (k + S = 8 rows a token)
+    name = "layer"
+    inp, b, out = _layer_forward(name)
+    dm = dims_of(synth.WORKLOADS[name])
+    w = b.topk_w if weighted else None
+    ref16 = torch.empty_like(b.out)
+    moe.moe_combine(dm, b.y, b.row_of, w, ref16)
+    out32 = torch.full((dm.T, dm.d), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_combine_f32(dm, b.y, b.row_of, w, out32)
+    torch.cuda.synchronize()
+    assert torch.equal(out32.to(torch.bfloat16).view(torch.int16), ref16.view(torch.int16))
+    if weighted:
+        assert torch.equal(ref16.view(torch.int16), out.view(torch.int16))
+        # against the oracle's combine of the GPU's own expert rows, FP64: FP32 sums
+        Y = host(b.y)
+        rof, tw = host(b.row_of), host(b.topk_w).astype(np.float64)
+        ts = np.arange(0, dm.T, 97)
+        ref = np.einsum("tj,tjd->td", tw[ts], Y[rof[ts]])
+        for s in range(dm.S):
+            ref += Y[b.Rr + s * dm.T + ts]
+        assert np.max(np.abs(host(out32)[ts] - ref)) <= 1e-5 * np.abs(ref).max()
