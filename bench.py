@@ -69,6 +69,10 @@ def parse():
     ap.add_argument("--gather", action="store_true",
                     help="the first GEMM and dW1 gather x rows through sorted_ids instead of "
                          "reading the permuted copy x_perm")
+    ap.add_argument("--library-gemm", action="store_true",
+                    help="context, not the contract line: cuBLAS (torch.bmm) on the same GEMM "
+                         "shapes with uniform groups, timed interleaved with this library's "
+                         "grouped-GEMM calls (1 GPU, train workload)")
     return ap.parse_args()
 
 
@@ -604,8 +608,108 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_library_gemm(args, rounds=8, timed=3):
+    """cuBLAS on the grouped GEMMs' shapes, for context.  Every expert gets exactly
+    T*k/E rows (cuBLAS has no ragged batches), the shared experts T rows; operands are
+    bf16, outputs bf16 (this library writes the dW in f32 and fuses SwiGLU and its
+    backward into its epilogues, which cuBLAS does not do here).  The weights are the
+    workload's own tensors, passed as (transposed) views.  Each round times every
+    mode once with cuBLAS and once with this library, back to back, so both see the
+    same clocks; the line reports medians over the rounds and the median of the
+    per-round ratios."""
+    import torch
+    import grouped_gemm_fp32_b200 as moe
+    from grouped_gemm_fp32_b200 import layer
+
+    wl, inp = workload("train")
+    dm = wl.dims
+    T, d, E, k, S, I = dm.T, dm.d, dm.E, dm.k, dm.S, dm.I
+    assert (T * k) % E == 0
+    Mr = T * k // E
+    dims = moe.MoeDims.of(T, d, E, k, S, I, dm.P, dm.rows_cap)
+    dev = torch.device("cuda", 0)
+    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
+    x, w1, w2, dout = bf(inp["x"]), bf(inp["w1"]), bf(inp["w2"]), bf(inp["dout"])
+    wg, bias = torch.from_numpy(inp["wg"]).to(dev), torch.from_numpy(inp["bias"]).to(dev)
+    b = layer.MoEBuffers(dims, device=dev, train=True)
+    layer.forward(b, x, wg, bias, w1, w2)
+    layer.backward(b, x, dout, w1, w2)
+    torch.cuda.synchronize()
+
+    g = torch.Generator(device=dev).manual_seed(11)
+    rnd = lambda *s: torch.randn(*s, device=dev, generator=g).to(torch.bfloat16)
+    w1r, w1s, w2r, w2s = w1[:E], w1[E:], w2[:E], w2[E:]
+    ops = {  # mode: ((A, B) routed, (A, B) shared)
+        "fwd1": ((rnd(E, Mr, d), w1r.transpose(1, 2)), (rnd(S, T, d), w1s.transpose(1, 2))),
+        "fwd2": ((rnd(E, Mr, I), w2r.transpose(1, 2)), (rnd(S, T, I), w2s.transpose(1, 2))),
+        "dx2": ((rnd(E, Mr, d), w2r), (rnd(S, T, d), w2s)),
+        "dx1": ((rnd(E, Mr, 2 * I), w1r), (rnd(S, T, 2 * I), w1s)),
+        "dw2": ((rnd(E, Mr, d).transpose(1, 2), rnd(E, Mr, I)),
+                (rnd(S, T, d).transpose(1, 2), rnd(S, T, I))),
+        "dw1": ((rnd(E, Mr, 2 * I).transpose(1, 2), rnd(E, Mr, d)),
+                (rnd(S, T, 2 * I).transpose(1, 2), rnd(S, T, d))),
+    }
+    L = moe
+    ours = {
+        "fwd1+fwd2": lambda: L.grouped_gemm_fwd(dims, b.ws, b.x_perm, x, w1, w2, b.h, b.a1, b.y),
+        "dx2": lambda: L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM2, b.dy, dout, w2, b.a1, b.da),
+        "dw2": lambda: L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM2, b.dy, dout, b.h, None,
+                                             b.dw2, 0),
+        "dx1": lambda: L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp),
+        "dw1": lambda: L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, x,
+                                             b.dw1, 0),
+    }
+    lib = {
+        "fwd1+fwd2": lambda: [torch.bmm(*ops[m][j]) for m in ("fwd1", "fwd2") for j in (0, 1)],
+        **{m: (lambda m=m: [torch.bmm(*ops[m][j]) for j in (0, 1)])
+           for m in ("dx2", "dw2", "dx1", "dw1")},
+    }
+    fl = gemm_flops(dm, True)
+    flops = {"fwd1+fwd2": fl["fwd"], **{m: fl[m] for m in ("dx2", "dw2", "dx1", "dw1")}}
+
+    def t_ms(f):
+        f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(timed):
+            f()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / timed
+
+    res = {m: {"cublas": [], "ours": []} for m in ours}
+    for r in range(rounds):
+        for m in ours:
+            pair = [("cublas", lib[m]), ("ours", ours[m])]
+            for name, f in (pair if r % 2 == 0 else pair[::-1]):
+                res[m][name].append(t_ms(f))
+    med = lambda v: sorted(v)[len(v) // 2]
+    modes = {}
+    for m, v in res.items():
+        c, o = med(v["cublas"]), med(v["ours"])
+        modes[m] = {"cublas_ms": round(c, 4), "ours_ms": round(o, 4),
+                    "cublas_tflops": round(flops[m] / c / 1e9, 1),
+                    "ours_tflops": round(flops[m] / o / 1e9, 1),
+                    "ours_over_cublas_time": round(med([a / b_ for a, b_ in
+                                                        zip(v["ours"], v["cublas"])]), 3)}
+    line = {"library_gemm": "cuBLAS torch.bmm, bf16 in/out, f32 accumulate, uniform groups",
+            "workload": f"train GEMM shapes: {E} routed experts x {Mr} rows + {S} shared x {T} "
+                        f"rows, d={d}, I={I}",
+            "rounds": rounds, "timed_per_round": timed, "modes": modes,
+            "total_ms": {"cublas": round(sum(v["cublas_ms"] for v in modes.values()), 3),
+                         "ours": round(sum(v["ours_ms"] for v in modes.values()), 3)},
+            "note": "ours: ragged groups padded to 128 rows (the routing of the workload's own "
+                    "batch), SwiGLU / SwiGLU-backward epilogues, saved activations, f32 dW; "
+                    "cuBLAS: plain products, bf16 outputs"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.library_gemm:
+        run_library_gemm(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
