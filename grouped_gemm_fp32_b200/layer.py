@@ -16,6 +16,9 @@ and "Load balancing"; §3.2 "Efficient implementation of Grouped GEMM"):
               [-> moe_bias_update (next step's selection bias)]
 The router backward runs when the gate weights are passed to ``backward``; the
 bias step when an update speed ``gamma`` is.
+Under token data parallelism, ``dp_bias_step`` (the bias step on the whole batch's
+loads) and ``dp_allreduce_grads`` (the weight gradients' sum) exchange what the
+ranks share, over torch.distributed.
 """
 from __future__ import annotations
 
@@ -141,6 +144,68 @@ def backward(b: MoEBuffers, x, dout, w1, w2, stream=None, wg=None, gamma=None, b
     if gamma is not None:
         L.moe_bias_update(dm, b.counts, gamma, bias, b.bias_next, stream)
     return b.dx, b.dw1, b.dw2, b.dw_comb
+
+
+# ------------------------------------------------------------- data parallel --
+# Token data parallelism: every rank holds the same weights and its own tokens.
+# The layer's forward and backward need nothing from the other ranks; two steps
+# do.  The bias step balances the loads of the whole batch, i.e. of all ranks'
+# tokens (dots.llm1 Technical Report, §"Load balancing": the bias follows the
+# experts' loads).  The weight gradients of the batch are the sums of the ranks'
+# own.  Both are all-reduces over torch.distributed (NCCL between GPUs), issued
+# on the layer's stream.
+
+def _on_stream(stream):
+    return torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else _Null()
+
+
+class _Null:
+    def __enter__(self):
+        return None
+
+    def __exit__(self, *a):
+        return False
+
+
+def dp_load_counts(counts, group=None, stream=None):
+    """Per-expert loads of the whole data-parallel batch: ``counts`` (int32 [E], this
+    rank's tokens per expert, as moe_permute_align writes them) summed over the ranks
+    of ``group``.  Returns a new tensor; ``counts`` itself is left as it is (the
+    backward GEMMs still read it)."""
+    import torch.distributed as dist
+    with _on_stream(stream):
+        total = counts.clone()
+        dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
+    return total
+
+
+def dp_dims(dims: L.MoeDims, world: int) -> L.MoeDims:
+    """The dims of the whole data-parallel batch: ``world`` ranks of ``dims.T`` tokens
+    each (every rank must hold the same number of tokens)."""
+    return L.MoeDims.of(dims.T * world, dims.d, dims.E, dims.k, dims.S, dims.I, dims.P,
+                        dims.rows_cap)
+
+
+def dp_bias_step(b: MoEBuffers, gamma, bias, group=None, stream=None):
+    """The aux-loss-free bias step on the loads of the whole batch:
+    ``b.bias_next = bias + gamma * sign(mean - load)`` with load = the experts' token
+    counts summed over the ranks of ``group`` and mean = world·T·k/E.  Every rank
+    gets the same ``b.bias_next``.  Returns the summed counts."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    total = dp_load_counts(b.counts, group, stream)
+    L.moe_bias_update(dp_dims(b.dims, world), total, gamma, bias, b.bias_next, stream)
+    return total
+
+
+def dp_allreduce_grads(grads, group=None, stream=None):
+    """Sum each gradient tensor (e.g. ``b.dw1``, ``b.dw2``, ``b.dwg``) over the ranks
+    of ``group``, in place: the gradients of the whole data-parallel batch."""
+    import torch.distributed as dist
+    with _on_stream(stream):
+        for g in grads:
+            dist.all_reduce(g, op=dist.ReduceOp.SUM, group=group)
+    return grads
 
 
 class HostPipeline:

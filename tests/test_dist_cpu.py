@@ -80,3 +80,63 @@ def test_reference_arm_under_torchrun_prints_once():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
     assert rec["value"] > 0 and rec["cpu_baseline"]["kind"] == "oracle"
+
+
+def _dp_worker(rank, world, port, q):
+    """Data-parallel exchange steps of the layer (grouped_gemm_fp32_b200.layer.dp_*) on
+    gloo: the whole batch's expert loads, the bias step they drive, the gradient sum."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    import bench
+    import oracle
+    from grouped_gemm_fp32_b200 import layer
+    w, r, _ = bench.dist_setup(types.SimpleNamespace(impl="reference"))  # gloo
+    wl, inp = bench.workload("tiny")
+    mine = bench.rank_shard(wl, inp, r)
+    dm = wl.dims
+    logits = oracle.gate_logits(mine["x"], mine["wg"])
+    _, idx, _, _ = oracle.route(logits, mine["bias"], dm.k)
+    counts = torch.from_numpy(np.bincount(idx.ravel(), minlength=dm.E).astype(np.int32))
+    before = counts.clone()
+    total = layer.dp_load_counts(counts)
+    every = [None] * w
+    dist.all_gather_object(every, idx)
+    whole = np.concatenate(every, axis=0)
+    # the bias step on the summed loads with the whole batch's token count, as the
+    # kernel applies it (bias + gamma * sign(T_all k - load E)), against the oracle's
+    # step on the concatenated batch
+    import grouped_gemm_fp32_b200 as moe
+    gdims = layer.dp_dims(moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P), w)
+    gamma = float(np.float32(1e-3))  # the step speed is an f32 on both sides
+    diff = gdims.T * dm.k - total.numpy().astype(np.int64) * dm.E
+    step = mine["bias"].astype(np.float64) + gamma * np.sign(diff)
+    ref = oracle.bias_update(whole, dm.E, mine["bias"], gamma)
+    g = torch.full((3, 4), float(rank + 1))
+    layer.dp_allreduce_grads([g])
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, torch.equal(counts, before), total.numpy().tolist(),
+           np.bincount(whole.ravel(), minlength=dm.E).tolist(), int(gdims.T),
+           float(np.abs(step - ref).max()), g.numpy().tolist()))
+
+
+def test_data_parallel_loads_bias_step_and_gradient_sum():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, untouched, total, whole_counts, T_all, step_err, g in out:
+        assert untouched                       # the rank's own counts stay as they were
+        assert total == whole_counts           # loads of the concatenated batch
+        assert T_all == 2 * 64                 # tiny workload: 64 tokens per rank
+        assert step_err == 0.0                 # the sign step on the whole batch's loads
+        assert g == [[3.0] * 4] * 3            # 1 + 2, on every rank
