@@ -10,6 +10,7 @@ from ._lib import (MOE_GEMM1, MOE_GEMM2, MoeDims, MoeError, grouped_gemm_bwd_dw,
                    grouped_gemm_bwd_dw1_gather, grouped_gemm_bwd_dx, grouped_gemm_fwd,
                    grouped_gemm_fwd_gather, grouped_gemm_set_groups, lib_path,
                    load, moe_bias_update, moe_combine, moe_combine_bwd, moe_combine_f32,
+                   moe_combine_split,
                    moe_gate_topk, moe_get_device_status, moe_last_cuda_error, moe_permute_align,
                    moe_permute_align_static, moe_router_bwd, moe_router_bwd_seqbal,
                    moe_rows_routed, moe_rows_total, moe_seq_balance_loss, moe_status_string,

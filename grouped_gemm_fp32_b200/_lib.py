@@ -18,7 +18,7 @@ EXPORTS = (
     "moe_rows_routed", "moe_rows_total", "moe_workspace_size", "moe_gate_topk",
     "moe_permute_align", "moe_permute_align_static", "grouped_gemm_set_groups",
     "grouped_gemm_fwd", "grouped_gemm_fwd_gather", "grouped_gemm_bwd_dx", "grouped_gemm_bwd_dw",
-    "grouped_gemm_bwd_dw1_gather", "moe_combine", "moe_combine_f32",
+    "grouped_gemm_bwd_dw1_gather", "moe_combine", "moe_combine_split", "moe_combine_f32",
     "moe_combine_bwd", "moe_router_bwd", "moe_router_bwd_seqbal", "moe_seq_balance_loss",
     "moe_bias_update", "moe_get_device_status",
     "moe_status_string", "moe_last_cuda_error",
@@ -78,6 +78,7 @@ def load():
         "grouped_gemm_bwd_dw": (i32, [D, vp, i32, vp, vp, vp, vp, vp, i32, vp]),
         "moe_combine": (i32, [D, vp, vp, vp, vp, vp]),
         "moe_combine_f32": (i32, [D, vp, vp, vp, vp, vp]),
+        "moe_combine_split": (i32, [D, vp, vp, vp, vp, vp, vp]),
         "moe_router_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
         "moe_router_bwd_seqbal": (i32, [D, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, i32, vp,
                                         sz, vp]),
@@ -200,6 +201,11 @@ def grouped_gemm_bwd_dw1_gather(dims, ws, sorted_ids, da, x, dw1, accumulate=0, 
 def moe_combine(dims, y, row_of, topk_w, out, stream=None):
     _ck(load().moe_combine(ctypes.byref(dims), _p(y), _p(row_of), _p(topk_w), _p(out),
                            _s(stream)), "moe_combine")
+
+
+def moe_combine_split(dims, y_routed, y_shared, row_of, topk_w, out, stream=None):
+    _ck(load().moe_combine_split(ctypes.byref(dims), _p(y_routed), _p(y_shared), _p(row_of),
+                                 _p(topk_w), _p(out), _s(stream)), "moe_combine_split")
 
 
 def moe_combine_f32(dims, y, row_of, topk_w, out, stream=None):

@@ -49,25 +49,27 @@ __device__ __forceinline__ void store8(void* out, int64_t i, const float* a) {
   }
 }
 
-// out[t] = sum_j w[t, j] y[row_of[t, j]] + sum_s y[Rr + s T + t]
+// out[t] = sum_j w[t, j] y[row_of[t, j]] + sum_s ys[s T + t]  (ys = y + Rr rows when the
+// shared experts' rows follow the routed ones in one buffer)
 template <int KMAX, bool F32>
-__global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
-                               const float* __restrict__ w, int64_t T, int row_vec, int k, int S,
-                               int64_t Rr, void* __restrict__ out) {
+__global__ void combine_kernel(const uint4* __restrict__ y, const uint4* __restrict__ ys,
+                               const int32_t* __restrict__ row_of, const float* __restrict__ w,
+                               int64_t T, int row_vec, int k, int S, int64_t Rr,
+                               void* __restrict__ out) {
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  int64_t rows[KMAX];
+  const uint4* src[KMAX];
   float wt[KMAX];
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     if (j < k) {
       const int32_t r = row_of[t * k + j];
       const bool ok = r >= 0 && r < Rr;  // -1 (a pick without a row) or stale: skipped
-      rows[j] = ok ? (int64_t)r * row_vec : 0;
+      src[j] = y + (ok ? (int64_t)r * row_vec : 0);
       wt[j] = ok ? (w ? w[t * k + j] : 1.0f) : 0.0f;
     } else if (j < k + S) {
-      rows[j] = (Rr + (int64_t)(j - k) * T + t) * row_vec;
+      src[j] = ys + ((int64_t)(j - k) * T + t) * row_vec;
       wt[j] = 1.0f;
     }
   }
@@ -76,7 +78,7 @@ __global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __res
     uint4 v[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)
-      if (j < k + S) v[j] = y[rows[j] + c];
+      if (j < k + S) v[j] = src[j][c];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)
       if (j < k + S) acc8(a, v[j], wt[j]);
@@ -86,18 +88,23 @@ __global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __res
 
 // Generic fallback (any k + S): rows gathered on the fly.
 template <bool F32>
-__global__ void combine_kernel_any(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
-                                   const float* __restrict__ w, int64_t T, int row_vec, int k,
-                                   int S, int64_t Rr, void* __restrict__ out) {
+__global__ void combine_kernel_any(const uint4* __restrict__ y, const uint4* __restrict__ ys,
+                                   const int32_t* __restrict__ row_of, const float* __restrict__ w,
+                                   int64_t T, int row_vec, int k, int S, int64_t Rr,
+                                   void* __restrict__ out) {
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   for (int c = lane; c < row_vec; c += 32) {
     float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int j = 0; j < k + S; ++j) {
-      const int64_t r = j < k ? (int64_t)row_of[t * k + j] : Rr + (int64_t)(j - k) * T + t;
-      if (j < k && (r < 0 || r >= Rr)) continue;  // a pick without a row
-      acc8(a, y[r * row_vec + c], j < k ? (w ? w[t * k + j] : 1.0f) : 1.0f);
+      if (j < k) {
+        const int64_t r = row_of[t * k + j];
+        if (r < 0 || r >= Rr) continue;  // a pick without a row
+        acc8(a, y[r * row_vec + c], w ? w[t * k + j] : 1.0f);
+      } else {
+        acc8(a, ys[((int64_t)(j - k) * T + t) * row_vec + c], 1.0f);
+      }
     }
     store8<F32>(out, t * row_vec + c, a);
   }
@@ -189,8 +196,8 @@ __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uin
 
 int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream);
 
-int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, const float* w,
-                   void* out, bool f32_out, void* stream) {
+int launch_combine(const moe_dims& dm, const void* y, const void* y_shared,
+                   const int32_t* row_of, const float* w, void* out, bool f32_out, void* stream) {
   if (dm.T == 0) return MOE_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int warps = 8;
@@ -198,20 +205,22 @@ int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, con
   const int row_vec = dm.d / 8;
   const int64_t Rr = rows_routed(dm);
   const uint4* yv = reinterpret_cast<const uint4*>(y);
+  // the shared experts' rows: their own buffer, or the rows after the routed ones
+  const uint4* ys = y_shared ? reinterpret_cast<const uint4*>(y_shared) : yv + Rr * row_vec;
   if (dm.k + dm.S <= 8) {
     if (f32_out)
-      combine_kernel<8, true><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
-                                                            dm.S, Rr, out);
+      combine_kernel<8, true><<<blocks, warps * 32, 0, st>>>(yv, ys, row_of, w, dm.T, row_vec,
+                                                            dm.k, dm.S, Rr, out);
     else
-      combine_kernel<8, false><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
-                                                             dm.S, Rr, out);
+      combine_kernel<8, false><<<blocks, warps * 32, 0, st>>>(yv, ys, row_of, w, dm.T, row_vec,
+                                                             dm.k, dm.S, Rr, out);
   } else {
     if (f32_out)
-      combine_kernel_any<true><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
-                                                             dm.S, Rr, out);
+      combine_kernel_any<true><<<blocks, warps * 32, 0, st>>>(yv, ys, row_of, w, dm.T, row_vec,
+                                                             dm.k, dm.S, Rr, out);
     else
-      combine_kernel_any<false><<<blocks, warps * 32, 0, st>>>(yv, row_of, w, dm.T, row_vec, dm.k,
-                                                              dm.S, Rr, out);
+      combine_kernel_any<false><<<blocks, warps * 32, 0, st>>>(yv, ys, row_of, w, dm.T, row_vec,
+                                                              dm.k, dm.S, Rr, out);
   }
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -242,7 +242,17 @@ int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, cons
   int rc = check_shape(dims, false);
   if (rc) return rc;
   if (dims->T > 0 && (!y || !row_of || !out)) return MOE_ERR_INVALID_ARG;
-  return launch_combine(*dims, y, row_of, topk_w, out, false, stream);
+  return launch_combine(*dims, y, nullptr, row_of, topk_w, out, false, stream);
+}
+
+int moe_combine_split(const moe_dims* dims, const void* y_routed, const void* y_shared,
+                      const int32_t* row_of, const float* topk_w, void* out, void* stream) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (dims->T > 0 && (!y_routed || !row_of || !out || (dims->S > 0 && !y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  return launch_combine(*dims, y_routed, dims->S > 0 ? y_shared : y_routed, row_of, topk_w, out,
+                        false, stream);
 }
 
 int moe_combine_f32(const moe_dims* dims, const void* y, const int32_t* row_of,
@@ -250,7 +260,7 @@ int moe_combine_f32(const moe_dims* dims, const void* y, const int32_t* row_of,
   int rc = check_shape(dims, false);
   if (rc) return rc;
   if (dims->T > 0 && (!y || !row_of || !out)) return MOE_ERR_INVALID_ARG;
-  return launch_combine(*dims, y, row_of, topk_w, out, true, stream);
+  return launch_combine(*dims, y, nullptr, row_of, topk_w, out, true, stream);
 }
 
 int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, const void* y,

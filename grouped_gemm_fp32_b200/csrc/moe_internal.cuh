@@ -126,8 +126,8 @@ int launch_gate_dx(const moe_dims& dm, const void* dl_planes, const void* wg_pla
                    int* status, void* stream);
 int launch_gate_dw(const moe_dims& dm, const void* dl_planes, const void* x, float* partial,
                    int* status, void* stream);
-int launch_combine(const moe_dims& dm, const void* y, const int32_t* row_of, const float* w,
-                   void* out, bool f32_out, void* stream);
+int launch_combine(const moe_dims& dm, const void* y, const void* y_shared,
+                   const int32_t* row_of, const float* w, void* out, bool f32_out, void* stream);
 int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
                        const int32_t* row_of, const float* w, void* dy, float* dw, void* stream);
 

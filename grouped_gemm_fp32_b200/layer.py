@@ -29,12 +29,16 @@ from . import _lib as L
 
 class MoEBuffers:
     def __init__(self, dims: L.MoeDims, device="cuda", train: bool = False,
-                 gather: bool = False):
+                 gather: bool = False, experts: bool = True):
         """``gather``: the first GEMM (and dW1) read the routed x rows straight from x
         through ``sorted_ids`` (grouped_gemm_fwd_gather / grouped_gemm_bwd_dw1_gather)
         and no x_perm [Rr, d] is allocated; otherwise (the default, faster on B200:
         the row copy costs less than the four-row gather copies) they read the
-        permuted copy ``x_perm`` that moe_permute_align writes."""
+        permuted copy ``x_perm`` that moe_permute_align writes.
+        ``experts=False``: the buffers of a rank whose routed rows are computed
+        elsewhere (expert parallelism): routing, permutation, combine and router
+        buffers, with y, dy and dxp holding the routed rows only [Rr, d]; no
+        expert activations (h, a1, da) and no expert weight gradients."""
         self.dims = dims
         self.train = train
         self.gather = gather
@@ -55,18 +59,19 @@ class MoEBuffers:
         self.sorted_ids = e(self.Rr, dt=i32)
         self.row_of = e(T, k, dt=i32)
         self.x_perm = None if gather else e(self.Rr, d)
-        self.h = e(self.Rt, I)
-        self.a1 = e(self.Rt, 2 * I) if train else None
-        self.y = e(self.Rt, d)
+        rows = self.Rt if experts else self.Rr
+        self.h = e(self.Rt, I) if experts else None
+        self.a1 = e(self.Rt, 2 * I) if train and experts else None
+        self.y = e(rows, d)
         self.out = e(T, d)
         if train:
             self.dy = e(self.Rr, d)
             self.dw_comb = e(T, k, dt=f32)
-            self.da = e(self.Rt, 2 * I)
-            self.dxp = e(self.Rt, d)
+            self.da = e(self.Rt, 2 * I) if experts else None
+            self.dxp = e(rows, d)
             self.dx = e(T, d)
-            self.dw1 = e(G, 2 * I, d, dt=f32)
-            self.dw2 = e(G, d, I, dt=f32)
+            self.dw1 = e(G, 2 * I, d, dt=f32) if experts else None
+            self.dw2 = e(G, d, I, dt=f32) if experts else None
             self.probs = e(T, E, dt=f32)
             self.dwg = e(E, d, dt=f32)
             self.bias_next = e(E, dt=f32)

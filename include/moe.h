@@ -17,6 +17,7 @@
  *   sequence-wise balance loss and its router gradient         (moe_seq_balance_loss,
  *                                                               moe_router_bwd_seqbal)
  *   aux-loss-free bias step                                    (moe_bias_update)
+ *   combine with the shared rows apart (expert parallelism)    (moe_combine_split)
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -259,6 +260,18 @@ int grouped_gemm_bwd_dw1_gather(const moe_dims* dims, const void* ws, const int3
  * nothing. */
 int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,
                 void* out, void* stream);
+
+/* moe_combine with the shared experts' rows in a buffer of their own:
+ *   out[t] = sum_j topk_w[t, j] * y_routed[row_of[t, j]] + sum_s y_shared[s*T + t]
+ * y_routed [Rr, d] bf16 (the routed rows of the grouped row space), y_shared
+ * [S, T, d] bf16 (NULL only when S = 0).  The sums, their order and the
+ * rounding are moe_combine's; with y_shared = y_routed + Rr rows the result is
+ * moe_combine's bit for bit.  Used under expert parallelism, where a rank's
+ * routed rows come back from the experts' owners into one buffer while its
+ * shared experts' rows stay in the buffer of its local grouped GEMM.
+ * topk_w = NULL: the un-permute-sum, as in moe_combine. */
+int moe_combine_split(const moe_dims* dims, const void* y_routed, const void* y_shared,
+                      const int32_t* row_of, const float* topk_w, void* out, void* stream);
 
 /* moe_combine with the FP32 sums stored as they are, out [T, d] f32, without the
  * final bf16 rounding (the same sums in the same order: rounding this output to

@@ -82,6 +82,9 @@ def test_validation_rejects_before_any_launch(lib):
         assert L.moe_combine(ctypes.byref(bad), p, p, p, p, nul) == -2
         assert L.moe_combine_f32(ctypes.byref(bad), p, p, p, p, nul) == -2
     assert L.moe_combine_f32(ctypes.byref(ok), p, p, p, nul, nul) == -1
+    # split combine: the shared rows' buffer is required when S > 0
+    assert L.moe_combine_split(ctypes.byref(ok), p, nul, p, p, p, nul) == -1
+    assert L.moe_combine_split(ctypes.byref(ok), nul, p, p, p, p, nul) == -1
     # backward needs P % 64 == 0
     assert L.grouped_gemm_bwd_dx(ctypes.byref(ok), p, 1, p, p, p, p, p, nul) == -2
     # null pointers / bad enum / small workspace

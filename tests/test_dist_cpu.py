@@ -140,3 +140,71 @@ def test_data_parallel_loads_bias_step_and_gradient_sum():
         assert T_all == 2 * 64                 # tiny workload: 64 tokens per rank
         assert step_err == 0.0                 # the sign step on the whole batch's loads
         assert g == [[3.0] * 4] * 3            # 1 + 2, on every rank
+
+
+def _ep_worker(rank, world, port, q):
+    """Expert-parallel exchange (grouped_gemm_fp32_b200.ep) on gloo with CPU tensors:
+    counts all-to-all, dispatch of padded segments to their owners (expert-major), and
+    the return of the owners' rows into each source's permuted layout."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from grouped_gemm_fp32_b200 import ep
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    E, P, d = 6 * world, 8, 4
+    El = E // world
+    rng = np.random.default_rng(100 + rank)
+    counts = rng.integers(0, 20, size=E).astype(np.int32)
+    counts[rank] = 0                                   # some empty segments
+    ct = torch.from_numpy(counts)
+    counts_in = torch.empty_like(ct)
+    dist.all_to_all_single(counts_in, ct)
+    plan = ep.EPPlan(counts, counts_in.numpy(), rank, world, P)
+    # permuted rows: row i of expert g's segment holds (rank, g, i), pad rows -1
+    x_perm = torch.full((plan.send_rows, d), -1.0)
+    for o, e, a, n in plan.to_owner:
+        g = o * El + e
+        for i in range(counts[g]):
+            x_perm[a + i] = torch.tensor([rank, g, i, 0.0])
+    x_recv = torch.full((plan.recv_rows, d), -7.0)
+    ep.exchange(*ep.dispatch_lists(plan, x_perm, x_recv), rank)
+    ok_dispatch = True
+    for s, e, a, n in plan.from_source:
+        c = int(counts_in.view(world, El)[s, e])
+        for i in range(n):
+            want = [s, rank * El + e, i, 0.0] if i < c else [-1.0] * 4
+            ok_dispatch &= x_recv[a + i].tolist() == want
+    # the owner's "expert" marks each row; the source must get its rows back in place
+    y_loc = x_recv.clone()
+    y_loc[:, 3] = 100.0 + rank
+    y_full = torch.full((plan.send_rows, d), -9.0)
+    ep.exchange(*ep.return_lists(plan, y_loc, y_full), rank)
+    ok_return = True
+    for o, e, a, n in plan.to_owner:
+        g = o * El + e
+        for i in range(n):
+            want = ([rank, g, i] if i < counts[g] else [-1.0] * 3) + [100.0 + o]
+            ok_return &= y_full[a + i].tolist() == want
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, ok_dispatch, ok_return, plan.recv_rows, int(plan.local_counts.sum())))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_expert_parallel_exchange_moves_segments_both_ways(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok_dispatch, ok_return, recv_rows, local_rows in out:
+        assert ok_dispatch, rank
+        assert ok_return, rank
+        assert recv_rows == local_rows
