@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--gather", action="store_true",
                     help="the first GEMM and dW1 gather x rows through sorted_ids instead of "
                          "reading the permuted copy x_perm")
+    ap.add_argument("--ep", action="store_true",
+                    help="a line of its own: the train step under expert parallelism over the "
+                         "ranks (one rank: every segment exchange a local copy)")
     ap.add_argument("--library-gemm", action="store_true",
                     help="context, not the contract line: cuBLAS (torch.bmm) on the same GEMM "
                          "shapes with uniform groups, timed interleaved with this library's "
@@ -705,8 +708,87 @@ def run_library_gemm(args, rounds=8, timed=3):
     print(json.dumps(line), flush=True)
 
 
+def run_ep(args):
+    """The train step under expert parallelism (grouped_gemm_fp32_b200.ep): every rank
+    routes its own T tokens over all E experts and owns E / W of them, the padded
+    segments travel to their owners and back by NCCL send/recv.  With one process the
+    group has one rank (every segment a local copy): the EP code path with no link
+    traffic.  The step runs as eager calls (the segment sizes come to the host once per
+    step, so it is not captured in a graph).  A line of its own, not the contract's."""
+    import torch
+    import torch.distributed as dist
+    import grouped_gemm_fp32_b200 as moe
+    from grouped_gemm_fp32_b200 import ep
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    if world == 1:
+        dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                                device_id=dev)
+    wl, inp = workload("train")
+    inp = rank_shard(wl, inp, rank)
+    dm = wl.dims
+    E, El = dm.E, dm.E // world
+    dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
+    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
+    x, dout = bf(inp["x"]), bf(inp["dout"])
+    w1, w2 = bf(inp["w1"]), bf(inp["w2"])
+    w1l = torch.cat([w1[rank * El:(rank + 1) * El], w1[E:]]).contiguous()
+    w2l = torch.cat([w2[rank * El:(rank + 1) * El], w2[E:]]).contiguous()
+    del w1, w2
+    wg, bias = torch.from_numpy(inp["wg"]).to(dev), torch.from_numpy(inp["bias"]).to(dev)
+    eb = ep.EPBuffers(dims, rank, world, train=True, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        ep.forward(eb, x, wg, bias, w1l, w2l, stream=stream, seq_balance=SEQ_BALANCE)
+        ep.backward(eb, x, dout, w1l, w2l, stream=stream, wg=wg, gamma=GAMMA, bias=bias)
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    for buf in (eb.full.ws, eb.loc.ws):
+        status = moe.moe_get_device_status(buf, stream)
+        if status != 0:
+            raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(status)}")
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.25)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    barrier(world)
+    clocks = clk.stop()
+    ms = dist_max(e0.elapsed_time(e1) / args.steps, world, dev)
+    recv = dist_max(float(eb.plan.recv_rows), world, dev)
+    if rank == 0:
+        line = {"metric": METRIC, "value": world * dm.T / (ms / 1000.0), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours-ep",
+                "config": {"workload": describe(wl) + ", expert parallel",
+                           "parallelism": f"ep{world}", "experts_per_rank": El,
+                           "tokens_per_gpu": dm.T, "seq_balance": {"alpha": SEQ_BALANCE[0],
+                                                                   "seq_len": SEQ_BALANCE[1]},
+                           "max_rows_received": int(recv),
+                           "step": "eager C-ABI calls; counts all-to-all, segment send/recv "
+                                   "over NCCL, segment sizes to the host once per step"},
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    dist.destroy_process_group()
+
+
 def main():
     args = parse()
+    if args.ep:
+        run_ep(args)
+        return
     if args.library_gemm:
         run_library_gemm(args)
         return
