@@ -35,6 +35,12 @@
 //   all warps        routing, one warp per token: softmax (max-subtracted, expf),
 //                    s = p + bias, k rounds of a warp-shuffle arg-max (equal s ->
 //                    lower index), the renormalised weights
+// With fewer 128-token tiles than half the SMs (T <= 9472 on 148 SMs) each tile
+// runs on a cluster pair instead: CTA 0 takes the first half of the K blocks,
+// CTA 1 the second, and after an exchange of partial logits through distributed
+// shared memory each CTA routes 64 of the tokens.  The kernel is bound by the
+// latency of its K-block chain, so halving the chain halves its time; the two
+// halves are added once, low + high, the same FP32 sum in both CTAs.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -200,6 +206,11 @@ __global__ void split_wg_kernel(const float* __restrict__ wg, int E, int e_pad, 
   }
 }
 
+// SPLIT: two CTAs of a cluster share one 128-token tile, CTA 0 taking the first
+// half of the K blocks and CTA 1 the second; each then adds the two partial
+// logits (low half + high half, the same FP32 sum in both) for 64 of the tokens
+// and routes them.  Used when one CTA per tile would leave most SMs idle.
+template <bool SPLIT>
 __global__ void __launch_bounds__(GT_THREADS, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const GateArgs a) {
@@ -208,8 +219,11 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
                                              ~uintptr_t(1023));
   GateCtl* ctl = reinterpret_cast<GateCtl*>(smem + (size_t)a.stages * a.stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * GT_BM;
-  const int nkb = a.d / GT_BK;
+  const uint32_t crank = SPLIT ? cluster_ctarank() : 0u;
+  const int64_t m0 = (int64_t)(SPLIT ? (blockIdx.x >> 1) : blockIdx.x) * GT_BM;
+  const int nkb_all = a.d / GT_BK;
+  const int kb0 = (SPLIT && crank) ? nkb_all / 2 : 0;  // this CTA's K blocks [kb0, kb0 + nkb)
+  const int nkb = SPLIT ? (crank ? nkb_all - nkb_all / 2 : nkb_all / 2) : nkb_all;
   const uint32_t plane_bytes = (uint32_t)a.e_pad * GT_BK * 2;
   volatile int* abort_flag = &ctl->abort_flag;
 
@@ -259,7 +273,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           break;
         mbar_arrive_expect_tx(&ctl->full[stage], GT_A_BYTES + 3 * plane_bytes);
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
-        const int k0 = kb * GT_BK;
+        const int k0 = (kb0 + kb) * GT_BK;
         tma_load_2d(st, &tmX, &ctl->full[stage], k0, (int32_t)m0);  // rows past T read as zero
 #pragma unroll
         for (int j = 0; j < 3; ++j)
@@ -372,8 +386,24 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     }
   }
   __syncthreads();
+  int r0 = 0, rows = GT_BM;
+  if constexpr (SPLIT) {
+    cluster_sync();  // both CTAs' partial logits are in shared memory
+    r0 = (int)crank * (GT_BM / 2);
+    rows = GT_BM / 2;
+    if (!aborted) {
+      const uint32_t peer = map_to_rank(L, crank ^ 1u);
+      for (int i = threadIdx.x; i < rows * a.E; i += blockDim.x) {
+        const int off = (r0 + i / a.E) * LS + i % a.E;
+        L[off] = L[off] + ld_shared_cluster_f32(peer + (uint32_t)off * 4u);
+      }
+    }
+    __syncthreads();
+  }
   if (!aborted)
-    route_tile(L, LS, m0, GT_BM, a.T, a.E, a.k, a.bias, a.topk_idx, a.topk_w, a.probs);
+    route_tile(L + r0 * LS, LS, m0 + r0, rows, a.T, a.E, a.k, a.bias, a.topk_idx, a.topk_w,
+               a.probs);
+  if constexpr (SPLIT) cluster_sync();  // the peer has read this CTA's partials
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, a.tmem_cols);
@@ -440,14 +470,37 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
     return MOE_ERR_CUDA;
   const size_t smem = fixed + (size_t)stages * a.stage_bytes;
   static bool attr_set = false;
+  static int num_sms = 0;
   if (!attr_set) {
-    if (!cuda_ok(cudaFuncSetAttribute(gate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      GT_MAX_SMEM)))
+    if (!cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GT_MAX_SMEM)) ||
+        !cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GT_MAX_SMEM)))
       return MOE_ERR_CUDA;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     attr_set = true;
   }
-  const int64_t blocks = (T + GT_BM - 1) / GT_BM;
-  gate_tc_kernel<<<(unsigned)blocks, GT_THREADS, smem, st>>>(mx, mw, a);
+  const int64_t tiles = (T + GT_BM - 1) / GT_BM;
+  if (2 * tiles <= num_sms && a.d / GT_BK >= 2) {
+    // fewer tiles than half the SMs: a CTA pair per tile, each on half of K
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * tiles));
+    cfg.blockDim = dim3(GT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, gate_tc_kernel<true>, mx, mw, a))) return MOE_ERR_CUDA;
+  } else {
+    gate_tc_kernel<false><<<(unsigned)tiles, GT_THREADS, smem, st>>>(mx, mw, a);
+  }
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 

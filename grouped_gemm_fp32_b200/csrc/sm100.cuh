@@ -98,6 +98,13 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
   }
 }
 
+// 32-bit load from another CTA's shared memory (address from map_to_rank).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 // Arrive on an mbarrier of another CTA of the cluster (address from map_to_rank).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
