@@ -134,6 +134,8 @@ class EPBuffers:
 
     def __init__(self, dims: L.MoeDims, rank: int, world: int, train: bool = False,
                  device="cuda", recv_rows_cap: int | None = None):
+        """``rank`` / ``world``: this process's rank in, and the size of, the process
+        group that the distributed driver is given."""
         if dims.E % world:
             raise ValueError(f"E = {dims.E} experts do not split over {world} ranks")
         El = dims.E // world
@@ -172,10 +174,16 @@ def route(eb: EPBuffers, x, wg, bias, stream=None, seq_balance=None):
             F.bal_seq_len = int(seq_len)
 
 
-def set_plan(eb: EPBuffers, counts_own, counts_in):
-    """Phase 2: this step's exchange tables from the host copies of the counts, and the
-    local groups' table."""
-    plan = EPPlan(counts_own, counts_in, eb.rank, eb.world, eb.dims.P)
+def make_plan(eb: EPBuffers, counts_own, counts_in) -> EPPlan:
+    """This step's exchange tables from the host copies of the counts."""
+    return EPPlan(counts_own, counts_in, eb.rank, eb.world, eb.dims.P)
+
+
+def set_plan(eb: EPBuffers, counts_own, counts_in, plan: EPPlan | None = None):
+    """Phase 2: this step's exchange tables (``plan``, or made from the counts) and the
+    local groups' table.  Raises when this rank would receive more rows than its buffers
+    hold (the distributed driver first agrees on that across the ranks)."""
+    plan = plan or make_plan(eb, counts_own, counts_in)
     if plan.recv_rows > eb.loc.Rr:
         raise RuntimeError(f"rank {eb.rank} receives {plan.recv_rows} rows, more than its "
                            f"{eb.loc.Rr}-row buffers (recv_rows_cap)")
@@ -236,6 +244,18 @@ def unpermute_and_router(eb: EPBuffers, x, wg=None, stream=None):
 
 # ------------------------------------------------------ distributed driver --
 
+def check_capacity(recv_rows: int, cap: int, group=None, device=None):
+    """Raise on every rank of ``group`` when any rank would receive more than ``cap``
+    rows: the ranks agree (an all-reduce of the largest overflow) before any rows move,
+    so that none is left waiting in the exchange for a rank that gave up."""
+    import torch.distributed as dist
+    over = torch.tensor([recv_rows - cap], dtype=torch.int64, device=device)
+    dist.all_reduce(over, op=dist.ReduceOp.MAX, group=group)
+    if int(over.item()) > 0:
+        raise RuntimeError(f"a rank would receive {int(over.item())} rows more than its "
+                           f"{cap}-row buffers (recv_rows_cap)")
+
+
 def _stream_ctx(stream):
     return torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else layer._Null()
 
@@ -250,7 +270,9 @@ def forward(eb: EPBuffers, x, wg, bias, w1_loc, w2_loc, group=None, stream=None,
         route(eb, x, wg, bias, stream, seq_balance)
         counts_in = torch.empty_like(F.counts)
         dist.all_to_all_single(counts_in, F.counts, group=group)
-        set_plan(eb, F.counts.cpu().numpy(), counts_in.cpu().numpy())
+        plan = make_plan(eb, F.counts.cpu().numpy(), counts_in.cpu().numpy())
+        check_capacity(plan.recv_rows, eb.loc.Rr, group, F.counts.device)
+        set_plan(eb, None, None, plan)
         exchange(*dispatch_lists(eb.plan, F.x_perm, eb.loc.x_perm), eb.rank, group)
         experts_forward(eb, x, w1_loc, w2_loc, stream)
         exchange(*return_lists(eb.plan, eb.loc.y, F.y), eb.rank, group)

@@ -208,3 +208,36 @@ def test_expert_parallel_exchange_moves_segments_both_ways(world):
         assert ok_dispatch, rank
         assert ok_return, rank
         assert recv_rows == local_rows
+
+
+def _cap_worker(rank, world, port, q):
+    """ep.check_capacity on gloo: one rank over its receive capacity makes every rank raise."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from grouped_gemm_fp32_b200 import ep
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ep.check_capacity(40 + rank, 100)          # everyone within capacity: no error
+    raised = False
+    try:
+        ep.check_capacity(120 if rank == 1 else 10, 100)
+    except RuntimeError:
+        raised = True
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, raised))
+
+
+def test_expert_parallel_capacity_overflow_raises_on_every_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cap_worker, args=(r, 3, port, q)) for r in range(3)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=240) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(raised for _, raised in out)
