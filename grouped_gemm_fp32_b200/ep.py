@@ -256,17 +256,13 @@ def check_capacity(recv_rows: int, cap: int, group=None, device=None):
                            f"{cap}-row buffers (recv_rows_cap)")
 
 
-def _stream_ctx(stream):
-    return torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else layer._Null()
-
-
 def forward(eb: EPBuffers, x, wg, bias, w1_loc, w2_loc, group=None, stream=None,
             seq_balance=None):
     """The layer's forward under expert parallelism over ``group`` (every rank calls it).
     Returns this rank's out [T, d].  The counts come to the host once per step."""
     import torch.distributed as dist
     F = eb.full
-    with _stream_ctx(stream):
+    with layer.on_stream(stream):
         route(eb, x, wg, bias, stream, seq_balance)
         counts_in = torch.empty_like(F.counts)
         dist.all_to_all_single(counts_in, F.counts, group=group)
@@ -288,7 +284,7 @@ def backward(eb: EPBuffers, x, dout, w1_loc, w2_loc, group=None, stream=None, wg
     if not eb.train:
         raise ValueError("buffers were allocated without train=True")
     F = eb.full
-    with _stream_ctx(stream):
+    with layer.on_stream(stream):
         combine_backward(eb, dout, stream)
         exchange(*dispatch_lists(eb.plan, F.dy, eb.loc.dy), eb.rank, group)
         experts_backward(eb, x, dout, w1_loc, w2_loc, stream)

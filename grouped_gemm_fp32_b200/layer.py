@@ -22,6 +22,8 @@ ranks share, over torch.distributed.
 """
 from __future__ import annotations
 
+from contextlib import nullcontext
+
 import torch
 
 from . import _lib as L
@@ -160,16 +162,9 @@ def backward(b: MoEBuffers, x, dout, w1, w2, stream=None, wg=None, gamma=None, b
 # own.  Both are all-reduces over torch.distributed (NCCL between GPUs), issued
 # on the layer's stream.
 
-def _on_stream(stream):
-    return torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else _Null()
-
-
-class _Null:
-    def __enter__(self):
-        return None
-
-    def __exit__(self, *a):
-        return False
+def on_stream(stream):
+    """``torch.cuda.stream(stream)`` for a torch stream, else no change of stream."""
+    return torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else nullcontext()
 
 
 def dp_load_counts(counts, group=None, stream=None):
@@ -178,7 +173,7 @@ def dp_load_counts(counts, group=None, stream=None):
     of ``group``.  Returns a new tensor; ``counts`` itself is left as it is (the
     backward GEMMs still read it)."""
     import torch.distributed as dist
-    with _on_stream(stream):
+    with on_stream(stream):
         total = counts.clone()
         dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
     return total
@@ -207,7 +202,7 @@ def dp_allreduce_grads(grads, group=None, stream=None):
     """Sum each gradient tensor (e.g. ``b.dw1``, ``b.dw2``, ``b.dwg``) over the ranks
     of ``group``, in place: the gradients of the whole data-parallel batch."""
     import torch.distributed as dist
-    with _on_stream(stream):
+    with on_stream(stream):
         for g in grads:
             dist.all_reduce(g, op=dist.ReduceOp.SUM, group=group)
     return grads
