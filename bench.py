@@ -64,6 +64,9 @@ def parse():
                              "tiny"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layer", action="store_true",
+                    help="skip the T = 8192 layer-forward measurement that the train run adds "
+                         "(key north_star_c3)")
     ap.add_argument("--eager", action="store_true",
                     help="time the step as eager C-ABI calls instead of a replayed CUDA graph")
     ap.add_argument("--gather", action="store_true",
@@ -318,71 +321,77 @@ def describe(wl):
 
 
 # ---------------------------------------------------------------- GPU (ours) --
-def run_ours(args):
-    import torch
+class Case:
+    """One workload on this GPU: its inputs in HBM, the layer's buffers and the
+    step as C-ABI calls, with an optional event between consecutive calls."""
 
-    world, rank, local = dist_setup(args)
-    import grouped_gemm_fp32_b200 as moe
-    from grouped_gemm_fp32_b200 import layer
+    def __init__(self, name, args, dev, rank=0):
+        import torch
+        import grouped_gemm_fp32_b200 as moe
+        from grouped_gemm_fp32_b200 import layer
 
-    wl, inp = workload(args.workload)
-    inp = rank_shard(wl, inp, rank)  # data parallel: each rank its own tokens
-    dm = wl.dims
-    dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
-    train = wl.backward
-    gemm_only = wl.group_rows is not None
-    gate_only = args.workload == "gate_only"
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.Stream(device=dev)
-    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
-    x = bf(inp["x"])
-    w1 = bf(inp["w1"]) if not gate_only else None
-    w2 = bf(inp["w2"]) if not gate_only else None
-    wg = torch.from_numpy(inp["wg"]).to(dev) if not gemm_only else None
-    bias = torch.from_numpy(inp["bias"]).to(dev) if not gemm_only else None
-    dout = bf(inp["dout"]) if train else None
-    if gate_only:
-        class _GateBufs:  # the gate's outputs only
-            topk_idx = torch.empty(dm.T, dm.k, dtype=torch.int32, device=dev)
-            topk_w = torch.empty(dm.T, dm.k, dtype=torch.float32, device=dev)
-            ws = torch.zeros(moe.moe_workspace_size(dims), dtype=torch.uint8, device=dev)
-            out = torch.empty(dm.T, dm.d, dtype=torch.bfloat16, device=dev)
-        b = _GateBufs()
-    else:
-        b = layer.MoEBuffers(dims, device=dev, train=train, gather=args.gather)
-    if gemm_only:
-        counts = torch.tensor(wl.group_rows, dtype=torch.int32, device=dev)
-        moe.grouped_gemm_set_groups(dims, counts, b.offsets, b.ws)
-    torch.cuda.synchronize()
+        wl, inp = workload(name)
+        inp = rank_shard(wl, inp, rank)  # data parallel: each rank its own tokens
+        dm = wl.dims
+        self.name, self.wl, self.inp, self.dm = name, wl, inp, dm
+        self.dims = dims = moe.MoeDims.of(dm.T, dm.d, dm.E, dm.k, dm.S, dm.I, dm.P, dm.rows_cap)
+        self.train = wl.backward
+        self.gemm_only = wl.group_rows is not None
+        self.gate_only = name == "gate_only"
+        self.gather = args.gather
+        bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
+        self.x = bf(inp["x"])
+        self.w1 = bf(inp["w1"]) if not self.gate_only else None
+        self.w2 = bf(inp["w2"]) if not self.gate_only else None
+        self.wg = torch.from_numpy(inp["wg"]).to(dev) if not self.gemm_only else None
+        self.bias = torch.from_numpy(inp["bias"]).to(dev) if not self.gemm_only else None
+        self.dout = bf(inp["dout"]) if self.train else None
+        if self.gate_only:
+            class _GateBufs:  # the gate's outputs only
+                topk_idx = torch.empty(dm.T, dm.k, dtype=torch.int32, device=dev)
+                topk_w = torch.empty(dm.T, dm.k, dtype=torch.float32, device=dev)
+                ws = torch.zeros(moe.moe_workspace_size(dims), dtype=torch.uint8, device=dev)
+                out = torch.empty(dm.T, dm.d, dtype=torch.bfloat16, device=dev)
+            self.b = _GateBufs()
+        else:
+            self.b = layer.MoEBuffers(dims, device=dev, train=self.train, gather=self.gather)
+        if self.gemm_only:
+            counts = torch.tensor(wl.group_rows, dtype=torch.int32, device=dev)
+            moe.grouped_gemm_set_groups(dims, counts, self.b.offsets, self.b.ws)
+        # the calls of one step, in order; an event before the first and after each
+        self.names = (["t0", "gate"] if self.gate_only else
+                      ["t0", "fwd"] if self.gemm_only else
+                      ["t0", "gate", "permute", "fwd", "combine"]) + (
+            ["seq_balance", "combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute", "router_bwd",
+             "bias_step"] if self.train else [])
+        torch.cuda.synchronize()
 
-    def step(s, xx=x, gg=dout, ev=None):
-        if gate_only:
-            if ev is not None:
-                ev["t0"].append(torch.cuda.Event(enable_timing=True))
-                ev["t0"][-1].record(s)
-            moe.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, b.ws, s)
-            if ev is not None:
-                ev["gate"].append(torch.cuda.Event(enable_timing=True))
-                ev["gate"][-1].record(s)
+    def step(self, s, xx=None, gg=None, ev=None):
+        """One step on stream ``s``; with ``ev`` (name -> event) an event is recorded
+        before the first call and after each call, under the names of ``self.names``."""
+        import grouped_gemm_fp32_b200 as L
+        from grouped_gemm_fp32_b200 import layer
+        xx = self.x if xx is None else xx
+        gg = self.dout if gg is None else gg
+        b, dims, train = self.b, self.dims, self.train
+        wg, bias, w1, w2 = self.wg, self.bias, self.w1, self.w2
+        rec = (lambda k: ev[k].record(s)) if ev is not None else (lambda k: None)
+        if self.gate_only:
+            rec("t0")
+            L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, None, b.ws, s)
+            rec("gate")
             return
-        if gemm_only:
-            if ev is not None:
-                ev["t0"].append(torch.cuda.Event(enable_timing=True))
-                ev["t0"][-1].record(s)
-            moe.grouped_gemm_fwd(dims, b.ws, xx, None, w1, w2, b.h, None, b.y, s)
-            if ev is not None:
-                ev["fwd"].append(torch.cuda.Event(enable_timing=True))
-                ev["fwd"][-1].record(s)
+        if self.gemm_only:
+            rec("t0")
+            L.grouped_gemm_fwd(dims, b.ws, xx, None, w1, w2, b.h, None, b.y, s)
+            rec("fwd")
             return
-        if ev is None:
+        if ev is None:  # the layer's own driver: the calls below, without events
             layer.forward(b, xx, wg, bias, w1, w2, stream=s,
                           seq_balance=SEQ_BALANCE if train else None)
             if train:
                 layer.backward(b, xx, gg, w1, w2, stream=s, wg=wg, gamma=GAMMA, bias=bias)
             return
-        # instrumented: events around each C-ABI call
-        L = moe
-        rec = lambda k: ev[k].append(torch.cuda.Event(enable_timing=True)) or ev[k][-1].record(s)
         rec("t0")
         L.moe_gate_topk(dims, xx, wg, bias, b.topk_idx, b.topk_w, b.probs if train else None,
                         b.ws, s)
@@ -397,59 +406,59 @@ def run_ours(args):
         rec("fwd")
         L.moe_combine(dims, b.y, b.row_of, b.topk_w, b.out, s)
         rec("combine")
-        if train:
-            L.moe_seq_balance_loss(dims, SEQ_BALANCE[1], SEQ_BALANCE[0], b.topk_idx, b.probs,
-                                   b.bal_loss, b.bal_grad, b.ws, s)
-            rec("seq_balance")
-        if train:
-            L.moe_combine_bwd(dims, b.ws, gg, b.y, b.row_of, b.topk_w, b.dy, b.dw_comb, s)
-            rec("combine_bwd")
-            L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM2, b.dy, gg, w2, b.a1, b.da, s)
-            rec("dx2")
-            L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM2, b.dy, gg, b.h, None, b.dw2, 0, s)
-            rec("dw2")
-            L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, s)
-            rec("dx1")
-            if b.gather:
-                L.grouped_gemm_bwd_dw1_gather(dims, b.ws, b.sorted_ids, b.da, xx, b.dw1, 0, s)
-            else:
-                L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, xx, b.dw1,
-                                      0, s)
-            rec("dw1")
-            L.moe_combine(dims, b.dxp, b.row_of, None, b.dx, s)
-            rec("unpermute")
-            L.moe_router_bwd_seqbal(dims, xx, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb,
-                                    b.bal_grad, SEQ_BALANCE[1], None, b.dx, b.dwg, 0, b.ws, s)
-            rec("router_bwd")
-            L.moe_bias_update(dims, b.counts, GAMMA, bias, b.bias_next, s)
-            rec("bias_step")
+        if not train:
+            return
+        L.moe_seq_balance_loss(dims, SEQ_BALANCE[1], SEQ_BALANCE[0], b.topk_idx, b.probs,
+                               b.bal_loss, b.bal_grad, b.ws, s)
+        rec("seq_balance")
+        L.moe_combine_bwd(dims, b.ws, gg, b.y, b.row_of, b.topk_w, b.dy, b.dw_comb, s)
+        rec("combine_bwd")
+        L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM2, b.dy, gg, w2, b.a1, b.da, s)
+        rec("dx2")
+        L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM2, b.dy, gg, b.h, None, b.dw2, 0, s)
+        rec("dw2")
+        L.grouped_gemm_bwd_dx(dims, b.ws, L.MOE_GEMM1, b.da, None, w1, None, b.dxp, s)
+        rec("dx1")
+        if b.gather:
+            L.grouped_gemm_bwd_dw1_gather(dims, b.ws, b.sorted_ids, b.da, xx, b.dw1, 0, s)
+        else:
+            L.grouped_gemm_bwd_dw(dims, b.ws, L.MOE_GEMM1, b.da, None, b.x_perm, xx, b.dw1, 0, s)
+        rec("dw1")
+        L.moe_combine(dims, b.dxp, b.row_of, None, b.dx, s)
+        rec("unpermute")
+        L.moe_router_bwd_seqbal(dims, xx, wg, b.probs, b.topk_idx, b.topk_w, b.dw_comb,
+                                b.bal_grad, SEQ_BALANCE[1], None, b.dx, b.dwg, 0, b.ws, s)
+        rec("router_bwd")
+        L.moe_bias_update(dims, b.counts, GAMMA, bias, b.bias_next, s)
+        rec("bias_step")
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step(stream)
-    stream.synchronize()
-    status = moe.moe_get_device_status(b.ws, stream)
-    if status != 0:
-        raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(status)}")
+    def check_status(self, stream, when):
+        import grouped_gemm_fp32_b200 as moe
+        status = moe.moe_get_device_status(self.b.ws, stream)
+        if status != 0:
+            raise RuntimeError(f"device status {when}: {moe.moe_status_string(status)}")
 
-    # The layer step as a CUDA graph of the same C-ABI calls (captured after the
-    # warm-up, replayed in the timed loop); the eager step is timed beside it.
-    use_graph = not args.eager and not (gate_only or gemm_only)
-    graph = None
+
+def timed_region(case, stream, steps, use_graph, world, dev, local):
+    """The headline timing: ``steps`` steps between a barrier + synchronize and a
+    synchronize + barrier, CUDA events on the launching stream, max over ranks, SM
+    clocks sampled meanwhile.  With ``use_graph`` every step is a replayed CUDA graph
+    of the step's C-ABI calls (one graph per timed step, captured beforehand).  Each
+    step also records an event before its first call and after each call (event
+    nodes inside the graphs), so the per-call breakdown comes from the timed steps
+    themselves.  Returns (ms per step, per-call ms, clocks, gap between steps in ms)."""
+    import torch
+    names = case.names
+    evs = [{n: torch.cuda.Event(enable_timing=True, external=use_graph) for n in names}
+           for _ in range(steps)]
+    graphs = []
     if use_graph:
-        graph = layer.GraphStep(b, x, wg, bias, w1, w2, dout=dout if train else None,
-                                gamma=GAMMA if train else None,
-                                seq_balance=SEQ_BALANCE if train else None)
-
-    def timed_steps(n):
-        with torch.cuda.stream(stream):
-            for _ in range(n):
-                if graph is not None:
-                    graph.replay()
-                else:
-                    step(stream)
-
-    # ---- timed region: device-resident inputs
+        for i in range(steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                case.step(stream, ev=evs[i])
+            graphs.append(g)
+        torch.cuda.synchronize(dev)
     clk = ClockSampler(local)
     clk.start()
     time.sleep(0.25)
@@ -458,52 +467,117 @@ def run_ours(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-    timed_steps(args.steps)
-    with torch.cuda.stream(stream):
+        for i in range(steps):
+            if use_graph:
+                graphs[i].replay()
+            else:
+                case.step(stream, ev=evs[i])
         e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize(dev)
     barrier(world)
     clocks = clk.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms = dist_max(ms, world, dev)
+    ms = dist_max(e0.elapsed_time(e1) / steps, world, dev)
+    per = {}
+    for i in range(1, len(names)):
+        per[names[i]] = sum(ev[names[i - 1]].elapsed_time(ev[names[i]]) for ev in evs) / steps
+    inside = sum(ev[names[0]].elapsed_time(ev[names[-1]]) for ev in evs) / steps
+    del graphs
+    return ms, per, clocks, ms - inside
+
+
+def gemm_roofline(case, per, pk, pk_src):
+    """The grouped GEMM's algorithmic TFLOP/s over its launches' event times."""
+    flops = gemm_flops(case.dm, case.train)
+    gemm_ms = sum(per[k] for k in flops)
+    achieved = sum(flops.values()) / (gemm_ms / 1000.0) / 1e12
+    burst = pk["bf16_tflops"]
+    sustained = pk.get("bf16_tflops_sustained", burst)
+    detail = {k: {"ms": round(per[k], 4), "tflops": round(flops[k] / per[k] / 1e9, 1)}
+              for k in flops}
+    return gemm_ms, achieved, burst, sustained, detail
+
+
+def north_star_layer(args, dev, local, pk, pk_src):
+    """The layer forward at T = 8192 (d = 4096, 128 routed experts top-6 + 2 shared,
+    I = 1408, pad block 128, near-uniform loads), the configuration on which the
+    grouped GEMM's share of the dense bf16 peak is judged: its own inputs, warm-up,
+    timed graph replays, clocks and per-call event times."""
+    import torch
+    case = Case("layer", args, dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            case.step(stream)
+    stream.synchronize()
+    case.check_status(stream, "after the layer warm-up")
+    steps = max(20, args.steps)
+    ms, per, clocks, gap = timed_region(case, stream, steps, True, 1, dev, local)
+    case.check_status(stream, "after the layer timing")
+    gemm_ms, achieved, burst, sustained, _ = gemm_roofline(case, per, pk, pk_src)
+    out = {"workload": describe(case.wl), "steps": steps, "ms_per_step": round(ms, 4),
+           "tokens_per_s": case.dm.T / (ms / 1000.0),
+           "grouped_gemm_ms": round(gemm_ms, 4), "grouped_gemm_tflops": round(achieved, 1),
+           "frac_of_burst_peak": round(achieved / burst, 4),
+           "frac_of_sustained_peak": round(achieved / sustained, 4),
+           "peak_burst": burst, "peak_sustained": sustained, "peak_source": pk_src,
+           "target_frac_of_burst": 0.60,
+           "breakdown_ms": {k: round(v, 4) for k, v in per.items()},
+           "breakdown_sum_over_step": round(sum(per.values()) / ms, 4),
+           "clocks": clocks}
+    del case
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_setup(args)
+    import grouped_gemm_fp32_b200 as moe
+    from grouped_gemm_fp32_b200 import layer
+
+    dev = torch.device("cuda", local)
+    case = Case(args.workload, args, dev, rank)
+    wl, inp, dm, dims, b = case.wl, case.inp, case.dm, case.dims, case.b
+    train, gemm_only, gate_only = case.train, case.gemm_only, case.gate_only
+    x, w1, w2, wg, bias, dout = case.x, case.w1, case.w2, case.wg, case.bias, case.dout
+    stream = torch.cuda.Stream(device=dev)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            case.step(stream)
+    stream.synchronize()
+    case.check_status(stream, "after warm-up")
+
+    # ---- timed region: device-resident inputs; the step as replayed CUDA graphs of
+    # the same C-ABI calls, per-call events inside them
+    use_graph = not args.eager and not (gate_only or gemm_only)
+    ms, per, clocks, gap = timed_region(case, stream, args.steps, use_graph, world, dev, local)
     ms_eager = None
-    if graph is not None:  # the same steps as eager calls, for comparison
+    if use_graph:  # the same steps as eager calls of the layer driver, for comparison
         barrier(world)
         torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(args.steps):
-                step(stream)
+                case.step(stream)
             e1.record(stream)
         e1.synchronize()
         ms_eager = dist_max(e0.elapsed_time(e1) / args.steps, world, dev)
     tokens_per_s = world * dm.T / (ms / 1000.0)
 
-    # ---- per-call breakdown (separate instrumented pass; not the headline)
-    names = (["t0", "gate"] if gate_only else
-             ["t0", "fwd"] if gemm_only else ["t0", "gate", "permute", "fwd", "combine"]) + (
-        ["seq_balance", "combine_bwd", "dx2", "dw2", "dx1", "dw1", "unpermute", "router_bwd",
-         "bias_step"]
-        if train else [])
-    ev = {n: [] for n in names}
-    nprof = max(3, min(args.steps, 20))
-    with torch.cuda.stream(stream):
-        for _ in range(nprof):
-            step(stream, ev=ev)
-    stream.synchronize()
-    per = {}
-    for i in range(1, len(names)):
-        a, c = ev[names[i - 1]], ev[names[i]]
-        per[names[i]] = sum(x0.elapsed_time(x1) for x0, x1 in zip(a, c)) / nprof
-    flops = gemm_flops(dm, train) if not gate_only else {"gate": 2 * dm.T * dm.d * dm.E}
-    gemm_ms = sum(per[k] for k in flops)
-    gemm_tflops = sum(flops.values()) / (gemm_ms / 1000.0) / 1e12
     pk, pk_src = peaks()
     traffic, traffic_note = gemm_traffic(args.workload)
-    sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    gemm_detail = {k: {"ms": round(per[k], 4), "tflops": round(flops[k] / per[k] / 1e9, 1)}
-                   for k in flops}
+    if gate_only:  # the gate's FP32-equivalent FLOPs, run as bf16 MMAs of exact splits
+        gemm_ms = per["gate"]
+        achieved = 2 * dm.T * dm.d * dm.E / (gemm_ms / 1000.0) / 1e12
+        burst = pk["bf16_tflops"]
+        sustained = pk.get("bf16_tflops_sustained", burst)
+        gemm_detail = {"gate": {"ms": round(gemm_ms, 4), "tflops": round(achieved, 1)}}
+    else:
+        gemm_ms, achieved, burst, sustained, gemm_detail = gemm_roofline(case, per, pk, pk_src)
 
     # ---- e2e: pinned host inputs in, results out, every step, through the same
     # C-ABI calls; neighbouring steps' copies overlap compute (layer.HostPipeline)
@@ -520,7 +594,7 @@ def run_ours(args):
             with torch.cuda.stream(stream):
                 for _ in range(nsteps):
                     dx_in.copy_(hx, non_blocking=True)
-                    step(stream, xx=dx_in)
+                    case.step(stream, xx=dx_in)
                     ho.copy_(out_dev, non_blocking=True)
         e2e_streams = [stream]
         e2e_note = "inputs H2D and results D2H every step, serialised with compute"
@@ -559,9 +633,7 @@ def run_ours(args):
     f1.record(e2e_streams[-1])
     f1.synchronize()
     e2e_ms = dist_max(f0.elapsed_time(f1) / ne2e, world, dev)
-    status = moe.moe_get_device_status(b.ws, stream)
-    if status != 0:
-        raise RuntimeError(f"device status after timing: {moe.moe_status_string(status)}")
+    case.check_status(stream, "after timing")
 
     # kernels per step: gate 2 (weight split, gate), permute 3 (histogram, groups,
     # scatter; + row copy and pad zeroing without gathering), forward GEMMs 2, combine 1;
@@ -579,7 +651,9 @@ def run_ours(args):
         "config": {"workload": describe(wl), "tokens_per_gpu": dm.T,
                    "global_batch_tokens": world * dm.T,
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "step": "CUDA graph replay" if graph is not None else "eager C-ABI calls",
+                   "step": ("CUDA graph replay (one captured graph per timed step, event "
+                            "nodes between its C-ABI calls)" if use_graph
+                            else "eager C-ABI calls"),
                    "x_rows": ("gathered from x by sorted_ids (tile::gather4)" if args.gather
                               else "permuted copy x_perm"),
                    "seq_balance": ({"alpha": SEQ_BALANCE[0], "seq_len": SEQ_BALANCE[1]}
@@ -587,20 +661,29 @@ def run_ours(args):
                    "ms_per_step_eager": ms_eager,
                    "l2": "no flush: weights (4.5 GB) and activations exceed the 126 MB L2"},
         "roofline": {"bound": "tensor", "kernel": "ggemm_kernel (all grouped-GEMM launches)",
-                     "achieved": gemm_tflops, "peak": sustained, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / sustained,
-                     "peak_kind": f"{pk_src} bf16 sustained (kernel timed inside a long step)",
-                     "frac_of_burst_peak": gemm_tflops / pk["bf16_tflops"],
+                     "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                     "frac": achieved / burst if burst else None,
+                     "peak_kind": f"{pk_src} bf16 burst (ms-scale launches; the clocks of the "
+                                  f"timed steps are in 'clocks')",
+                     "frac_of_sustained_peak": achieved / sustained if sustained else None,
+                     "peak_sustained": sustained,
+                     "timing": "event pairs around each grouped-GEMM call inside the timed steps",
                      "traffic": traffic, "traffic_unit": "bytes per step",
                      "traffic_note": traffic_note},
         "grouped_gemm": gemm_detail,
         "breakdown_ms": {k: round(v, 4) for k, v in per.items()},
+        "breakdown_sum_over_step": round(sum(per.values()) / ms, 4),
+        "gap_between_steps_ms": round(gap, 4),
         "e2e": {"value": world * dm.T / (e2e_ms / 1000.0), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "note": e2e_note},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if args.workload == "train" and world == 1 and not args.no_layer:
+        del pipe
+        torch.cuda.empty_cache()
+        line["north_star_c3"] = north_star_layer(args, dev, local, pk, pk_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not (gemm_only or gate_only):
         line["cpu_baseline"] = cpu_baseline(wl, inp)
     if rank == 0:

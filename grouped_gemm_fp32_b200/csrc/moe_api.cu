@@ -21,7 +21,7 @@ bool cuda_ok(cudaError_t e) {
 
 }  // namespace moe
 
-namespace {
+namespace moe {
 
 bool dims_ok(const moe_dims* dm) {
   if (!dm) return false;
@@ -44,6 +44,10 @@ int check_shape(const moe_dims* dm, bool need_bwd) {
   if (rows_routed(*dm) < 0) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
+
+}  // namespace moe
+
+namespace {
 
 bool ws_ok(const moe_dims* dm, const void* ws, size_t bytes) {
   return ws != nullptr && bytes >= ws_layout(*dm).bytes;

@@ -14,6 +14,13 @@ namespace moe {
 // Records the error of a failing CUDA call for moe_last_cuda_error(); true on success.
 bool cuda_ok(cudaError_t e);
 
+// Argument and shape checks every entry point runs first (moe_api.cu): dims_ok
+// is false for a null or non-positive shape; check_shape returns
+// MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE / MOE_OK for the shapes the
+// kernels support (include/moe.h), need_bwd adding the backward's P % 64 == 0.
+bool dims_ok(const moe_dims* dm);
+int check_shape(const moe_dims* dm, bool need_bwd);
+
 // One group of the grouped GEMM: a routed expert (g < E) or a shared expert.
 //   a_row    first row of the group in its A source (x_perm for routed groups,
 //            x for shared groups, i.e. 0)

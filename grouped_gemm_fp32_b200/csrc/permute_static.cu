@@ -25,7 +25,10 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_permute_scratch[kStaticScratchBytes];
 
 // Device address of g_permute_scratch for each device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached for the life of the process.
+// The cache does not survive a cudaDeviceReset (or any teardown of the
+// device's primary context): after one, the cached address is stale, so a
+// process that resets a device must not call this entry point on it again.
 void* scratch_for_current_device(int* rc) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
@@ -56,13 +59,9 @@ extern "C" int moe_permute_align_static(const moe_dims* dims, const int32_t* top
                                         const void* x, int32_t* counts, int32_t* offsets,
                                         int32_t* sorted_ids, int32_t* row_of, void* x_perm,
                                         void* stream) {
-  if (!dims || dims->T < 0 || dims->d <= 0 || dims->E <= 0 || dims->k <= 0 || dims->S < 0 ||
-      dims->I <= 0 || dims->P <= 0)
-    return MOE_ERR_INVALID_ARG;
-  if (dims->d % 64 || dims->I % 64 || dims->E > 256 || dims->k > dims->E || dims->S > 8 ||
-      dims->P % 8 || dims->P < 8 || rows_total(*dims) >= (int64_t(1) << 31) ||
-      dims->T * dims->k >= (int64_t(1) << 31))
-    return MOE_ERR_UNSUPPORTED_SHAPE;
+  // the same argument and shape checks as every other entry point
+  const int shape_rc = check_shape(dims, false);
+  if (shape_rc != MOE_OK) return shape_rc;
   // the scratch this call needs must fit the fixed array
   if (ws_layout(*dims).bytes > kStaticScratchBytes) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!counts || !offsets || !sorted_ids) return MOE_ERR_INVALID_ARG;

@@ -77,11 +77,13 @@ typedef struct moe_dims {
 enum { MOE_GEMM1 = 1, /* gate|up projection  A1 = A W1^T  (N = 2I, K = d) */
        MOE_GEMM2 = 2  /* down projection     Y  = H W2^T  (N = d,  K = I) */ };
 
-/* Rr and Rt as defined above (-1 for invalid dims). */
+/* Rr and Rt as defined above (-1 for invalid dims).  Host-side sizes: the pages
+ * have no counterpart. */
 int64_t moe_rows_routed(const moe_dims* dims);
 int64_t moe_rows_total(const moe_dims* dims);
 
-/* Bytes of device workspace that the calls taking `ws` need.  One workspace
+/* Bytes of device workspace that the calls taking `ws` need (host-side, no
+ * counterpart on the pages).  One workspace
  * serves a whole layer.  It starts with the routing tables (the status word,
  * the group table, tile prefixes, per-chunk histograms): moe_permute_align (or
  * grouped_gemm_set_groups) writes them, the GEMM and combine-backward calls
@@ -153,17 +155,24 @@ int moe_permute_align(const moe_dims* dims, const int32_t* topk_idx, const void*
  * a host framework whose allocator owns every device buffer, foreign-function
  * callers that pass only inputs and outputs, paths where cudaMalloc is not
  * allowed.  It calls no cudaMalloc or cudaFree.
- *   - Limit: the call's scratch, the routing-table part of the workspace
- *     (moe_workspace_size(dims) without the gate's weight planes), must be at
- *     most 1 MiB (about 2 million routed assignments at E = 128); larger
- *     shapes return MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - Limit: the call's scratch is the routing-table part of the workspace
+ *     only (not the gate planes or router-backward scratch that
+ *     moe_workspace_size also counts): a 64-byte header, 16 G bytes of group
+ *     table, 4 (G + 1) of tile prefix, 4 G of group order and
+ *     4 E max(1, ceil(T k / 1024)) of chunk histograms, each part starting on
+ *     a 16-byte boundary and the sum rounded up to 256.  It must be at most
+ *     1 MiB (1,048,576 bytes; about 2 million routed assignments at E = 128,
+ *     1 million at E = 256); larger shapes return MOE_ERR_UNSUPPORTED_SHAPE
+ *     before anything is launched.
  *   - The array is shared by every call in the process and keeps the last
  *     call's contents; each call clears what must start at zero.  Calls whose
  *     executions overlap on the GPU (other streams, other threads) race on it
  *     and must be serialised by the caller.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any stream
- *     capture.
+ *     capture.  The address is kept for the life of the process: it does not
+ *     survive cudaDeviceReset, after which this call must not be used on that
+ *     device again.
  *   - Routing errors (expert id outside [0, E), padded rows above Rr) leave
  *     sorted_ids and row_of at -1 and x_perm unwritten; no device status is
  *     kept. */
@@ -172,7 +181,10 @@ int moe_permute_align_static(const moe_dims* dims, const int32_t* topk_idx, cons
                              int32_t* row_of, void* x_perm, void* stream);
 
 /* Group table from given per-expert row counts, for callers that already hold
- * the permuted rows (the grouped GEMM used on its own).  counts [E] int32
+ * the permuted rows (the grouped GEMM used on its own).
+ * Passage: dots.llm1 Technical Report, §3.2 "Efficient implementation of
+ * Grouped GEMM" (g groups with per-group row counts M_i, each aligned to a
+ * fixed block).  counts [E] int32
  * (device); writes offsets [E + 1] (device) and the group table in ws, with
  * segments padded to P as in moe_permute_align. */
 int grouped_gemm_set_groups(const moe_dims* dims, const int32_t* counts, int32_t* offsets,
@@ -212,6 +224,9 @@ int grouped_gemm_fwd_gather(const moe_dims* dims, const void* ws, const int32_t*
                             void* y, void* stream);
 
 /* Backward data-gradient grouped GEMMs.
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
+ * (the SwiGLU expert FFN whose input gradient this is) and §3.2 "Performance
+ * comparison" (the backward grouped GEMM, timed against Transformer Engine).
  *   which = MOE_GEMM2: dH = dY W2, then the SwiGLU backward with the saved a1:
  *       dG = dH * U * s * (1 + G (1 - s)), s = sigmoid(G);  dU = dH * silu(G)
  *     dy_routed [Rr, d] bf16 (from moe_combine_bwd), dy_shared [T, d] bf16 (the
@@ -226,6 +241,11 @@ int grouped_gemm_bwd_dx(const moe_dims* dims, const void* ws, int which, const v
 
 /* Backward weight-gradient grouped GEMMs; the reduction runs over each group's
  * (padded) rows.
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
+ * (the expert weights being trained) and §3.2 "Performance comparison" (the
+ * backward grouped GEMM); the aligned segments of §3.2 "Efficient
+ * implementation of Grouped GEMM" keep every 64-row reduction block inside one
+ * expert (hence P % 64 == 0).
  *   which = MOE_GEMM2: dW2_g = dY_g^T H_g
  *     lhs_routed = dY [Rr, d], lhs_shared = upstream gradient [T, d],
  *     rhs_routed = H [Rt, I], rhs_shared ignored  -> dw = dW2 [G, d, I] f32
@@ -238,7 +258,9 @@ int grouped_gemm_bwd_dw(const moe_dims* dims, const void* ws, int which, const v
                         const void* lhs_shared, const void* rhs_routed, const void* rhs_shared,
                         float* dw, int accumulate, void* stream);
 
-/* dW1_g = dA_g^T X_g (grouped_gemm_bwd_dw with which = MOE_GEMM1) with the
+/* Passage: as grouped_gemm_bwd_dw above (§Architecture "Mixture of Experts
+ * layer"; §3.2 "Performance comparison").
+ * dW1_g = dA_g^T X_g (grouped_gemm_bwd_dw with which = MOE_GEMM1) with the
  * routed groups' x rows gathered from x by sorted_ids as in
  * grouped_gemm_fwd_gather; no x_perm.
  *   sorted_ids [Rr] int32, da [Rt, 2I] bf16, x [T, d] bf16 (NULL only when T = 0)
@@ -261,7 +283,10 @@ int grouped_gemm_bwd_dw1_gather(const moe_dims* dims, const void* ws, const int3
 int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, const float* topk_w,
                 void* out, void* stream);
 
-/* moe_combine with the shared experts' rows in a buffer of their own:
+/* Passage: as moe_combine above; the expert-parallel layout it serves is the
+ * pages' training setting (§3.1, all-to-all dispatch and combine of expert
+ * parallelism overlapped with computation).
+ * moe_combine with the shared experts' rows in a buffer of their own:
  *   out[t] = sum_j topk_w[t, j] * y_routed[row_of[t, j]] + sum_s y_shared[s*T + t]
  * y_routed [Rr, d] bf16 (the routed rows of the grouped row space), y_shared
  * [S, T, d] bf16 (NULL only when S = 0).  The sums, their order and the
@@ -273,7 +298,8 @@ int moe_combine(const moe_dims* dims, const void* y, const int32_t* row_of, cons
 int moe_combine_split(const moe_dims* dims, const void* y_routed, const void* y_shared,
                       const int32_t* row_of, const float* topk_w, void* out, void* stream);
 
-/* moe_combine with the FP32 sums stored as they are, out [T, d] f32, without the
+/* Passage: as moe_combine above (§Architecture "Mixture of Experts layer").
+ * moe_combine with the FP32 sums stored as they are, out [T, d] f32, without the
  * final bf16 rounding (the same sums in the same order: rounding this output to
  * bf16 gives moe_combine's bits).  For callers that keep the layer output, or
  * dX before the router's term is added, in FP32. */
@@ -281,6 +307,10 @@ int moe_combine_f32(const moe_dims* dims, const void* y, const int32_t* row_of,
                     const float* topk_w, float* out, void* stream);
 
 /* Backward of the weighted combine.
+ * Passage: dots.llm1 Technical Report, §Architecture "Mixture of Experts layer"
+ * (the output is the affinity-weighted sum of the routed experts plus the
+ * shared experts; this is its gradient with respect to the routed rows and the
+ * weights).
  *   dout [T, d] bf16, y [Rt, d] bf16 (forward output rows), row_of, topk_w
  * Out:
  *   dy_routed [Rr, d] bf16   dy[row_of[t, j]] = topk_w[t, j] * dout[t];
@@ -347,7 +377,9 @@ int moe_seq_balance_loss(const moe_dims* dims, int64_t seq_len, float alpha,
                          const int32_t* topk_idx, const float* probs, float* loss,
                          float* seq_grad, void* ws, size_t ws_bytes, void* stream);
 
-/* moe_router_bwd with the sequence-wise balance loss's gradient included: for a
+/* Passage: as moe_router_bwd and moe_seq_balance_loss above (§Architecture
+ * "Mixture of Experts layer" and "Load balancing").
+ * moe_router_bwd with the sequence-wise balance loss's gradient included: for a
  * token t of sequence s = t / seq_len, dp[e] += seq_grad[s, e] for every expert
  * before the softmax backward, so dlogits, the gate's dx term and dwg carry
  * both losses.  seq_grad and seq_len as written and used by
@@ -370,14 +402,15 @@ int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
                     const float* bias_in, float* bias_out, void* stream);
 
 /* Reads and clears the device status word of `ws` (synchronises `stream`).
+ * Error reporting of this library: the pages have no counterpart.
  * *status_out receives MOE_OK or the first device error recorded. */
 int moe_get_device_status(void* ws, int32_t* status_out, void* stream);
 
 /* The CUDA error string behind the calling thread's most recent MOE_ERR_CUDA
- * ("no error" if there was none). */
+ * ("no error" if there was none).  No counterpart on the pages. */
 const char* moe_last_cuda_error(void);
 
-/* Human-readable name of a moe_status value. */
+/* Human-readable name of a moe_status value.  No counterpart on the pages. */
 const char* moe_status_string(int status);
 
 #ifdef __cplusplus

@@ -118,3 +118,24 @@ def check_routing(gidx, gw, probs, oidx, ow, margin, bias):
         gw_al = np.take_along_axis(gw, align, axis=1)
         assert np.max(np.abs(gw_al[same] - ow[same])) <= W_TOL
     return same, align
+
+
+def sample_tokens(oidx, cand, n, seed, per_expert=16):
+    """A seeded sample of ``n`` tokens for full-size parity checks: tokens of the
+    most-loaded and of the least-loaded non-empty routed experts (``per_expert``
+    of each), the first and last candidates, and random ones, all from ``cand``
+    (tokens eligible for an exact comparison), sorted and unique."""
+    rng = np.random.default_rng(seed)
+    cand = np.asarray(cand, dtype=np.int64)
+    E = int(oidx.max()) + 1
+    counts = np.bincount(oidx.ravel(), minlength=E)
+    nonempty = np.nonzero(counts)[0]
+    pick = []
+    for e in (int(counts.argmax()), int(nonempty[counts[nonempty].argmin()])):
+        mask = np.any(oidx[cand] == e, axis=1)
+        pick.extend(cand[mask][:per_expert].tolist())
+    pick.extend([int(cand[0]), int(cand[-1])])
+    rest = np.setdiff1d(cand, np.array(pick, dtype=np.int64))
+    need = max(0, n - len(set(pick)))
+    pick.extend(rng.choice(rest, min(need, len(rest)), replace=False).tolist())
+    return np.unique(np.array(pick, dtype=np.int64))

@@ -36,6 +36,38 @@ def test_header_declares_the_layer_calls():
         assert n in names
 
 
+def declaration_comments():
+    """Each declared function with the comment block that precedes it (a
+    comment may cover several consecutive declarations)."""
+    src = open(HEADER).read()
+    out = {}
+    last = ""
+    pos = 0
+    for m in re.finditer(r"/\*.*?\*/|;", src, flags=re.S):
+        chunk = src[pos:m.start()]
+        for n in re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\**"
+                            r"([a-z_][a-z0-9_]*)\s*\(", chunk, flags=re.M):
+            out[n] = last
+        if m.group(0).startswith("/*"):
+            last = m.group(0)
+        pos = m.end()
+    return out
+
+
+def test_every_entry_point_cites_its_passage():
+    """Every call of the layer names the passage of the pages that defines the
+    operation; host-side helpers and additions say the pages have none."""
+    comments = declaration_comments()
+    assert set(comments) == set(declared_functions())
+    for name in ("moe_gate_topk", "moe_permute_align", "grouped_gemm_fwd", "grouped_gemm_bwd_dx",
+                 "grouped_gemm_bwd_dw", "moe_combine", "moe_combine_bwd", "moe_router_bwd",
+                 "moe_seq_balance_loss", "moe_bias_update"):
+        assert "Passage:" in comments[name], name
+    for name, text in comments.items():
+        flat = " ".join(re.sub(r"\n\s*\*(?!/)", " ", text).split()).lower()
+        assert "passage:" in flat or "no counterpart" in flat, name
+
+
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", lib.lib_path()], capture_output=True,
                          text=True, check=True).stdout

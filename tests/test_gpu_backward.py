@@ -10,7 +10,8 @@ import torch
 
 import oracle
 import synth
-from common import assert_close, dev, dims_of, host, oracle_routing, workload_inputs
+from common import (assert_close, dev, dims_of, host, oracle_routing, sample_tokens,
+                    workload_inputs)
 import grouped_gemm_fp32_b200 as moe
 from grouped_gemm_fp32_b200 import layer
 
@@ -92,25 +93,34 @@ def test_backward_train_sampled():
     S, E, I = wl.dims.S, wl.dims.E, wl.dims.I
     p, oidx, ow, margin = oracle_routing(name)
     b, dx, dw1, dw2, dwc = _run(wl, inp, routing=(oidx, ow))
-    rng = np.random.default_rng(4)
-    tokens = np.sort(rng.choice(wl.dims.T, 24, replace=False)).astype(np.int64)
+    # 512 tokens, among them the hottest and the least-loaded experts' tokens (each
+    # token's out, dX and combine-weight gradient depend on that token alone)
+    tokens = sample_tokens(oidx, np.arange(wl.dims.T), 512, 4)
     ref_out = oracle.layer_fwd(inp["x"], oidx, ow, inp["w1"], inp["w2"], S, tokens=tokens)
     assert_close(host(b.out)[tokens], ref_out, "out")
     rdx, rdw = oracle.layer_bwd(inp["x"], oidx, ow, inp["w1"], inp["w2"], inp["dout"], S,
                                 tokens=tokens)
     assert_close(host(dx)[tokens], rdx, "dx")
     assert_close(host(dwc)[tokens], rdw, "d(combine weight)")
-    # sampled weight-gradient entries of 5 groups, every token of the group included
+    # the whole dW1 and dW2 of four routed experts (most-loaded, least-loaded
+    # non-empty, two random), each summing over every token of the expert
+    rng = np.random.default_rng(4)
     counts = np.bincount(oidx.ravel(), minlength=E)
     nonempty = np.nonzero(counts)[0]
     groups = [int(counts.argmax()), int(nonempty[counts[nonempty].argmin()]),
-              *map(int, rng.choice(E, 2, replace=False)), E]
-    rows1 = np.array([0, 1, I - 1, I, 2 * I - 1, int(rng.integers(0, 2 * I))], np.int32)
-    cols2 = np.array([0, 127, 128, I - 1, int(rng.integers(0, I))], np.int32)
-    DW1, DW2 = dw1, dw2
+              *map(int, rng.choice(E, 2, replace=False))]
     for g in groups:
-        r1, r2 = oracle.group_dw(inp["x"], oidx, ow, inp["w1"], inp["w2"], inp["dout"], S, g,
-                                 w1_rows=rows1, w2_cols=cols2)
-        assert_close(DW1[g][torch.from_numpy(rows1).long().cuda()].cpu().numpy(), r1, f"dW1[{g}]")
-        assert_close(DW2[g][:, torch.from_numpy(cols2).long().cuda()].cpu().numpy(), r2,
-                     f"dW2[{g}]")
+        r1, r2 = oracle.group_dw(inp["x"], oidx, ow, inp["w1"], inp["w2"], inp["dout"], S, g)
+        assert_close(dw1[g].cpu().numpy(), r1, f"dW1[{g}]")
+        assert_close(dw2[g].cpu().numpy(), r2, f"dW2[{g}]")
+    # shared expert 0 sums over all 16384 tokens (its whole dW is about 1 TFLOP of FP64
+    # work in the oracle): every 8th row of dW1 and column of dW2, plus the edges of
+    # the gate / up halves and of the 128-column tiles
+    rows1 = np.unique(np.concatenate([np.arange(0, 2 * I, 8), [1, I - 1, I, 2 * I - 1]])
+                      ).astype(np.int32)
+    cols2 = np.unique(np.concatenate([np.arange(0, I, 8), [127, 128, I - 1]])).astype(np.int32)
+    r1, r2 = oracle.group_dw(inp["x"], oidx, ow, inp["w1"], inp["w2"], inp["dout"], S, E,
+                             w1_rows=rows1, w2_cols=cols2)
+    assert_close(dw1[E][torch.from_numpy(rows1).long().cuda()].cpu().numpy(), r1, f"dW1[{E}]")
+    assert_close(dw2[E][:, torch.from_numpy(cols2).long().cuda()].cpu().numpy(), r2,
+                 f"dW2[{E}]")

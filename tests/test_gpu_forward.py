@@ -13,7 +13,7 @@ import torch
 import oracle
 import synth
 from common import (assert_close, check_routing, dev, dims_of, host, oracle_routing,
-                    workload_inputs)
+                    sample_tokens, workload_inputs)
 import grouped_gemm_fp32_b200 as moe
 from grouped_gemm_fp32_b200 import layer
 
@@ -88,7 +88,7 @@ def _layer_forward(name, dims_override=None, inputs=None):
     return inp, b, out
 
 
-@pytest.mark.parametrize("name,nsample", [("tiny", None), ("layer", 64), ("skewed", 64)])
+@pytest.mark.parametrize("name,nsample", [("tiny", None), ("layer", 512), ("skewed", 512)])
 def test_layer_forward_matches_oracle(name, nsample):
     inp, b, out = _layer_forward(name)
     wl = synth.WORKLOADS[name]
@@ -100,13 +100,8 @@ def test_layer_forward_matches_oracle(name, nsample):
     if nsample is None:
         tokens = np.nonzero(same)[0]
     else:
-        rng = np.random.default_rng(wl.seed)
-        cand = np.nonzero(same)[0]
-        # the heaviest expert's tokens and plain random ones
-        heavy = np.bincount(oidx.ravel(), minlength=wl.dims.E).argmax()
-        tok_heavy = [t for t in cand if heavy in oidx[t]][:8]
-        tokens = np.unique(np.concatenate([rng.choice(cand, nsample, replace=False), tok_heavy,
-                                           [cand[0], cand[-1]]])).astype(np.int64)
+        # 512 tokens: the hottest and the least-loaded experts' tokens among them
+        tokens = sample_tokens(oidx, np.nonzero(same)[0], nsample, wl.seed)
     ref, yr, ys = oracle.layer_fwd(inp["x"], oidx, ow, inp["w1"], inp["w2"], S, tokens=tokens,
                                    want_y=True)
     assert_close(host(out)[tokens], ref, f"{name} out")
