@@ -74,7 +74,7 @@ def parse():
                          "reading the permuted copy x_perm")
     ap.add_argument("--ep", action="store_true",
                     help="a line of its own: the train step under expert parallelism over the "
-                         "ranks (one rank: every segment exchange a local copy)")
+                         "ranks (one rank: every peer pointer the rank's own buffer)")
     ap.add_argument("--library-gemm", action="store_true",
                     help="context, not the contract line: cuBLAS (torch.bmm) on the same GEMM "
                          "shapes with uniform groups, timed interleaved with this library's "
@@ -792,16 +792,18 @@ def run_library_gemm(args, rounds=8, timed=3):
 
 
 def run_ep(args):
-    """The train step under expert parallelism (grouped_gemm_fp32_b200.ep): every rank
-    routes its own T tokens over all E experts and owns E / W of them, the padded
-    segments travel to their owners and back by NCCL send/recv.  With one process the
-    group has one rank (every segment a local copy): the EP code path with no link
-    traffic.  The step runs as eager calls (the segment sizes come to the host once per
-    step, so it is not captured in a graph).  A line of its own, not the contract's."""
+    """The train step under expert parallelism (grouped_gemm_fp32_b200.ep) over the ranks:
+    every rank routes its own T tokens over all E experts and owns E / W of them; rows move
+    by kernels writing into the other ranks' buffers (symmetric memory), with an NCCL
+    all-gather of the counts and all-reduce of the loads, and no host sync, so the step is
+    captured in a CUDA graph and replayed.  With one process the group has one rank (every
+    peer pointer the rank's own buffer): the EP code path with no link traffic, timed
+    beside the single-GPU layer step in the same process (alternating rounds, same clocks).
+    A line of its own, not the contract's."""
     import torch
     import torch.distributed as dist
     import grouped_gemm_fp32_b200 as moe
-    from grouped_gemm_fp32_b200 import ep
+    from grouped_gemm_fp32_b200 import ep, layer
 
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
@@ -818,51 +820,87 @@ def run_ep(args):
     w1, w2 = bf(inp["w1"]), bf(inp["w2"])
     w1l = torch.cat([w1[rank * El:(rank + 1) * El], w1[E:]]).contiguous()
     w2l = torch.cat([w2[rank * El:(rank + 1) * El], w2[E:]]).contiguous()
-    del w1, w2
+    if world > 1:
+        del w1, w2
     wg, bias = torch.from_numpy(inp["wg"]).to(dev), torch.from_numpy(inp["bias"]).to(dev)
-    eb = ep.EPBuffers(dims, rank, world, train=True, device=dev)
+    eb = ep.EPBuffers(dims, rank, world, train=True, device=dev,
+                      alloc=ep.symmetric_alloc(world, dev))
+    ep.connect(eb)
     stream = torch.cuda.Stream(device=dev)
 
     def step():
         ep.forward(eb, x, wg, bias, w1l, w2l, stream=stream, seq_balance=SEQ_BALANCE)
         ep.backward(eb, x, dout, w1l, w2l, stream=stream, wg=wg, gamma=GAMMA, bias=bias)
 
-    for _ in range(args.warmup):
-        step()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
     stream.synchronize()
-    for buf in (eb.full.ws, eb.loc.ws):
-        status = moe.moe_get_device_status(buf, stream)
-        if status != 0:
-            raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(status)}")
+    st = ep.status(eb, stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(st)}")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    single = None
+    if world == 1:  # the single-GPU layer step on the same batch, for the same-clock ratio
+        b1 = layer.MoEBuffers(dims, device=dev, train=True)
+        single = layer.GraphStep(b1, x, wg, bias, w1, w2, dout=dout, gamma=GAMMA,
+                                 seq_balance=SEQ_BALANCE)
+
+    def timed(replay, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n):
+                replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / n
+
     clk = ClockSampler(local)
     clk.start()
     time.sleep(0.25)
     barrier(world)
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    e1.synchronize()
+    rounds = 4 if single is not None else 1
+    per = max(1, args.steps // rounds)
+    ep_ms, one_ms = [], []
+    for r in range(rounds):
+        pair = [("ep", lambda: graph.replay()), ("one", lambda: single.replay())]
+        if single is None:
+            pair = pair[:1]
+        for name, f in (pair if r % 2 == 0 else pair[::-1]):
+            (ep_ms if name == "ep" else one_ms).append(timed(f, per))
     barrier(world)
     clocks = clk.stop()
-    ms = dist_max(e0.elapsed_time(e1) / args.steps, world, dev)
-    recv = dist_max(float(eb.plan.recv_rows), world, dev)
+    st = ep.status(eb, stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {moe.moe_status_string(st)}")
+    ms = dist_max(sum(ep_ms) / len(ep_ms), world, dev)
+    med = lambda v: sorted(v)[len(v) // 2]
     if rank == 0:
         line = {"metric": METRIC, "value": world * dm.T / (ms / 1000.0), "unit": "tokens/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "n_gpus": world, "steps": per * rounds, "warmup": args.warmup,
                 "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours-ep",
                 "config": {"workload": describe(wl) + ", expert parallel",
                            "parallelism": f"ep{world}", "experts_per_rank": El,
                            "tokens_per_gpu": dm.T, "seq_balance": {"alpha": SEQ_BALANCE[0],
                                                                    "seq_len": SEQ_BALANCE[1]},
-                           "max_rows_received": int(recv),
-                           "step": "eager C-ABI calls; counts all-to-all, segment send/recv "
-                                   "over NCCL, segment sizes to the host once per step"},
+                           "recv_rows_cap": eb.cap,
+                           "step": "CUDA graph replay: gate, routing tables, NCCL all-gather "
+                                   "of the counts, device plan, rows written into the owners' "
+                                   "buffers, owners' grouped GEMMs (shared tiles first, "
+                                   "bounded waits for the rows), outputs written back into "
+                                   "the sources' buffers, combine; backward likewise; no "
+                                   "host sync"},
                 "clocks": clocks}
+        if one_ms:
+            line["single_gpu_step_ms"] = sum(one_ms) / len(one_ms)
+            line["ep_over_single_gpu"] = med([a / b for a, b in zip(ep_ms, one_ms)])
         print(json.dumps(line), flush=True)
+    del graph
     barrier(world)
     dist.destroy_process_group()
 

@@ -14,4 +14,7 @@ from ._lib import (MOE_GEMM1, MOE_GEMM2, MoeDims, MoeError, grouped_gemm_bwd_dw,
                    moe_gate_topk, moe_get_device_status, moe_last_cuda_error, moe_permute_align,
                    moe_permute_align_static, moe_router_bwd, moe_router_bwd_seqbal,
                    moe_rows_routed, moe_rows_total, moe_seq_balance_loss, moe_status_string,
-                   moe_workspace_size)
+                   moe_workspace_size, MOE_EP_MAX_WORLD, MOE_EP_WAIT_DX, MOE_EP_WAIT_Y,
+                   MoeEpPeers, grouped_gemm_bwd_dx_ep, grouped_gemm_fwd_ep, moe_ep_combine_bwd,
+                   moe_ep_dispatch, moe_ep_plan, moe_ep_wait, moe_ep_workspace_size,
+                   moe_ep_zero_pads)

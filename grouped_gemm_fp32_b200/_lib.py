@@ -22,7 +22,11 @@ EXPORTS = (
     "moe_combine_bwd", "moe_router_bwd", "moe_router_bwd_seqbal", "moe_seq_balance_loss",
     "moe_bias_update", "moe_get_device_status",
     "moe_status_string", "moe_last_cuda_error",
+    "moe_ep_workspace_size", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_zero_pads", "moe_ep_wait",
+    "moe_ep_combine_bwd", "grouped_gemm_fwd_ep", "grouped_gemm_bwd_dx_ep",
 )
+MOE_EP_MAX_WORLD = 8
+MOE_EP_WAIT_Y, MOE_EP_WAIT_DX = 3, 5
 
 
 class MoeError(RuntimeError):
@@ -46,6 +50,26 @@ class MoeDims(ctypes.Structure):
 
     def __repr__(self):
         return ("MoeDims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")")
+
+
+class MoeEpPeers(ctypes.Structure):
+    """Mirror of ``struct moe_ep_peers`` in include/moe.h: this rank, the world, and
+    every rank's EP workspace and destination rows as device addresses mapped in
+    this process."""
+    _fields_ = [("rank", ctypes.c_int32), ("world", ctypes.c_int32),
+                ("rows_cap", ctypes.c_int64),
+                ("ep_ws", ctypes.c_void_p * MOE_EP_MAX_WORLD),
+                ("rows", ctypes.c_void_p * MOE_EP_MAX_WORLD)]
+
+    @classmethod
+    def of(cls, rank, world, ep_ws, rows=None, rows_cap=0):
+        """``ep_ws`` / ``rows``: per-rank device addresses (ints) or tensors."""
+        p = cls()
+        p.rank, p.world, p.rows_cap = int(rank), int(world), int(rows_cap)
+        for o in range(world):
+            p.ep_ws[o] = _p(ep_ws[o])
+            p.rows[o] = _p(rows[o]) if rows is not None else None
+        return p
 
 
 def lib_path() -> str:
@@ -86,6 +110,17 @@ def load():
         "moe_bias_update": (i32, [D, vp, ctypes.c_float, vp, vp, vp]),
         "moe_combine_bwd": (i32, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
         "moe_get_device_status": (i32, [vp, vp, vp]),
+        "moe_ep_workspace_size": (sz, [D, i32]),
+        "moe_ep_plan": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, i64, vp]),
+        "moe_ep_dispatch": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, vp, vp, vp]),
+        "moe_ep_zero_pads": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp]),
+        "moe_ep_wait": (i32, [ctypes.POINTER(MoeEpPeers), i32, vp]),
+        "moe_ep_combine_bwd": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, vp, vp, vp, vp, vp,
+                                     vp]),
+        "grouped_gemm_fwd_ep": (i32, [D, vp, ctypes.POINTER(MoeEpPeers), vp, vp, vp, vp, vp, vp,
+                                      vp, vp]),
+        "grouped_gemm_bwd_dx_ep": (i32, [D, vp, ctypes.POINTER(MoeEpPeers), i32, vp, vp, vp, vp,
+                                         vp, vp]),
         "moe_status_string": (ctypes.c_char_p, [i32]),
         "moe_last_cuda_error": (ctypes.c_char_p, []),
     }
@@ -252,3 +287,45 @@ def moe_get_device_status(ws, stream=None) -> int:
     _ck(load().moe_get_device_status(_p(ws), ctypes.addressof(out), _s(stream)),
         "moe_get_device_status")
     return int(out.value)
+
+
+# ------------------------------------------------------ expert parallelism --
+def moe_ep_workspace_size(dims, world) -> int:
+    return int(load().moe_ep_workspace_size(ctypes.byref(dims), int(world)))
+
+
+def moe_ep_plan(dims, peers, counts_all, counts_loc, recv_cap, stream=None):
+    _ck(load().moe_ep_plan(ctypes.byref(dims), ctypes.byref(peers), _p(counts_all),
+                           _p(counts_loc), int(recv_cap), _s(stream)), "moe_ep_plan")
+
+
+def moe_ep_dispatch(dims, peers, topk_idx, row_of, offsets, x, stream=None):
+    _ck(load().moe_ep_dispatch(ctypes.byref(dims), ctypes.byref(peers), _p(topk_idx), _p(row_of),
+                               _p(offsets), _p(x), _s(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_zero_pads(dims, peers, recv, stream=None):
+    _ck(load().moe_ep_zero_pads(ctypes.byref(dims), ctypes.byref(peers), _p(recv), _s(stream)),
+        "moe_ep_zero_pads")
+
+
+def moe_ep_wait(peers, which, stream=None):
+    _ck(load().moe_ep_wait(ctypes.byref(peers), int(which), _s(stream)), "moe_ep_wait")
+
+
+def moe_ep_combine_bwd(dims, peers, dout, y, row_of, topk_w, topk_idx, offsets, dw, stream=None):
+    _ck(load().moe_ep_combine_bwd(ctypes.byref(dims), ctypes.byref(peers), _p(dout), _p(y),
+                                  _p(row_of), _p(topk_w), _p(topk_idx), _p(offsets), _p(dw),
+                                  _s(stream)), "moe_ep_combine_bwd")
+
+
+def grouped_gemm_fwd_ep(dims, ws, peers, x_recv, x, w1, w2, h, a1, y, stream=None):
+    _ck(load().grouped_gemm_fwd_ep(ctypes.byref(dims), _p(ws), ctypes.byref(peers), _p(x_recv),
+                                   _p(x), _p(w1), _p(w2), _p(h), _p(a1), _p(y), _s(stream)),
+        "grouped_gemm_fwd_ep")
+
+
+def grouped_gemm_bwd_dx_ep(dims, ws, peers, which, dy_recv, dy_shared, w, a1, out, stream=None):
+    _ck(load().grouped_gemm_bwd_dx_ep(ctypes.byref(dims), _p(ws), ctypes.byref(peers), int(which),
+                                      _p(dy_recv), _p(dy_shared), _p(w), _p(a1), _p(out),
+                                      _s(stream)), "grouped_gemm_bwd_dx_ep")

@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "ep_internal.cuh"
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -115,24 +116,24 @@ __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* 
                                    const int32_t* __restrict__ row_of, const float* __restrict__ w,
                                    int64_t T, int row_vec, int k, int64_t Rr,
                                    uint4* __restrict__ dy,
-                                   float* __restrict__ dw) {
+                                   float* __restrict__ dw, EpDy ep) {
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  for (int j = 0; j < k; ++j) {
+  for (int j = 0; t < T && j < k; ++j) {
     const int64_t r = row_of[t * k + j];
     const float wj = w[t * k + j];
     if (r < 0 || r >= Rr) {  // a pick without a row: nothing to scatter, no gradient
       if (lane == 0) dw[t * k + j] = 0.0f;
       continue;
     }
+    uint4* drow = ep_dy_row(ep, dy, t, k, j, r, row_vec);
     float dot = 0.0f;
     for (int c = lane; c < row_vec; c += 32) {
       const uint4 g = dout[t * row_vec + c];
       const uint4 yv = y[r * row_vec + c];
       float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       acc8(a, g, wj);
-      dy[r * row_vec + c] = pack8(a);
+      if (drow) drow[c] = pack8(a);
       const uint32_t gu[4] = {g.x, g.y, g.z, g.w}, yu[4] = {yv.x, yv.y, yv.z, yv.w};
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
@@ -144,6 +145,7 @@ __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* 
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     if (lane == 0) dw[t * k + j] = dot;
   }
+  if (ep.W) ep_signal_last_cta(ep.done, ep.peer_ws, ep.W, EP_CTR_DY);
 }
 
 // Same, with the token's dOut row held in registers for all k picks: lane l owns
@@ -153,21 +155,23 @@ template <int VPL>
 __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                                        const int32_t* __restrict__ row_of,
                                        const float* __restrict__ w, int64_t T, int k, int64_t Rr,
-                                       uint4* __restrict__ dy, float* __restrict__ dw) {
+                                       uint4* __restrict__ dy, float* __restrict__ dw, EpDy ep) {
   constexpr int row_vec = 32 * VPL;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (t >= T) return;
   uint4 g[VPL];
+  if (t < T) {
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) g[i] = dout[t * row_vec + lane + 32 * i];
-  for (int j = 0; j < k; ++j) {
+    for (int i = 0; i < VPL; ++i) g[i] = dout[t * row_vec + lane + 32 * i];
+  }
+  for (int j = 0; t < T && j < k; ++j) {
     const int64_t r = row_of[t * k + j];
     const float wj = w[t * k + j];
     if (r < 0 || r >= Rr) {  // a pick without a row: nothing to scatter, no gradient
       if (lane == 0) dw[t * k + j] = 0.0f;
       continue;
     }
+    uint4* drow = ep_dy_row(ep, dy, t, k, j, r, row_vec);
     uint4 yv[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) yv[i] = y[r * row_vec + lane + 32 * i];
@@ -176,7 +180,7 @@ __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uin
     for (int i = 0; i < VPL; ++i) {
       float a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       acc8(a, g[i], wj);
-      dy[r * row_vec + lane + 32 * i] = pack8(a);
+      if (drow) drow[lane + 32 * i] = pack8(a);
       const uint32_t gu[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
       const uint32_t yu[4] = {yv[i].x, yv[i].y, yv[i].z, yv[i].w};
 #pragma unroll
@@ -190,6 +194,7 @@ __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uin
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     if (lane == 0) dw[t * k + j] = dot;
   }
+  if (ep.W) ep_signal_last_cta(ep.done, ep.peer_ws, ep.W, EP_CTR_DY);
 }
 
 }  // namespace
@@ -225,30 +230,59 @@ int launch_combine(const moe_dims& dm, const void* y, const void* y_shared,
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
-                       const int32_t* row_of, const float* w, void* dy, float* dw, void* stream) {
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int rc = launch_zero_pad_rows(dm, ws, dy, dm.d, stream);
-  if (rc != MOE_OK || dm.T == 0) return rc;
+static int combine_bwd_kernels(const moe_dims& dm, const void* dout, const void* y,
+                               const int32_t* row_of, const float* w, void* dy, float* dw,
+                               const EpDy& ep, cudaStream_t st) {
   const int warps = 8;
-  const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);
+  // one CTA at least: under expert parallelism the last CTA signals the owners
+  const unsigned blocks = (unsigned)(dm.T > 0 ? (dm.T + warps - 1) / warps : 1);
   const int64_t Rr = rows_routed(dm);
   const uint4* dv = reinterpret_cast<const uint4*>(dout);
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* dyv = reinterpret_cast<uint4*>(dy);
   const int row_vec = dm.d / 8;
   // the register-resident form uses ~170 registers a thread: 4-warp CTAs, three per SM
-  const unsigned blocks4 = (unsigned)((dm.T + 3) / 4);
+  const unsigned blocks4 = (unsigned)(dm.T > 0 ? (dm.T + 3) / 4 : 1);
   if (row_vec == 512)
     combine_bwd_reg_kernel<16><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, Rr, dyv,
-                                                        dw);
+                                                        dw, ep);
   else if (row_vec == 256)
     combine_bwd_reg_kernel<8><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, Rr, dyv,
-                                                       dw);
+                                                       dw, ep);
   else
     combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, row_vec, dm.k, Rr,
-                                                      dyv, dw);
+                                                      dyv, dw, ep);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
+                       const int32_t* row_of, const float* w, void* dy, float* dw, void* stream) {
+  int rc = launch_zero_pad_rows(dm, ws, dy, dm.d, stream);
+  if (rc != MOE_OK || dm.T == 0) return rc;
+  EpDy none{};
+  return combine_bwd_kernels(dm, dout, y, row_of, w, dy, dw, none,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Under expert parallelism: dY rows go to their owners' receive buffers (whose
+// pad rows the owners zero), and the last CTA signals every owner.
+int launch_combine_bwd_ep(const moe_dims& dm, const moe_ep_peers& pe, const void* dout,
+                          const void* y, const int32_t* row_of, const float* w,
+                          const int32_t* idx, const int32_t* offsets, float* dw, void* stream) {
+  const EpLayout L = ep_layout(dm.E, pe.world);
+  uint8_t* epb = reinterpret_cast<uint8_t*>(pe.ep_ws[pe.rank]);
+  EpDy ep{};
+  ep.rows = ep_ptrs(pe.rows, pe.world);
+  ep.peer_ws = ep_ptrs(pe.ep_ws, pe.world);
+  ep.send_dst = reinterpret_cast<const int32_t*>(epb + L.send_dst);
+  ep.over = reinterpret_cast<const int32_t*>(epb + L.over);
+  ep.idx = idx;
+  ep.offsets = offsets;
+  ep.done = reinterpret_cast<int*>(epb) + EP_DONE_DY;
+  ep.El = dm.E / pe.world;
+  ep.W = pe.world;
+  return combine_bwd_kernels(dm, dout, y, row_of, w, nullptr, dw, ep,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace moe

@@ -37,9 +37,11 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <type_traits>
 
+#include "ep_internal.cuh"
 #include "moe_internal.cuh"
 #include "sm100.cuh"
 
@@ -87,6 +89,15 @@ struct GemmArgs {
   uint64_t budget_ns;
   const int32_t* gather_ids;  // FWD1 / DW1: token of each routed row, or null
   int gather_T;               // rows of the gathered tensor x
+  int shared_first;           // FWD / DX: the shared groups' tiles come first
+  EpGemm ep;                  // expert parallelism: rows to wait for, outputs to return
+};
+
+// Tensor maps of every source rank's rows (expert parallelism: FWD2 / DX1 write
+// a routed group's output rows straight into the buffers of the ranks the rows
+// came from).
+struct EpMaps {
+  CUtensorMap m[kEpMaxWorld];
 };
 
 // full[] and tempty[] are used in the leader CTA only (both CTAs' producers and
@@ -162,8 +173,13 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     t.nw = (a.n_out - t.n0 > 128) ? 256 : 128;
     t.half = 0;
   } else {
-    // largest g with prefix[g] * NT <= tile  (the prefix is non-decreasing)
     const int* pre = a.mtile_prefix;
+    if (a.shared_first) {  // rotate: the shared groups' tiles (they need no exchange) first
+      const int tot = __ldg(pre + a.G) * a.NT, sh = __ldg(pre + a.E) * a.NT;
+      tile += sh;
+      if (tile >= tot) tile -= tot;
+    }
+    // largest g with prefix[g] * NT <= tile  (the prefix is non-decreasing)
     int lo = 0, hi = a.G - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -275,7 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                  const __grid_constant__ CUtensorMap tmA0h /* half tiles: 64-row A boxes */,
                  const __grid_constant__ CUtensorMap tmA1h,
                  const __grid_constant__ CUtensorMap tmBh /* FWD1 half tiles: 64-row B boxes */,
-                 const GemmArgs args) {
+                 const __grid_constant__ EpMaps epm, const GemmArgs args) {
   constexpr bool A_MN = (MODE == MODE_DW2 || MODE == MODE_DW1);
   constexpr bool B_MN = (MODE != MODE_FWD1 && MODE != MODE_FWD2);
   constexpr bool IS_DW = A_MN;
@@ -352,11 +368,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, lastpar = 0;
       bool ok = true;
+      bool rows_in = args.ep.wait_ctr == 0;  // the routed rows of other ranks have arrived
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<MODE>(tile, args);
         const GroupRec gr = load_group(args, t.g);
         const int roff = (int)rank * (t.half ? BM / 2 : BM);  // this CTA's rows of A
         const bool shared = t.g >= args.E;
+        if (!shared && !rows_in) {
+          // expert parallelism: every source's rows of this rank's experts must have
+          // landed before the first routed tile's copies (bounded wait)
+          int got = 1;
+          if (lane == 0) {
+            got = ep_wait_counter(args.ep.ep_ws, args.ep.wait_ctr, args.ep.world, args.status,
+                                  MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
+            // the rows were written through the generic proxy; the copies read them
+            // through the async proxy
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+          }
+          if constexpr (WIDE) got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            if (lane == 0) abort_pair();
+            break;
+          }
+          rows_in = true;
+        }
         const bool gat = WIDE && !shared;
         // this CTA's half of B: N/2 columns from n0 + rank * N/2, in 64-column chunks
         const int bchunks = t.nw / 128;
@@ -696,7 +731,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(u[8 * j + i]);
               pk[4 + j] = pack_bf16x8(v);
             }
-            staged_store<false>(slot, pk, &tmO0, t.n0 + coff + c0, gr.out_row + rb, lane);
+            const CUtensorMap* om = &tmO0;
+            int orow_y = gr.out_row + rb;
+            if (args.ep.ret_ctr != 0 && t.g < args.E) {
+              // this 32-row block lies inside one source's segment (segments are
+              // padded to a multiple of 32 rows): its rows go back to that rank
+              const int El = args.ep.El;
+              int src = 0;
+              while (src + 1 < args.ep.world && orow_y >= __ldg(args.ep.recv_row + (src + 1) * El + t.g))
+                ++src;
+              orow_y = __ldg(args.ep.src_off + src * El + t.g) +
+                       (orow_y - __ldg(args.ep.recv_row + src * El + t.g));
+              om = &epm.m[src];
+            }
+            staged_store<false>(slot, pk, om, t.n0 + coff + c0, orow_y, lane);
           } else if (rv) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -798,7 +846,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
     }
     // every staged store has finished (written to global memory) before the CTA can exit
-    if (lane == 0) bulk_wait_all();
+    if (lane == 0) {
+      bulk_wait_all();
+      if (args.ep.ret_ctr != 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
     __syncwarp();
   }
 
@@ -815,13 +866,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
+  // expert parallelism: once every CTA's output rows are in their sources'
+  // buffers, the last CTA tells each source rank
+  if (args.ep.ret_ctr != 0)
+    ep_signal_last_cta(const_cast<int*>(args.ep.ep_ws) + args.ep.done_word, args.ep.peer_ws,
+                       args.ep.world, args.ep.ret_ctr);
 }
 
 template <int MODE>
 int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
                 const CUtensorMap& b1, const CUtensorMap& c, const CUtensorMap& o0,
                 const CUtensorMap& o1, const CUtensorMap& a0h, const CUtensorMap& a1h,
-                const CUtensorMap& bh, const GemmArgs& args, cudaStream_t st) {
+                const CUtensorMap& bh, const EpMaps& epm, const GemmArgs& args, cudaStream_t st) {
   static int num_sms = 0;
   static bool attr_set = false;
   constexpr size_t kSmem = smem_bytes<MODE>();
@@ -848,7 +904,7 @@ int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
     attr_set = true;
   }
   ggemm_kernel<MODE><<<num_sms, NUM_THREADS, kSmem, st>>>(a0, a1, b0, b1, c, o0, o1, a0h, a1h,
-                                                          bh, args);
+                                                          bh, epm, args);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -927,6 +983,30 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   a.aux = ops.aux;
   a.accumulate = ops.accumulate;
   a.budget_ns = wait_budget_ns();
+  a.shared_first = ops.shared_first;
+
+  // expert parallelism: rows to wait for (FWD1 / DX2), outputs to return (FWD2 / DX1)
+  EpMaps epm;
+  memset(&epm, 0, sizeof(epm));
+  if (ops.ep != nullptr) {
+    const moe_ep_peers& pe = *ops.ep;
+    const EpLayout EL = ep_layout(dm.E * pe.world, pe.world);
+    const uint8_t* epb = reinterpret_cast<const uint8_t*>(pe.ep_ws[pe.rank]);
+    a.ep.ep_ws = reinterpret_cast<const int*>(epb);
+    a.ep.world = pe.world;
+    a.ep.El = dm.E;
+    a.ep.peer_ws = ep_ptrs(pe.ep_ws, pe.world);
+    a.ep.recv_row = reinterpret_cast<const int32_t*>(epb + EL.recv_row);
+    a.ep.src_off = reinterpret_cast<const int32_t*>(epb + EL.src_off);
+    if (mode == MODE_FWD1 || mode == MODE_DX2) {
+      a.ep.wait_ctr = mode == MODE_FWD1 ? EP_CTR_ROWS : EP_CTR_DY;
+    } else if (mode == MODE_FWD2 || mode == MODE_DX1) {
+      a.ep.ret_ctr = mode == MODE_FWD2 ? EP_CTR_Y : EP_CTR_DX;
+      a.ep.done_word = mode == MODE_FWD2 ? EP_DONE_Y : EP_DONE_DX;
+      for (int o = 0; o < pe.world; ++o)
+        if (!make_map_2d(&epm.m[o], pe.rows[o], pe.rows_cap, dm.d, 2, 32)) return MOE_ERR_CUDA;
+    }
+  }
 
   CUtensorMap m0{}, m1{}, n0{}, n1{}, c0{}, o0{}, o1{};
   CUtensorMap mh0{}, mh1{}, nh{};  // half tiles: 64-row boxes of A (and of B in FWD1)
@@ -971,7 +1051,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_2d(&o0, ops.out, Rt, I, 2, 32);
       if (ops.out2 != nullptr) ok &= make_map_2d(&o1, ops.out2, Rt, 2 * I, 2, 32); else same(o1, o0);
       if (!ok) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, o0, o1, mh0, mh1, nh, a, st);
+      return launch_mode<MODE_FWD1>(m0, m1, n0, n1, n0, o0, o1, mh0, mh1, nh, epm, a, st);
     }
     case MODE_FWD2: {
       a.K = I;
@@ -992,7 +1072,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, a, st);
+      return launch_mode<MODE_FWD2>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, epm, a, st);
     }
     case MODE_DX2: {
       a.K = d;
@@ -1017,7 +1097,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, 2 * I, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, o0, o0, mh0, mh1, nh, a, st);
+      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, o0, o0, mh0, mh1, nh, epm, a, st);
     }
     case MODE_DX1: {
       a.K = 2 * I;
@@ -1040,7 +1120,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, a, st);
+      return launch_mode<MODE_DX1>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, epm, a, st);
     }
     case MODE_DW2: {  // dW2_g [d, I] = dY_g^T H_g
       a.m_out = d;
@@ -1056,7 +1136,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * d, I, 4, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, a, st);
+      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, epm, a, st);
     }
     case MODE_DW1: {  // dW1_g [2I, d] = dA_g^T X_g
       a.m_out = 2 * I;
@@ -1079,7 +1159,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * 2 * I, d, 4, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, a, st);
+      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, epm, a, st);
     }
   }
   return MOE_ERR_INVALID_ARG;

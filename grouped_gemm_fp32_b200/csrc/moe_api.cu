@@ -3,6 +3,7 @@
 // (except moe_get_device_status), nothing but plain pointers and sizes.
 #include <cuda_runtime.h>
 
+#include "ep_internal.cuh"
 #include "moe_internal.cuh"
 
 using namespace moe;
@@ -275,6 +276,117 @@ int moe_combine_bwd(const moe_dims* dims, const void* ws, const void* dout, cons
   if (!ws || !dy_routed) return MOE_ERR_INVALID_ARG;
   if (dims->T > 0 && (!dout || !y || !row_of || !topk_w || !dw)) return MOE_ERR_INVALID_ARG;
   return launch_combine_bwd(*dims, ws, dout, y, row_of, topk_w, dy_routed, dw, stream);
+}
+
+// ------------------------------------------------------ expert parallelism --
+static int check_ep(const moe_dims* dims, const moe_ep_peers* peers, bool need_rows) {
+  int rc = check_shape(dims, false);
+  if (rc) return rc;
+  if (!ep_peers_ok(peers, need_rows)) return MOE_ERR_INVALID_ARG;
+  if (dims->E % peers->world || dims->P % 32 || dims->k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+size_t moe_ep_workspace_size(const moe_dims* dims, int32_t world) {
+  if (!dims_ok(dims) || world < 1 || world > MOE_EP_MAX_WORLD || dims->E % world) return 0;
+  return ep_layout(dims->E, world).bytes;
+}
+
+int moe_ep_plan(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* counts_all,
+                int32_t* counts_loc, int64_t recv_cap, void* stream) {
+  int rc = check_ep(dims, peers, false);
+  if (rc) return rc;
+  if (!counts_all || !counts_loc || recv_cap < 0) return MOE_ERR_INVALID_ARG;
+  return launch_ep_plan(*dims, *peers, counts_all, counts_loc, recv_cap, stream);
+}
+
+int moe_ep_dispatch(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* topk_idx,
+                    const int32_t* row_of, const int32_t* offsets, const void* x, void* stream) {
+  int rc = check_ep(dims, peers, true);
+  if (rc) return rc;
+  if (!offsets || (dims->T > 0 && (!topk_idx || !row_of || !x))) return MOE_ERR_INVALID_ARG;
+  return launch_ep_dispatch(*dims, *peers, topk_idx, row_of, offsets, x, stream);
+}
+
+int moe_ep_zero_pads(const moe_dims* dims, const moe_ep_peers* peers, void* recv, void* stream) {
+  int rc = check_ep(dims, peers, false);
+  if (rc) return rc;
+  if (!recv) return MOE_ERR_INVALID_ARG;
+  return launch_ep_zero_pads(*dims, *peers, recv, stream);
+}
+
+int moe_ep_wait(const moe_ep_peers* peers, int which, void* stream) {
+  if (!ep_peers_ok(peers, false)) return MOE_ERR_INVALID_ARG;
+  if (which != MOE_EP_WAIT_Y && which != MOE_EP_WAIT_DX) return MOE_ERR_INVALID_ARG;
+  return launch_ep_wait(*peers, which, stream);
+}
+
+int moe_ep_combine_bwd(const moe_dims* dims, const moe_ep_peers* peers, const void* dout,
+                       const void* y, const int32_t* row_of, const float* topk_w,
+                       const int32_t* topk_idx, const int32_t* offsets, float* dw, void* stream) {
+  int rc = check_ep(dims, peers, true);
+  if (rc) return rc;
+  if (!offsets || (dims->T > 0 && (!dout || !y || !row_of || !topk_w || !topk_idx || !dw)))
+    return MOE_ERR_INVALID_ARG;
+  return launch_combine_bwd_ep(*dims, *peers, dout, y, row_of, topk_w, topk_idx, offsets, dw,
+                               stream);
+}
+
+// The local dims of an owner: E_l routed groups; its peers' ep workspaces were sized
+// for E = E_l W.
+static int check_ep_local(const moe_dims* dims, const moe_ep_peers* peers, bool need_rows) {
+  int rc = check_shape(dims, true);
+  if (rc) return rc;
+  if (!ep_peers_ok(peers, need_rows)) return MOE_ERR_INVALID_ARG;
+  if (dims->P % 32 || (int64_t)dims->E * peers->world > 256) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+int grouped_gemm_fwd_ep(const moe_dims* dims, const void* ws, const moe_ep_peers* peers,
+                        const void* x_recv, const void* x, const void* w1, const void* w2,
+                        void* h, void* a1, void* y, void* stream) {
+  int rc = check_ep_local(dims, peers, true);
+  if (rc) return rc;
+  if (!ws || !x_recv || !w1 || !w2 || !h || !y || (dims->S > 0 && dims->T > 0 && !x))
+    return MOE_ERR_INVALID_ARG;
+  GemmOperands o{};
+  o.a0 = x_recv;
+  o.a1 = x;
+  o.b0 = w1;
+  o.out = h;
+  o.out2 = a1;
+  o.ep = peers;
+  o.shared_first = 1;
+  rc = launch_grouped_gemm(MODE_FWD1, *dims, ws, o, stream);
+  if (rc) return rc;
+  GemmOperands o2{};
+  o2.a0 = h;
+  o2.b0 = w2;
+  o2.out = y;
+  o2.ep = peers;
+  return launch_grouped_gemm(MODE_FWD2, *dims, ws, o2, stream);
+}
+
+int grouped_gemm_bwd_dx_ep(const moe_dims* dims, const void* ws, const moe_ep_peers* peers,
+                           int which, const void* dy_recv, const void* dy_shared, const void* w,
+                           const void* a1, void* out, void* stream) {
+  int rc = check_ep_local(dims, peers, which == MOE_GEMM1);
+  if (rc) return rc;
+  if (!ws || !dy_recv || !w || !out) return MOE_ERR_INVALID_ARG;
+  GemmOperands o{};
+  o.a0 = dy_recv;
+  o.b0 = w;
+  o.out = out;
+  o.ep = peers;
+  if (which == MOE_GEMM2) {
+    if (!a1 || (dims->S > 0 && dims->T > 0 && !dy_shared)) return MOE_ERR_INVALID_ARG;
+    o.a1 = dy_shared;
+    o.aux = a1;
+    o.shared_first = 1;
+    return launch_grouped_gemm(MODE_DX2, *dims, ws, o, stream);
+  }
+  if (which == MOE_GEMM1) return launch_grouped_gemm(MODE_DX1, *dims, ws, o, stream);
+  return MOE_ERR_INVALID_ARG;
 }
 
 int moe_get_device_status(void* ws, int32_t* status_out, void* stream) {

@@ -153,6 +153,11 @@ struct GemmOperands {
   // FWD1 / DW1: when set, the routed groups' x rows are gathered from a1 (x)
   // through these token ids (sorted_ids [Rr]) instead of read from a permuted copy
   const int32_t* gather_ids;
+  // expert parallelism (null: none): this rank's routed groups are its local
+  // experts; FWD1 / DX2 wait for the other ranks' rows, FWD2 / DX1 write the
+  // routed output rows into their sources' buffers (ep->rows) and signal them
+  const moe_ep_peers* ep;
+  int shared_first;  // the shared groups' tiles first (they need no exchange)
 };
 
 // Tensor map of a row-major bf16 matrix [rows, cols] (cols contiguous): box of
@@ -164,5 +169,18 @@ uint64_t wait_budget_ns();
 
 int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
                         const GemmOperands& ops, void* stream);
+
+// Expert parallelism (ep.cu); each returns a moe_status.
+bool ep_peers_ok(const moe_ep_peers* p, bool need_rows);
+int launch_ep_plan(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* counts_all,
+                   int32_t* counts_loc, int64_t cap, void* stream);
+int launch_ep_dispatch(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* idx,
+                       const int32_t* row_of, const int32_t* offsets, const void* x,
+                       void* stream);
+int launch_ep_zero_pads(const moe_dims& dm, const moe_ep_peers& pe, void* buf, void* stream);
+int launch_ep_wait(const moe_ep_peers& pe, int ctr, void* stream);
+int launch_combine_bwd_ep(const moe_dims& dm, const moe_ep_peers& pe, const void* dout,
+                          const void* y, const int32_t* row_of, const float* w,
+                          const int32_t* idx, const int32_t* offsets, float* dw, void* stream);
 
 }  // namespace moe

@@ -401,6 +401,128 @@ int moe_router_bwd_seqbal(const moe_dims* dims, const void* x, const float* wg,
 int moe_bias_update(const moe_dims* dims, const int32_t* counts, float gamma,
                     const float* bias_in, float* bias_out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Expert parallelism on the device.
+ * Passage: dots.llm1 Technical Report, §3.1 "Interleaved-1F1B based
+ * communication/computation overlap" (the all-to-all dispatch and combine of
+ * expert parallelism, overlapped with computation) and §3.2 (expert-aligned
+ * segments).
+ *
+ * W <= MOE_EP_MAX_WORLD ranks of one node; rank r owns the routed experts
+ * r E_l .. (r + 1) E_l - 1 (E_l = E / W) and every rank keeps the S shared
+ * experts for its own tokens.  Each rank routes and permutes its own T tokens
+ * over all E experts (moe_gate_topk, moe_permute_align with x_perm = NULL); an
+ * owner lays out what it receives expert-major: for each of its experts, the
+ * P-padded segments of ranks 0 .. W-1.
+ *
+ * Rows move by kernels that write straight into other ranks' buffers through
+ * peer pointers (device memory of the other GPUs mapped into this process, e.g.
+ * symmetric memory; a rank's own entries are its own buffers).  Every sending
+ * kernel ends with its last CTA adding 1 to a counter in each receiving rank's EP
+ * workspace; every receiver waits on the device, bounded by the library's wait
+ * budget, until its counter reaches W x (its step count).  No size or count
+ * comes to the host, so a whole step can be captured in a CUDA graph.
+ *
+ * Order of one training step on every rank (one stream):
+ *   moe_gate_topk, moe_permute_align (x_perm = NULL), an all-gather of every
+ *   rank's counts into counts_all [W, E] (e.g. NCCL), moe_ep_plan,
+ *   grouped_gemm_set_groups (local dims, counts_loc), moe_ep_zero_pads (the
+ *   receive buffer of x rows), moe_ep_dispatch, grouped_gemm_fwd_ep,
+ *   moe_ep_wait(MOE_EP_WAIT_Y), moe_combine_split;
+ *   moe_ep_zero_pads (the receive buffer of dY), moe_ep_combine_bwd,
+ *   grouped_gemm_bwd_dx_ep(MOE_GEMM2), grouped_gemm_bwd_dw (both), and only then
+ *   grouped_gemm_bwd_dx_ep(MOE_GEMM1), moe_ep_wait(MOE_EP_WAIT_DX),
+ *   moe_combine_split (topk_w = NULL) and the router backward.
+ * The data-gradient return comes last on purpose: a source starts writing its
+ * next step's rows into an owner's receive buffers only after every owner has
+ * returned its dX rows, and by then that owner has finished reading them.
+ * Every rank must run the same number of steps.  A receive buffer too small for
+ * the rows a step sends it (recv_cap) is reported as MOE_ERR_BAD_ROUTING in the
+ * EP workspace's status word and nothing is written into it.  A wait that runs
+ * out sets MOE_ERR_DEVICE_TIMEOUT (in the EP workspace for moe_ep_wait, in the
+ * layer workspace for the GEMMs) and the call returns without its rows.
+ * Requires P % 32 == 0, E % W == 0 and k <= 32.
+ * ------------------------------------------------------------------------- */
+#define MOE_EP_MAX_WORLD 8
+
+typedef struct moe_ep_peers {
+  int32_t rank;   /* this process's rank */
+  int32_t world;  /* W, 1 .. MOE_EP_MAX_WORLD */
+  int64_t rows_cap;                /* rows of each buffer in rows[] */
+  void* ep_ws[MOE_EP_MAX_WORLD];   /* every rank's EP workspace, as mapped here */
+  void* rows[MOE_EP_MAX_WORLD];    /* every rank's buffer this call writes rows into
+                                      (bf16 [rows_cap, d]); unused entries NULL */
+} moe_ep_peers;
+
+/* Which counter moe_ep_wait waits on. */
+enum { MOE_EP_WAIT_Y = 3,  /* every owner has written its Y rows into this rank's buffer */
+       MOE_EP_WAIT_DX = 5  /* every owner has written its dX rows into this rank's buffer */ };
+
+/* Bytes of a rank's EP workspace (counters, status word and the step's plan;
+ * host-side size, no counterpart on the pages).
+ * It must be zeroed once before the first step and be reachable from every
+ * rank; afterwards only the calls below touch it. */
+size_t moe_ep_workspace_size(const moe_dims* dims, int32_t world);
+
+/* The step's exchange plan from every rank's per-expert counts (Passage: §3.1
+ * and §3.2, as above).
+ *   dims        the layer's dims (all E experts, this rank's T tokens)
+ *   counts_all  [W, E] int32 (device): row s = rank s's counts from moe_permute_align
+ *   counts_loc  [E_l] int32 (device) out: rows of each local expert, all segments
+ *               padded to P (for grouped_gemm_set_groups on the local dims)
+ *   recv_cap    rows of every rank's receive buffers (the same on all ranks)
+ * Also advances this rank's step count.  peers->rows is not used. */
+int moe_ep_plan(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* counts_all,
+                int32_t* counts_loc, int64_t recv_cap, void* stream);
+
+/* Dispatch (Passage: §3.1, the all-to-all dispatch): x[t] to the owner of
+ * each of its picks, at its row in the owner's
+ * receive buffer (peers->rows[o], [recv_cap, d] bf16); then every owner's
+ * arrival counter is raised.  topk_idx, row_of, offsets as moe_permute_align
+ * wrote them for this rank; x [T, d] bf16. */
+int moe_ep_dispatch(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* topk_idx,
+                    const int32_t* row_of, const int32_t* offsets, const void* x, void* stream);
+
+/* Owner (Passage: §3.2, segments padded to a fixed block): zero the pad rows
+ * of every received segment of its receive buffer
+ * recv [recv_cap, d] bf16 (x rows before the forward, dY rows before the
+ * backward), as the plan lays them out. */
+int moe_ep_zero_pads(const moe_dims* dims, const moe_ep_peers* peers, void* recv, void* stream);
+
+/* Source: wait (bounded) until every owner has returned this step's rows
+ * (Passage: §3.1, the combine side of the all-to-all). */
+int moe_ep_wait(const moe_ep_peers* peers, int which, void* stream);
+
+/* moe_combine_bwd under expert parallelism (Passage: §Architecture "Mixture of
+ * Experts layer" and §3.1): dw [T, k] as there; each pick's dY
+ * row goes to its owner's receive buffer (peers->rows[o]), then every owner's
+ * arrival counter is raised.  Pad rows are zeroed by the owners
+ * (moe_ep_zero_pads).  y [Rr, d] = this rank's routed rows returned by the
+ * forward; topk_idx and offsets as for moe_ep_dispatch. */
+int moe_ep_combine_bwd(const moe_dims* dims, const moe_ep_peers* peers, const void* dout,
+                       const void* y, const int32_t* row_of, const float* topk_w,
+                       const int32_t* topk_idx, const int32_t* offsets, float* dw, void* stream);
+
+/* Passage: §3.1 (communication overlapped with computation) and §3.2.
+ * grouped_gemm_fwd on an owner (dims_loc: E = E_l local experts, rows_cap =
+ * recv_cap): the first GEMM starts with the shared experts' tiles and waits
+ * (bounded) for every source's rows before its first routed tile; the second
+ * GEMM writes each routed group's Y rows straight into the buffer of the rank
+ * they came from (peers->rows[s], [rows_cap, d]: the source's routed rows, in its
+ * permuted layout) instead of into y, then raises every source's counter.  The
+ * shared experts' rows land in y at rows Rr_loc + s T as usual. */
+int grouped_gemm_fwd_ep(const moe_dims* dims_loc, const void* ws, const moe_ep_peers* peers,
+                        const void* x_recv, const void* x, const void* w1, const void* w2,
+                        void* h, void* a1, void* y, void* stream);
+
+/* Passage: §3.1 and §3.2, as grouped_gemm_fwd_ep.
+ * grouped_gemm_bwd_dx on an owner: MOE_GEMM2 waits for every source's dY rows
+ * (shared tiles first); MOE_GEMM1 writes each routed group's dX rows into the
+ * buffer of the rank they came from (peers->rows[s]) and raises its counter. */
+int grouped_gemm_bwd_dx_ep(const moe_dims* dims_loc, const void* ws, const moe_ep_peers* peers,
+                           int which, const void* dy_recv, const void* dy_shared, const void* w,
+                           const void* a1, void* out, void* stream);
+
 /* Reads and clears the device status word of `ws` (synchronises `stream`).
  * Error reporting of this library: the pages have no counterpart.
  * *status_out receives MOE_OK or the first device error recorded. */

@@ -139,3 +139,41 @@ def sample_tokens(oidx, cand, n, seed, per_expert=16):
     need = max(0, n - len(set(pick)))
     pick.extend(rng.choice(rest, min(need, len(rest)), replace=False).tolist())
     return np.unique(np.array(pick, dtype=np.int64))
+
+
+def ep_plan_reference(counts_all, rank, P, cap):
+    """The exchange plan of expert parallelism written out from its definition, for
+    checking the device plan (moe_ep_plan) and the cross-rank agreement of offsets.
+    counts_all [W, E]: rank s's tokens per expert.  Rank o owns experts o E_l ..
+    (o + 1) E_l - 1 and lays out what it receives expert-major: for each local expert,
+    the P-padded segments of ranks 0 .. W - 1.  Returns a dict of numpy int arrays:
+    send_dst [E] (this rank's segment of expert g starts at that row of its owner's
+    buffer), recv_row / recv_cnt / recv_real / src_off [W, E_l] (this rank as owner: where
+    source s's segment of local expert e lands, its padded and real rows, and where it
+    starts in source s's permuted rows), counts_loc [E_l], over [W]."""
+    c = np.asarray(counts_all, dtype=np.int64)
+    W, E = c.shape
+    El = E // W
+    pad = (c + P - 1) // P * P
+    out = {k: np.zeros((W, El), np.int64) for k in ("recv_row", "recv_cnt", "recv_real",
+                                                       "src_off")}
+    send_dst = np.zeros(E, np.int64)
+    over = np.zeros(W, np.int64)
+    for o in range(W):
+        row = 0
+        for e in range(El):
+            g = o * El + e
+            for s in range(W):
+                if s == rank:
+                    send_dst[g] = row
+                if o == rank:
+                    out["recv_row"][s, e] = row
+                    out["recv_cnt"][s, e] = pad[s, g]
+                    out["recv_real"][s, e] = c[s, g]
+                    out["src_off"][s, e] = pad[s, :g].sum()
+                row += pad[s, g]
+        over[o] = row > cap
+    out["send_dst"] = send_dst
+    out["counts_loc"] = pad[:, rank * El:(rank + 1) * El].sum(axis=0)
+    out["over"] = over
+    return out

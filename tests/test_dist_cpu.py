@@ -143,57 +143,65 @@ def test_data_parallel_loads_bias_step_and_gradient_sum():
 
 
 def _ep_worker(rank, world, port, q):
-    """Expert-parallel exchange (grouped_gemm_fp32_b200.ep) on gloo with CPU tensors:
-    counts all-to-all, dispatch of padded segments to their owners (expert-major), and
-    the return of the owners' rows into each source's permuted layout."""
+    """Expert parallelism's host side on gloo with CPU tensors: the all-gather of every
+    rank's per-expert counts (ep.gather_counts, the only collective the exchange needs)
+    and the plan every rank derives from them: what a source writes where must be where
+    its owner expects it, for every pair of ranks, including ranks that send an owner
+    nothing."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
     sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
     import torch
     import torch.distributed as dist
-    from grouped_gemm_fp32_b200 import ep
+    from common import ep_plan_reference
+    from grouped_gemm_fp32_b200 import MoeDims, ep
     dist.init_process_group("gloo", rank=rank, world_size=world)
-    E, P, d = 6 * world, 8, 4
+    E, P, k, T = 4 * world, 32, 2, 40
     El = E // world
+    eb = ep.EPBuffers(MoeDims.of(T, 64, E, k, 1, 64, P), rank, world, device="cpu")
     rng = np.random.default_rng(100 + rank)
     counts = rng.integers(0, 20, size=E).astype(np.int32)
-    counts[rank] = 0                                   # some empty segments
-    ct = torch.from_numpy(counts)
-    counts_in = torch.empty_like(ct)
-    dist.all_to_all_single(counts_in, ct)
-    plan = ep.EPPlan(counts, counts_in.numpy(), rank, world, P)
-    # permuted rows: row i of expert g's segment holds (rank, g, i), pad rows -1
-    x_perm = torch.full((plan.send_rows, d), -1.0)
-    for o, e, a, n in plan.to_owner:
-        g = o * El + e
-        for i in range(counts[g]):
-            x_perm[a + i] = torch.tensor([rank, g, i, 0.0])
-    x_recv = torch.full((plan.recv_rows, d), -7.0)
-    ep.exchange(*ep.dispatch_lists(plan, x_perm, x_recv), rank)
-    ok_dispatch = True
-    for s, e, a, n in plan.from_source:
-        c = int(counts_in.view(world, El)[s, e])
-        for i in range(n):
-            want = [s, rank * El + e, i, 0.0] if i < c else [-1.0] * 4
-            ok_dispatch &= x_recv[a + i].tolist() == want
-    # the owner's "expert" marks each row; the source must get its rows back in place
-    y_loc = x_recv.clone()
-    y_loc[:, 3] = 100.0 + rank
-    y_full = torch.full((plan.send_rows, d), -9.0)
-    ep.exchange(*ep.return_lists(plan, y_loc, y_full), rank)
-    ok_return = True
-    for o, e, a, n in plan.to_owner:
-        g = o * El + e
-        for i in range(n):
-            want = ([rank, g, i] if i < counts[g] else [-1.0] * 3) + [100.0 + o]
-            ok_return &= y_full[a + i].tolist() == want
+    counts[rank] = 0                             # an empty segment on every rank
+    if rank == 0 and world > 2:
+        counts[2 * El:3 * El] = 0                # rank 0 sends owner 2 nothing at all
+    eb.full.counts.copy_(torch.from_numpy(counts))
+    ep.gather_counts(eb)
+    table = eb.counts_all.numpy().copy()
+    cap = eb.cap
+    plans = [ep_plan_reference(table, r, P, cap) for r in range(world)]
+    mine = plans[rank]
+    ok = bool(np.array_equal(table[rank], counts))
+    # the table is the same on every rank
+    allt = [torch.zeros_like(eb.counts_all) for _ in range(world)]
+    dist.all_gather(allt, eb.counts_all)
+    ok &= all(torch.equal(t, eb.counts_all) for t in allt)
+    pad = (table + P - 1) // P * P
+    for o in range(world):
+        own = plans[o]
+        # source `rank`'s segment of each expert of owner o lands where o expects it
+        for e in range(El):
+            g = o * El + e
+            ok &= int(mine["send_dst"][g]) == int(own["recv_row"][rank, e])
+            ok &= int(own["recv_cnt"][rank, e]) == int(pad[rank, g])
+            ok &= int(own["src_off"][rank, e]) == int(pad[rank, :g].sum())
+        # owner o's received segments tile its rows [0, total) in expert-major order
+        spans = sorted((int(own["recv_row"][s, e]), int(own["recv_cnt"][s, e]))
+                       for e in range(El) for s in range(world))
+        pos = 0
+        for start, n in spans:
+            ok &= start == pos
+            pos += n
+        ok &= pos == int(own["counts_loc"].sum())
+    zero_from_peer = any(pad[s, o * El:(o + 1) * El].sum() == 0
+                         for s in range(world) for o in range(world) if s != o)
     dist.barrier()
     dist.destroy_process_group()
-    q.put((rank, ok_dispatch, ok_return, plan.recv_rows, int(plan.local_counts.sum())))
+    q.put((rank, ok, zero_from_peer, [int(v) for v in mine["over"]]))
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_expert_parallel_exchange_moves_segments_both_ways(world):
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_expert_parallel_plan_agrees_across_ranks(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -204,40 +212,18 @@ def test_expert_parallel_exchange_moves_segments_both_ways(world):
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, ok_dispatch, ok_return, recv_rows, local_rows in out:
-        assert ok_dispatch, rank
-        assert ok_return, rank
-        assert recv_rows == local_rows
+    for rank, ok, zero_from_peer, over in out:
+        assert ok, rank
+        assert over == [0] * world
+    if world > 2:
+        assert any(z for _, _, z, _ in out)  # some rank receives zero rows from a peer
 
 
-def _cap_worker(rank, world, port, q):
-    """ep.check_capacity on gloo: one rank over its receive capacity makes every rank raise."""
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
-                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
-    sys.path.insert(0, ROOT)
-    import torch.distributed as dist
-    from grouped_gemm_fp32_b200 import ep
-    dist.init_process_group("gloo", rank=rank, world_size=world)
-    ep.check_capacity(40 + rank, 100)          # everyone within capacity: no error
-    raised = False
-    try:
-        ep.check_capacity(120 if rank == 1 else 10, 100)
-    except RuntimeError:
-        raised = True
-    dist.barrier()
-    dist.destroy_process_group()
-    q.put((rank, raised))
-
-
-def test_expert_parallel_capacity_overflow_raises_on_every_rank():
-    ctx = mp.get_context("spawn")
-    q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_cap_worker, args=(r, 3, port, q)) for r in range(3)]
-    for p in procs:
-        p.start()
-    out = [q.get(timeout=240) for _ in procs]
-    for p in procs:
-        p.join(timeout=60)
-        assert p.exitcode == 0
-    assert all(raised for _, raised in out)
+def test_expert_parallel_plan_flags_an_owner_over_capacity():
+    # rank 1 is sent more rows than the receive buffers hold: every rank's plan says so
+    # (the device kernels then write nothing into that owner's buffers)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from common import ep_plan_reference
+    table = np.array([[100, 0, 300, 40], [5, 0, 200, 1]])
+    for r in range(2):
+        assert ep_plan_reference(table, r, 32, 600)["over"].tolist() == [0, 1]

@@ -61,3 +61,49 @@ def test_bounded_waits_report_timeout_and_keep_context():
     assert "gemm status -4" in p.stdout, p.stdout
     assert "gate status -4" in p.stdout, p.stdout
     assert "context ok True" in p.stdout, p.stdout
+
+
+CHILD_EP = r'''
+import sys
+sys.path.insert(0, ROOT)
+import torch
+import grouped_gemm_fp32_b200 as moe
+from grouped_gemm_fp32_b200 import ep
+import synth
+# one rank whose exchange partners never deliver: the owner's GEMM waits for rows that
+# no dispatch sends, the source waits for Y rows that no owner returns
+dims = moe.MoeDims.of(256, 128, 8, 2, 1, 64, 64)
+eb = ep.EPBuffers(dims, 0, 1, train=False)
+ep.connect(eb)
+eb.counts_all.fill_(64)          # as if every expert had 64 tokens
+ep.plan(eb)
+bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).cuda()
+x = bf(synth.normal_bf16(3, 1, (256, 128), 1.0))
+w1 = bf(synth.normal_bf16(3, 4, (9, 128, 128), 0.05))
+w2 = bf(synth.normal_bf16(3, 5, (9, 128, 64), 0.05))
+ep.experts_forward(eb, x, w1, w2)          # no dispatch ran: its first routed tile waits
+torch.cuda.synchronize()
+print("gemm status", moe.moe_get_device_status(eb.loc.ws))
+# the owner above returned (garbage) rows, so raise the step count once more and wait
+# for an owner that never comes
+ep.plan(eb)
+moe.moe_ep_wait(eb.peers["ws"], moe.MOE_EP_WAIT_Y)
+torch.cuda.synchronize()
+print("wait status", moe.moe_get_device_status(eb.ep_ws))
+z = torch.arange(1000, device="cuda", dtype=torch.float32).sum().item()
+print("context ok", z == 499500.0)
+'''
+
+
+@pytest.mark.gpu
+def test_expert_parallel_waits_report_timeout_and_keep_context():
+    """Bounded waits of the expert-parallel exchange: rows that never arrive give
+    MOE_ERR_DEVICE_TIMEOUT (in the GEMM's workspace, and in the EP workspace for the
+    source's wait) within a 20 ms budget, and the context stays usable."""
+    env = dict(os.environ, MOE_WAIT_BUDGET_NS="20000000")
+    p = subprocess.run([sys.executable, "-c", f"ROOT = {ROOT!r}\n" + CHILD_EP], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stdout + p.stderr
+    assert "gemm status -4" in p.stdout, p.stdout
+    assert "wait status -4" in p.stdout, p.stdout
+    assert "context ok True" in p.stdout, p.stdout
