@@ -10,7 +10,10 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIB_DEBUG=1 loads the debug build (libmoe_debug.so: device-side checks of the
+# group table and tile coordinates, MOE_ERR_BAD_ROUTING instead of a bad access)
+_LIB_PATH = os.path.join(_HERE, "libmoe_debug.so" if os.environ.get("MOE_LIB_DEBUG") == "1"
+                         else "libmoe.so")
 _lib = None
 
 MOE_GEMM1, MOE_GEMM2 = 1, 2

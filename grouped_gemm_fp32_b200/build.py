@@ -1,4 +1,7 @@
-"""Build ``libmoe.so`` (the C-ABI CUDA library) in-tree with nvcc for sm_100a.
+"""Build ``libmoe.so`` (the C-ABI CUDA library) in-tree with nvcc for sm_100a, and
+``libmoe_debug.so``, the same sources with MOE_DEBUG=1 (device-side checks of the
+group table and tile coordinates that report MOE_ERR_BAD_ROUTING instead of
+following a bad entry; loaded instead of libmoe.so when MOE_LIB_DEBUG=1).
 
     python -m grouped_gemm_fp32_b200.build [--force]
 """
@@ -12,6 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe.so")
+LIB_DEBUG = os.path.join(HERE, "libmoe_debug.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
@@ -31,10 +35,10 @@ def deps():
         [os.path.join(INCLUDE, "moe.h"), os.path.abspath(__file__)]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in deps())
 
 
@@ -45,15 +49,22 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *sources()]
+def _build_one(lib: str, extra, force: bool, verbose: bool):
+    if not force and not stale(lib):
+        return
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Both libraries (the debug one unless ``debug`` is False); returns libmoe.so's path."""
+    _build_one(LIB, [], force, verbose)
+    if debug:
+        _build_one(LIB_DEBUG, ["-DMOE_DEBUG=1"], force, verbose)
     return LIB
 
 

@@ -91,6 +91,9 @@ struct GemmArgs {
   int gather_T;               // rows of the gathered tensor x
   int shared_first;           // FWD / DX: the shared groups' tiles come first
   EpGemm ep;                  // expert parallelism: rows to wait for, outputs to return
+  // extents for the checks of the debug build: rows of the grouped row space (Rt), of
+  // the routed A / B sources (Rr) and of x (T)
+  int64_t rows_total, rows_routed, rows_x;
 };
 
 // Tensor maps of every source rank's rows (expert parallelism: FWD2 / DX1 write
@@ -169,6 +172,12 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     const int nt = local / a.MT, mt = local - nt * a.MT;
     t.m0 = mt * PM;
     t.n0 = nt * 256;
+    if (MOE_DEBUG && (t.g < 0 || t.g >= a.G)) {
+      t.nkb = 0;
+      t.nw = 256;
+      t.half = 0;
+      return t;
+    }
     t.nkb = (load_group(a, t.g).rows_pad + BK - 1) / BK;  // the tail block reads zeros past the end
     t.nw = (a.n_out - t.n0 > 128) ? 256 : 128;
     t.half = 0;
@@ -203,6 +212,29 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const GemmArgs& a) {
     t.half = a.half_ok && load_group(a, lo).rows_pad - t.m0 <= BM;
   }
   return t;
+}
+
+// Debug build: the tile's group id and its record must describe rows inside the
+// tensors the kernel reads and writes; otherwise MOE_ERR_BAD_ROUTING is recorded
+// and every role skips the tile (all roles decide alike, from the same record).
+template <int MODE>
+__device__ __forceinline__ bool tile_ok(const GemmArgs& a, const TileInfo& t) {
+  if constexpr (!MOE_DEBUG) {
+    return true;
+  } else {
+    bool ok = t.g >= 0 && t.g < a.G;
+    if (ok) {
+      const GroupRec gr = load_group(a, t.g);
+      const bool shared = t.g >= a.E;
+      ok = gr.rows_pad >= 0 && gr.out_row >= 0 && gr.a_row >= 0 &&
+           (int64_t)gr.out_row + gr.rows_pad <= a.rows_total &&
+           (int64_t)gr.a_row + gr.rows_pad <= (shared ? a.rows_x : a.rows_routed);
+      if (MODE == MODE_DW2 || MODE == MODE_DW1) ok = ok && t.m0 < a.m_out && t.n0 < a.n_out;
+      else ok = ok && t.n0 < a.n_out && t.m0 < gr.rows_pad;
+    }
+    if (!ok) atomicCAS(a.status, 0, MOE_ERR_BAD_ROUTING);
+    return ok;
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -371,6 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool rows_in = args.ep.wait_ctr == 0;  // the routed rows of other ranks have arrived
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<MODE>(tile, args);
+        if (!tile_ok<MODE>(args, t)) continue;
         const GroupRec gr = load_group(args, t.g);
         const int roff = (int)rank * (t.half ? BM / 2 : BM);  // this CTA's rows of A
         const bool shared = t.g >= args.E;
@@ -534,10 +567,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (leader && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
+      int it = 0;  // tiles processed (the debug build skips invalid ones)
       bool ok = true;
-      for (int tile = pair; ok && tile < total_tiles; tile += npairs, ++it) {
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<MODE>(tile, args);
+        if (!tile_ok<MODE>(args, t)) continue;
         const int acc = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
         if (!mbar_wait(&ctl->tempty[acc], (use & 1u) ^ 1u, abort_flag, args.status,
@@ -575,6 +609,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         umma_commit_pair(&ctl->tfull[acc], 0x3);  // both CTAs' epilogues may read
+        ++it;
       }
       // Drain: every MMA issued completes before tensor memory is freed.
       umma_commit_pair(&ctl->drain, 0x1);
@@ -600,9 +635,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(tempty_leader[acc]);
     };
-    int it = 0;
+    int it = 0;  // tiles processed
     for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
       const TileInfo t = decode_tile<MODE>(tile, args);
+      if (!tile_ok<MODE>(args, t)) {
+        --it;
+        continue;
+      }
       const int acc = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (!mbar_wait(&ctl->tfull[acc], use & 1u, abort_flag, args.status, MOE_ERR_DEVICE_TIMEOUT,
@@ -984,6 +1023,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   a.accumulate = ops.accumulate;
   a.budget_ns = wait_budget_ns();
   a.shared_first = ops.shared_first;
+  a.rows_total = Rt;
+  a.rows_routed = Rr;
+  a.rows_x = T;
 
   // expert parallelism: rows to wait for (FWD1 / DX2), outputs to return (FWD2 / DX1)
   EpMaps epm;

@@ -9,6 +9,14 @@
 
 #include "moe.h"  // include/ is on the include path
 
+// MOE_DEBUG=1 (libmoe_debug.so): kernels that take the group table, the tile
+// prefix or row indices from memory a caller could have overwritten validate
+// them against the tensor extents before using them; a bad entry records
+// MOE_ERR_BAD_ROUTING in the status word and its work is skipped.  Nothing traps.
+#ifndef MOE_DEBUG
+#define MOE_DEBUG 0
+#endif
+
 namespace moe {
 
 // Records the error of a failing CUDA call for moe_last_cuda_error(); true on success.

@@ -247,9 +247,14 @@ __global__ void copy_rows_kernel_bigk(const uint4* __restrict__ x, int64_t T, in
 // Zero the pad rows [off_e + c_e, off_e + roundup(c_e, P)) of every routed
 // segment (of a bf16 [Rr, row_vec * 8] matrix).  grid.x = E.
 __global__ void zero_pad_rows_kernel(const GroupRec* __restrict__ groups, int row_vec,
-                                     uint4* __restrict__ m) {
+                                     uint4* __restrict__ m, int64_t Rr, int* status) {
   const GroupRec g = groups[blockIdx.x];
   const int64_t r0 = (int64_t)g.out_row + g.rows, r1 = (int64_t)g.out_row + g.rows_pad;
+  if (MOE_DEBUG && (g.out_row < 0 || g.rows < 0 || r0 > r1 || r1 > Rr)) {
+    // debug build: a group record outside the routed rows is reported, not followed
+    if (threadIdx.x == 0) atomicCAS(status, 0, MOE_ERR_BAD_ROUTING);
+    return;
+  }
   const int64_t n = (r1 - r0) * row_vec;
   const uint4 z = make_uint4(0, 0, 0, 0);
   // blockIdx.y splits one group's pad rows across several CTAs
@@ -310,7 +315,8 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
                                                          row_vec, dm.k, row_of,
                                                          reinterpret_cast<uint4*>(x_perm), status);
   zero_pad_rows_kernel<<<dim3(dm.E, kPadSplit), 256, 0, st>>>(
-      reinterpret_cast<const GroupRec*>(wsb + L.groups), row_vec, reinterpret_cast<uint4*>(x_perm));
+      reinterpret_cast<const GroupRec*>(wsb + L.groups), row_vec, reinterpret_cast<uint4*>(x_perm),
+      Rr, status);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -332,7 +338,8 @@ int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, 
   const WsLayout L = ws_layout(dm);
   const uint8_t* wsb = reinterpret_cast<const uint8_t*>(ws);
   zero_pad_rows_kernel<<<dim3(dm.E, kPadSplit), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const GroupRec*>(wsb + L.groups), cols / 8, reinterpret_cast<uint4*>(m));
+      reinterpret_cast<const GroupRec*>(wsb + L.groups), cols / 8, reinterpret_cast<uint4*>(m),
+      rows_routed(dm), reinterpret_cast<int*>(const_cast<uint8_t*>(wsb)));
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
