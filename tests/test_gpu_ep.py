@@ -223,3 +223,58 @@ def test_combine_split_is_the_combine_bit_for_bit():
         moe.moe_combine_split(dims, y[:Rr], shared, row_of, wt, b)
         torch.cuda.synchronize()
         assert torch.equal(a, b)
+
+
+def test_owner_over_capacity_is_reported_without_writes_or_hangs():
+    """Receive buffers smaller than what a step sends an owner: every rank's plan flags
+    that owner (MOE_ERR_BAD_ROUTING in the EP workspace), no sender writes into it, its
+    group table is refused, and the step still completes (every arrival counter moves, so
+    no wait runs out).  Every buffer other ranks write into sits between guard bands that
+    must stay intact."""
+    from test_gpu_guard import Guarded
+    W, E, k, T, P = 2, 8, 2, 256, 64
+    wl = synth.Workload("epcap", synth.Dims(T=T, d=128, E=E, k=k, S=1, I=64, P=P), seed=31,
+                        w1_std=0.05, w2_std=0.05, wg_std=0.05, backward=True)
+    base, xs, douts = _rank_inputs(wl, W)
+    base["bias"][:E // W] = 1.0           # every token picks owner 0's experts
+    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).cuda()
+    w1, w2 = bf(base["w1"]), bf(base["w2"])
+    wg, bias = torch.from_numpy(base["wg"]).cuda(), torch.from_numpy(base["bias"]).cuda()
+    x = [bf(a) for a in xs]
+    dout = [bf(a) for a in douts]
+    dims = dims_of(wl)
+    El = E // W
+    g = Guarded()
+    alloc = lambda shape, dtype: g.wrap(torch.zeros(shape, dtype=dtype, device="cuda"))
+    cap = 3 * P                           # far below the 2 * T * k rows owner 0 is sent
+    ebs = [ep.EPBuffers(dims, r, W, train=True, recv_rows_cap=cap, alloc=alloc)
+           for r in range(W)]
+    ep.connect_emulated(ebs)
+    wl1 = [torch.cat([w1[r * El:(r + 1) * El], w1[E:]]).contiguous() for r in range(W)]
+    wl2 = [torch.cat([w2[r * El:(r + 1) * El], w2[E:]]).contiguous() for r in range(W)]
+    for r, eb in enumerate(ebs):
+        ep.route(eb, x[r], wg, bias)
+    table = torch.stack([eb.full.counts for eb in ebs])
+    for eb in ebs:
+        eb.counts_all.copy_(table)
+        ep.plan(eb)
+    for r, eb in enumerate(ebs):
+        ep.dispatch(eb, x[r])
+    for r, eb in enumerate(ebs):
+        ep.experts_forward(eb, x[r], wl1[r], wl2[r])
+    for eb in ebs:
+        ep.combine(eb)
+    for r, eb in enumerate(ebs):
+        ep.backward_dispatch(eb, dout[r])
+    for r, eb in enumerate(ebs):
+        ep.experts_backward(eb, x[r], dout[r], wl1[r], wl2[r])
+    for r, eb in enumerate(ebs):
+        ep.unpermute_and_router(eb, x[r], wg)
+    torch.cuda.synchronize()
+    for eb in ebs:
+        assert _device_plan(eb)["over"].tolist() == [1, 0]
+    statuses = [moe.moe_get_device_status(eb.ep_ws) for eb in ebs]
+    assert statuses == [-5, -5], statuses          # the plan's report, on both ranks
+    assert moe.moe_get_device_status(ebs[0].loc.ws) == -5   # owner 0's group table refused
+    assert moe.moe_get_device_status(ebs[1].loc.ws) == 0
+    assert g.intact(), "a write landed outside a receive or return buffer"
