@@ -317,7 +317,7 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ggemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                 const __grid_constant__ CUtensorMap tmC /* DX2: saved [G | U] */,
+                 const __grid_constant__ CUtensorMap tmC /* unused (the slot of a third operand) */,
                  const __grid_constant__ CUtensorMap tmO0 /* output (FWD1: H) */,
                  const __grid_constant__ CUtensorMap tmO1 /* FWD1: saved A1 */,
                  const __grid_constant__ CUtensorMap tmA0h /* half tiles: 64-row A boxes */,
@@ -360,7 +360,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
-    if (MODE == MODE_DX2) tma_prefetch_desc(&tmC);
     if (args.staged) {
       tma_prefetch_desc(&tmO0);
       if (MODE == MODE_FWD1 && args.out2 != nullptr) tma_prefetch_desc(&tmO1);
@@ -484,17 +483,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                              t.g * args.b_group_rows + t.n0 + (int)rank * 128);
           } else if constexpr (MODE == MODE_DX2 || MODE == MODE_DX1) {
             if constexpr (MODE == MODE_DX2) {
-              // the epilogue of this tile reads the saved [G | U] of its rows: start
-              // pulling them into L2 now, a whole K loop ahead
-              if (kb == 0) {
-                const int y = gr.out_row + t.m0 + roff;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                  if (t.n0 + c * 64 < args.I) {
-                    tma_prefetch_l2_2d(&tmC, t.n0 + c * 64, y);
-                    tma_prefetch_l2_2d(&tmC, args.I + t.n0 + c * 64, y);
-                  }
-              }
               tma_load_2d_pair(a_dst,
                                t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0),
                                fb, k0, (shared ? 0 : gr.a_row) + t.m0 + roff);
@@ -1050,7 +1038,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
     }
   }
 
-  CUtensorMap m0{}, m1{}, n0{}, n1{}, c0{}, o0{}, o1{};
+  CUtensorMap m0{}, m1{}, n0{}, n1{}, o0{}, o1{};
   CUtensorMap mh0{}, mh1{}, nh{};  // half tiles: 64-row boxes of A (and of B in FWD1)
   bool ok = true;
   // a dummy map stands in for unused slots (never read by the kernel)
@@ -1129,7 +1117,6 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (dm.S > 0 && T > 0) ok &= make_map_bf16(&m1, ops.a1, T, d, BM); else same(m1, m0);
       ok &= make_map_bf16(&n0, ops.b0, (int64_t)G * d, I, 64);
       same(n1, n0);
-      ok &= make_map_bf16(&c0, ops.aux, Rt, 2 * I, BM);  // saved [G | U], prefetched into L2
       a.half_ok = 1;
       a.idesc_h = idesc_bf16_f32(BM, 256, false, true);
       a.idesc_h_narrow = idesc_bf16_f32(BM, 128, false, true);
@@ -1139,7 +1126,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, 2 * I, 2, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DX2>(m0, m1, n0, n1, c0, o0, o0, mh0, mh1, nh, epm, a, st);
+      return launch_mode<MODE_DX2>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, epm, a, st);
     }
     case MODE_DX1: {
       a.K = 2 * I;
