@@ -892,7 +892,7 @@ def run_ep(args):
                            "step": "CUDA graph replay: gate, routing tables, NCCL all-gather "
                                    "of the counts, device plan, rows written into the owners' "
                                    "buffers, owners' grouped GEMMs (shared tiles first, "
-                                   "bounded waits for the rows), outputs written back into "
+                                   "a bounded wait per expert for its segments), outputs written back into "
                                    "the sources' buffers, combine; backward likewise; no "
                                    "host sync"},
                 "clocks": clocks}

@@ -115,7 +115,7 @@ def load():
         "moe_get_device_status": (i32, [vp, vp, vp]),
         "moe_ep_workspace_size": (sz, [D, i32]),
         "moe_ep_plan": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, i64, vp]),
-        "moe_ep_dispatch": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, vp, vp, vp]),
+        "moe_ep_dispatch": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, vp, vp]),
         "moe_ep_zero_pads": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp]),
         "moe_ep_wait": (i32, [ctypes.POINTER(MoeEpPeers), i32, vp]),
         "moe_ep_combine_bwd": (i32, [D, ctypes.POINTER(MoeEpPeers), vp, vp, vp, vp, vp, vp, vp,
@@ -302,8 +302,8 @@ def moe_ep_plan(dims, peers, counts_all, counts_loc, recv_cap, stream=None):
                            _p(counts_loc), int(recv_cap), _s(stream)), "moe_ep_plan")
 
 
-def moe_ep_dispatch(dims, peers, topk_idx, row_of, offsets, x, stream=None):
-    _ck(load().moe_ep_dispatch(ctypes.byref(dims), ctypes.byref(peers), _p(topk_idx), _p(row_of),
+def moe_ep_dispatch(dims, peers, sorted_ids, offsets, x, stream=None):
+    _ck(load().moe_ep_dispatch(ctypes.byref(dims), ctypes.byref(peers), _p(sorted_ids),
                                _p(offsets), _p(x), _s(stream)), "moe_ep_dispatch")
 
 

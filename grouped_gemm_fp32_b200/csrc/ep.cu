@@ -1,7 +1,7 @@
 // ep.cu -- expert parallelism on the device: the step's exchange plan built from
 // the ranks' per-expert counts, the dispatch of x rows straight into the
-// owners' receive buffers, the owners' pad rows, and the bounded wait on an
-// arrival counter.
+// owners' receive buffers (segment by segment, each expert's arrival signalled on
+// its own), the owners' pad rows, and the bounded wait on an arrival counter.
 //
 // Passage: dots.llm1 Technical Report, §3.1 "Interleaved-1F1B based
 // communication/computation overlap" (all-to-all dispatch and combine of expert
@@ -81,6 +81,26 @@ __global__ void __launch_bounds__(256)
     for (int s = 0; s < W; ++s) n += s_pad[s][rank * El + e];
     counts_loc[e] = n;
   }
+  // this rank as a source: its rows per expert, and its dispatch work items of
+  // kEpDispatchRows rows (one at least per expert, so that every owner hears about
+  // every expert every step), counted in the order q = e W + o
+  int32_t* own_cnt = reinterpret_cast<int32_t*>(wsb + L.own_cnt);
+  int32_t* done = reinterpret_cast<int32_t*>(wsb + L.done);
+  int32_t* chunk_pre = reinterpret_cast<int32_t*>(wsb + L.chunk_pre);
+  for (int g = tid; g < E; g += blockDim.x) {
+    own_cnt[g] = counts_all[rank * E + g];
+    done[g] = 0;
+  }
+  if (tid == 0) {
+    int32_t acc = 0;
+    for (int q = 0; q < E; ++q) {
+      chunk_pre[q] = acc;
+      const int g = (q % W) * El + q / W;
+      const int c = counts_all[rank * E + g];
+      acc += c > 0 ? (c + kEpDispatchRows - 1) / kEpDispatchRows : 1;
+    }
+    chunk_pre[E] = acc;
+  }
   __syncthreads();
   if (tid == 0) {
     if (s_bad) atomicCAS(ws + EP_STATUS, 0, MOE_ERR_BAD_ROUTING);
@@ -88,53 +108,60 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// One warp per token: x[t] goes to the owner of each of its k picks, at the row
-// the plan gives its segment, written through the owner's peer pointer (each
-// lane holds four 16-byte pieces of the row at a time and writes them to every
-// destination).  The last CTA then adds 1 to EP_CTR_ROWS of every rank.
-template <int KMAX>
-__global__ void ep_dispatch_kernel(const uint4* __restrict__ x, int64_t T, int row_vec, int k,
-                                   const int32_t* __restrict__ idx,
-                                   const int32_t* __restrict__ row_of,
-                                   const int32_t* __restrict__ offsets, int64_t Rr, int* ws,
-                                   EpLayout L, EpPtrs rows, EpPtrs peer_ws, int W, int El) {
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+// Dispatch, segment by segment: work item i of expert g copies rows
+// [16 i, 16 i + 16) of this rank's segment of g (the tokens sorted_ids lists, in
+// order) into the owner's receive buffer at the row the plan gives, through the
+// owner's peer pointer, two rows a warp.  Items run in the order q = e W + o, so
+// every owner receives its local experts' segments in expert order.  The CTA that
+// finishes an expert's last item raises that expert's arrival counter at its owner,
+// so the owner's grouped GEMM can start on the expert before later ones arrive.
+__global__ void __launch_bounds__(256)
+    ep_dispatch_kernel(const uint4* __restrict__ x, int64_t T, int row_vec,
+                       const int32_t* __restrict__ sorted_ids,
+                       const int32_t* __restrict__ offsets, int* ws, EpLayout L, EpPtrs rows,
+                       EpPtrs peer_ws, int W, int El) {
   const int E = W * El;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint8_t* wsb = reinterpret_cast<const uint8_t*>(ws);
   const int32_t* send_dst = reinterpret_cast<const int32_t*>(wsb + L.send_dst);
   const int32_t* over = reinterpret_cast<const int32_t*>(wsb + L.over);
-  if (t < T) {
-    uint4* dst[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      dst[j] = nullptr;
-      if (j < k) {
-        const int g = idx[t * k + j];
-        const int64_t r = row_of[t * k + j];
-        // a pick without a row, or an owner whose buffers are too small (the plan
-        // reported it): nothing written
-        if (g >= 0 && g < E && r >= 0 && r < Rr && !over[g / El])
-          dst[j] = reinterpret_cast<uint4*>(rows.p[g / El]) +
-                   ((int64_t)send_dst[g] + (r - offsets[g])) * row_vec;
+  const int32_t* own_cnt = reinterpret_cast<const int32_t*>(wsb + L.own_cnt);
+  const int32_t* chunk_pre = reinterpret_cast<const int32_t*>(wsb + L.chunk_pre);
+  int32_t* done = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + L.done);
+  const int arrive_word = (int)(L.arrive / sizeof(int32_t));
+  const int total = chunk_pre[E];
+  for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    int lo = 0, hi = E - 1;  // largest q with chunk_pre[q] <= item
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (chunk_pre[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    const int q = lo, e = q / W, o = q - e * W, g = o * El + e;
+    const int c = own_cnt[g];
+    // an owner whose buffers are too small (the plan reported it) gets no rows
+    if (!over[o]) {
+      for (int rr = warp; rr < kEpDispatchRows; rr += blockDim.x >> 5) {
+        const int row = (item - chunk_pre[q]) * kEpDispatchRows + rr;
+        if (row >= c) break;
+        const int tok = sorted_ids[offsets[g] + row];
+        if (tok < 0 || tok >= T) continue;  // a routing the permutation refused
+        const uint4* src = x + (int64_t)tok * row_vec;
+        uint4* dst =
+            reinterpret_cast<uint4*>(rows.p[o]) + ((int64_t)send_dst[g] + row) * row_vec;
+        for (int cc = lane; cc < row_vec; cc += 32) dst[cc] = src[cc];
       }
     }
-    const uint4* src = x + t * row_vec;
-    for (int c = lane; c < row_vec; c += 128) {
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (c + 32 * u < row_vec) v[u] = src[c + 32 * u];
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (dst[j] == nullptr) continue;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (c + 32 * u < row_vec) dst[j][c + 32 * u] = v[u];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence_system();  // this CTA's rows before its count
+      const int nch = chunk_pre[q + 1] - chunk_pre[q];
+      if (atomicAdd(done + g, 1) + 1 == nch) {
+        __threadfence_system();  // every item of the segment counted: release them all
+        atomicAdd_system(reinterpret_cast<int*>(peer_ws.p[o]) + arrive_word + e, 1);
       }
     }
+    __syncthreads();
   }
-  ep_signal_last_cta(ws + EP_DONE_ROWS, peer_ws, W, EP_CTR_ROWS);
 }
 
 // Owner: zero the pad rows of every received segment of a [cap, row_vec * 8]
@@ -187,25 +214,22 @@ int launch_ep_plan(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* co
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_ep_dispatch(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* idx,
-                       const int32_t* row_of, const int32_t* offsets, const void* x,
-                       void* stream) {
+int launch_ep_dispatch(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* sorted_ids,
+                       const int32_t* offsets, const void* x, void* stream) {
   const EpLayout L = ep_layout(dm.E, pe.world);
-  const int warps = 8;
-  // at least one CTA, so that the arrival counters move even without tokens
-  const unsigned blocks = (unsigned)(dm.T > 0 ? (dm.T + warps - 1) / warps : 1);
-  auto go = [&](auto kern) {
-    kern<<<blocks, warps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<const uint4*>(x), dm.T, dm.d / 8, dm.k, idx, row_of, offsets,
-        rows_routed(dm), reinterpret_cast<int*>(pe.ep_ws[pe.rank]), L,
-        ep_ptrs(pe.rows, pe.world), ep_ptrs(pe.ep_ws, pe.world), pe.world, dm.E / pe.world);
-  };
-  if (dm.k <= 8)
-    go(ep_dispatch_kernel<8>);
-  else if (dm.k <= 32)
-    go(ep_dispatch_kernel<32>);
-  else
-    return MOE_ERR_UNSUPPORTED_SHAPE;
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        num_sms <= 0)
+      num_sms = 148;
+  }
+  // persistent CTAs over the step's work items (their number lives on the device)
+  ep_dispatch_kernel<<<(unsigned)(4 * num_sms), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint4*>(x), dm.T, dm.d / 8, sorted_ids, offsets,
+      reinterpret_cast<int*>(pe.ep_ws[pe.rank]), L, ep_ptrs(pe.rows, pe.world),
+      ep_ptrs(pe.ep_ws, pe.world), pe.world, dm.E / pe.world);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -24,11 +24,11 @@ constexpr int kEpMaxWorld = MOE_EP_MAX_WORLD;
 enum EpWord {
   EP_STATUS = 0,     // device status word (moe_get_device_status reads it)
   EP_EPOCH = 1,      // steps planned so far on this rank
-  EP_CTR_ROWS = 2,   // forward rows arrived (one per source and step)
+  EP_CTR_ROWS = 2,   // (unused: forward rows arrive per expert, in `arrive` below)
   EP_CTR_Y = 3,      // expert outputs returned (one per owner and step)
   EP_CTR_DY = 4,     // backward rows arrived (one per source and step)
   EP_CTR_DX = 5,     // data gradients returned (one per owner and step)
-  EP_DONE_ROWS = 6,  // launch counters of the sending kernels (last CTA signals)
+  EP_DONE_ROWS = 6,  // (unused)
   EP_DONE_Y = 7,
   EP_DONE_DY = 8,
   EP_DONE_DX = 9,
@@ -45,9 +45,19 @@ enum EpWord {
 //   recv_real[W][E_l]   its real rows c[s][r E_l + e]
 //   src_off  [W][E_l]   the same segment's first row in source s's permuted rows
 //   over     [W]        1 when owner o would receive more rows than its buffers hold
+//   arrive   [E_l]      (owner) forward segments of local expert e arrived: one per
+//                       source and step, never reset
+//   own_cnt  [E]        (source) this rank's rows of expert g, c[r][g]
+//   done     [E]        (source) dispatch work items of expert g finished this step
+//                       (zeroed by the plan)
+//   chunk_pre[E + 1]    (source) prefix of the dispatch work items per expert, in the
+//                       order q = e W + o (each owner's local expert 0 first, then 1, ...)
 struct EpLayout {
-  size_t send_dst, recv_row, recv_cnt, recv_real, src_off, over, bytes;
+  size_t send_dst, recv_row, recv_cnt, recv_real, src_off, over, arrive, own_cnt, done,
+      chunk_pre, bytes;
 };
+
+constexpr int kEpDispatchRows = 16;  // rows of one segment a dispatch work item copies
 
 inline EpLayout ep_layout(int E, int world) {
   EpLayout L;
@@ -65,6 +75,14 @@ inline EpLayout ep_layout(int E, int world) {
   off += sizeof(int32_t) * world * El;
   L.over = off;
   off += sizeof(int32_t) * world;
+  L.arrive = off;
+  off += sizeof(int32_t) * El;
+  L.own_cnt = off;
+  off += sizeof(int32_t) * E;
+  L.done = off;
+  off += sizeof(int32_t) * E;
+  L.chunk_pre = off;
+  off += sizeof(int32_t) * (E + 1);
   L.bytes = align_up(off, 256);
   return L;
 }
@@ -126,7 +144,8 @@ __device__ __forceinline__ bool ep_wait_counter(const int* ep_ws, int ctr, int w
 // into their sources' buffers and signal them (FWD2 / DX1).
 struct EpGemm {
   const int* ep_ws;      // this rank's EP workspace (null: no exchange)
-  int wait_ctr;          // EP_CTR_ROWS / EP_CTR_DY, or 0: no wait
+  int wait_ctr;          // word of the counter to wait on (EP_CTR_DY), or 0: no wait
+  int per_group;         // 1: wait on word wait_ctr + g (the group's own arrival counter)
   int world, El;
   int ret_ctr;           // EP_CTR_Y / EP_CTR_DX, or 0: outputs stay local
   int done_word;         // EP_DONE_Y / EP_DONE_DX

@@ -400,19 +400,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0, issued = 0, lastpar = 0;
       bool ok = true;
       bool rows_in = args.ep.wait_ctr == 0;  // the routed rows of other ranks have arrived
+      int waited_g = -1;  // per-group waits: the last group whose rows this CTA waited for
       for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
         const TileInfo t = decode_tile<MODE>(tile, args);
         if (!tile_ok<MODE>(args, t)) continue;
         const GroupRec gr = load_group(args, t.g);
         const int roff = (int)rank * (t.half ? BM / 2 : BM);  // this CTA's rows of A
         const bool shared = t.g >= args.E;
-        if (!shared && !rows_in) {
-          // expert parallelism: every source's rows of this rank's experts must have
-          // landed before the first routed tile's copies (bounded wait)
+        if (!shared && !rows_in && t.g != waited_g) {
+          // expert parallelism: every source's rows of this group (per-group counters),
+          // or of all groups, must have landed before the tile's copies (bounded wait)
           int got = 1;
           if (lane == 0) {
-            got = ep_wait_counter(args.ep.ep_ws, args.ep.wait_ctr, args.ep.world, args.status,
-                                  MOE_ERR_DEVICE_TIMEOUT, args.budget_ns);
+            got = ep_wait_counter(args.ep.ep_ws, args.ep.wait_ctr + (args.ep.per_group ? t.g : 0),
+                                  args.ep.world, args.status, MOE_ERR_DEVICE_TIMEOUT,
+                                  args.budget_ns);
             // the rows were written through the generic proxy; the copies read them
             // through the async proxy
             asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -422,7 +424,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0) abort_pair();
             break;
           }
-          rows_in = true;
+          if (args.ep.per_group) waited_g = t.g; else rows_in = true;
         }
         const bool gat = WIDE && !shared;
         // this CTA's half of B: N/2 columns from n0 + rank * N/2, in 64-column chunks
@@ -1028,8 +1030,11 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
     a.ep.peer_ws = ep_ptrs(pe.ep_ws, pe.world);
     a.ep.recv_row = reinterpret_cast<const int32_t*>(epb + EL.recv_row);
     a.ep.src_off = reinterpret_cast<const int32_t*>(epb + EL.src_off);
-    if (mode == MODE_FWD1 || mode == MODE_DX2) {
-      a.ep.wait_ctr = mode == MODE_FWD1 ? EP_CTR_ROWS : EP_CTR_DY;
+    if (mode == MODE_FWD1) {  // each local expert's rows arrive on their own
+      a.ep.wait_ctr = (int)(EL.arrive / sizeof(int32_t));
+      a.ep.per_group = 1;
+    } else if (mode == MODE_DX2) {
+      a.ep.wait_ctr = EP_CTR_DY;
     } else if (mode == MODE_FWD2 || mode == MODE_DX1) {
       a.ep.ret_ctr = mode == MODE_FWD2 ? EP_CTR_Y : EP_CTR_DX;
       a.ep.done_word = mode == MODE_FWD2 ? EP_DONE_Y : EP_DONE_DX;

@@ -300,12 +300,12 @@ int moe_ep_plan(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* 
   return launch_ep_plan(*dims, *peers, counts_all, counts_loc, recv_cap, stream);
 }
 
-int moe_ep_dispatch(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* topk_idx,
-                    const int32_t* row_of, const int32_t* offsets, const void* x, void* stream) {
+int moe_ep_dispatch(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* sorted_ids,
+                    const int32_t* offsets, const void* x, void* stream) {
   int rc = check_ep(dims, peers, true);
   if (rc) return rc;
-  if (!offsets || (dims->T > 0 && (!topk_idx || !row_of || !x))) return MOE_ERR_INVALID_ARG;
-  return launch_ep_dispatch(*dims, *peers, topk_idx, row_of, offsets, x, stream);
+  if (!offsets || !sorted_ids || (dims->T > 0 && !x)) return MOE_ERR_INVALID_ARG;
+  return launch_ep_dispatch(*dims, *peers, sorted_ids, offsets, x, stream);
 }
 
 int moe_ep_zero_pads(const moe_dims* dims, const moe_ep_peers* peers, void* recv, void* stream) {

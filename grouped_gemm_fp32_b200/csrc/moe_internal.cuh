@@ -182,9 +182,8 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
 bool ep_peers_ok(const moe_ep_peers* p, bool need_rows);
 int launch_ep_plan(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* counts_all,
                    int32_t* counts_loc, int64_t cap, void* stream);
-int launch_ep_dispatch(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* idx,
-                       const int32_t* row_of, const int32_t* offsets, const void* x,
-                       void* stream);
+int launch_ep_dispatch(const moe_dims& dm, const moe_ep_peers& pe, const int32_t* sorted_ids,
+                       const int32_t* offsets, const void* x, void* stream);
 int launch_ep_zero_pads(const moe_dims& dm, const moe_ep_peers& pe, void* buf, void* stream);
 int launch_ep_wait(const moe_ep_peers& pe, int ctr, void* stream);
 int launch_combine_bwd_ep(const moe_dims& dm, const moe_ep_peers& pe, const void* dout,

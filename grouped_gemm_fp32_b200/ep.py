@@ -12,9 +12,12 @@ of E int32 counts per rank gives every rank the whole count table, from which
 ``moe_ep_plan`` computes every offset on the device.  The rows then move by kernels that
 write straight into the other ranks' buffers through peer pointers:
 
-  forward   moe_ep_dispatch writes x rows into the owners' receive buffers; the owners'
-            grouped GEMM runs its shared-expert tiles first and waits (bounded) for the
-            sources' rows before its first routed tile; its second GEMM writes each routed
+  forward   moe_ep_dispatch writes x rows into the owners' receive buffers, segment by
+            segment, raising the owner's arrival counter of each expert as its segment
+            lands; the owners' grouped GEMM runs its shared-expert tiles first and, before
+            each local expert's tiles, waits (bounded) for that expert's segments from
+            every source, so it starts on the first experts while later ones still
+            arrive; its second GEMM writes each routed
             row of Y straight back into the source's buffer (``grouped_gemm_fwd_ep``); the
             source waits for every owner (``moe_ep_wait``) and combines.
   backward  moe_ep_combine_bwd writes dY rows into the owners' buffers; the owners run
@@ -184,7 +187,7 @@ def plan(eb: EPBuffers, stream=None):
 def dispatch(eb: EPBuffers, x, stream=None):
     """This rank's x rows into their owners' receive buffers."""
     F = eb.full
-    L.moe_ep_dispatch(eb.dims, eb.peers["x_in"], F.topk_idx, F.row_of, F.offsets, x, stream)
+    L.moe_ep_dispatch(eb.dims, eb.peers["x_in"], F.sorted_ids, F.offsets, x, stream)
 
 
 def experts_forward(eb: EPBuffers, x, w1_loc, w2_loc, stream=None):

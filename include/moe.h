@@ -475,13 +475,17 @@ size_t moe_ep_workspace_size(const moe_dims* dims, int32_t world);
 int moe_ep_plan(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* counts_all,
                 int32_t* counts_loc, int64_t recv_cap, void* stream);
 
-/* Dispatch (Passage: §3.1, the all-to-all dispatch): x[t] to the owner of
- * each of its picks, at its row in the owner's
- * receive buffer (peers->rows[o], [recv_cap, d] bf16); then every owner's
- * arrival counter is raised.  topk_idx, row_of, offsets as moe_permute_align
- * wrote them for this rank; x [T, d] bf16. */
-int moe_ep_dispatch(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* topk_idx,
-                    const int32_t* row_of, const int32_t* offsets, const void* x, void* stream);
+/* Dispatch (Passage: §3.1, the all-to-all dispatch): this rank's segment of each
+ * expert g -- the rows of x that sorted_ids lists for it, in order -- into the
+ * owner's receive buffer (peers->rows[o], [recv_cap, d] bf16) at the rows the
+ * plan gives.  Segments go out local expert by local expert (every owner's first
+ * expert, then every owner's second, ...), and as soon as a segment is written the
+ * owner's arrival counter of that expert is raised, so the owner's grouped GEMM
+ * starts on an expert while later ones are still arriving.
+ *   sorted_ids [Rr], offsets [E + 1] as moe_permute_align wrote them for this
+ *   rank; x [T, d] bf16. */
+int moe_ep_dispatch(const moe_dims* dims, const moe_ep_peers* peers, const int32_t* sorted_ids,
+                    const int32_t* offsets, const void* x, void* stream);
 
 /* Owner (Passage: §3.2, segments padded to a fixed block): zero the pad rows
  * of every received segment of its receive buffer
@@ -505,8 +509,9 @@ int moe_ep_combine_bwd(const moe_dims* dims, const moe_ep_peers* peers, const vo
 
 /* Passage: §3.1 (communication overlapped with computation) and §3.2.
  * grouped_gemm_fwd on an owner (dims_loc: E = E_l local experts, rows_cap =
- * recv_cap): the first GEMM starts with the shared experts' tiles and waits
- * (bounded) for every source's rows before its first routed tile; the second
+ * recv_cap): the first GEMM starts with the shared experts' tiles and, before the
+ * tiles of each local expert, waits (bounded) until every source's segment of that
+ * expert has arrived; the second
  * GEMM writes each routed group's Y rows straight into the buffer of the rank
  * they came from (peers->rows[s], [rows_cap, d]: the source's routed rows, in its
  * permuted layout) instead of into y, then raises every source's counter.  The
