@@ -8,7 +8,8 @@
 // a per-group prefix of 256-row tile counts that is built on the device (no host
 // round trip).  The pages' version targets sm_90 warpgroup MMA; this one is
 // written for sm_100a.  CTAs run in pairs (a 2-CTA cluster, one CTA per SM) and
-// walk 256 x 256 tiles persistently with the paired tcgen05.mma (cta_group::2):
+// work through 256 x 256 tiles persistently, each pair drawing its next tile from
+// a counter in the workspace, with the paired tcgen05.mma (cta_group::2):
 // each CTA stages its own 128 rows of A and half of B (N/2 columns), so one
 // SM's shared memory feeds half the B traffic of a 1-CTA 128 x 256 tile.
 //   warp 0        TMA producer of this CTA's halves (6-stage ring, 32 KB a stage);
@@ -61,6 +62,11 @@ constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;     // two 256-column FP32 accumulators
 constexpr int MAX_GROUPS = 264;  // E <= 256 routed + S <= 8 shared
 constexpr int M_BAND = 8;        // m-tiles per band of the FWD / DX tile order
+// Tile indices reach the roles of a pair through a ring of SCHED_SLOTS entries in
+// each CTA's shared memory.  Each entry is read once by the MMA thread, by the
+// peer CTA's producer and by every epilogue warp of both CTAs.
+constexpr int SCHED_SLOTS = 8;
+constexpr int SCHED_READERS = 2 + 2 * EPI_WARPS;
 
 struct GemmArgs {
   int* status;
@@ -86,10 +92,14 @@ struct GemmArgs {
   uint32_t idesc_h_narrow;  // half tile with N = 128
   int half_ok;              // FWD / DX modes: a group's last 128 rows run as a half tile
   int staged;             // epilogue writes through shared memory + TMA stores
+  int mn3;                // DX / DW: an N- or M-major operand's two 64-column chunks of a
+                          // stage come in one 3-D copy (bit 0: A, bit 1: B)
   uint64_t budget_ns;
   const int32_t* gather_ids;  // FWD1 / DW1: token of each routed row, or null
   int gather_T;               // rows of the gathered tensor x
   int shared_first;           // FWD / DX: the shared groups' tiles come first
+  int* tile_ctr;              // this mode's tile counter in the workspace header (0 between
+                              // launches; the launch's last ticket puts it back to 0)
   EpGemm ep;                  // expert parallelism: rows to wait for, outputs to return
   // extents for the checks of the debug build: rows of the grouped row space (Rt), of
   // the routed A / B sources (Rr) and of x (T)
@@ -105,13 +115,18 @@ struct EpMaps {
 
 // full[] and tempty[] are used in the leader CTA only (both CTAs' producers and
 // epilogues signal the leader's); empty[] and tfull[] exist in both CTAs and
-// receive the leader's multicast commits.
+// receive the leader's multicast commits.  The tile ring: the leader's producer
+// writes sched[] in both CTAs and arrives on both CTAs' sfull[]; every reader
+// arrives on the leader's sempty[].
 struct SmemCtl {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  uint64_t sfull[SCHED_SLOTS];
+  uint64_t sempty[SCHED_SLOTS];
+  int sched[SCHED_SLOTS];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -317,12 +332,14 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ggemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-                 const __grid_constant__ CUtensorMap tmC /* unused (the slot of a third operand) */,
+                 const __grid_constant__ CUtensorMap tmC /* DW1: shared groups' x as 3-D chunks */,
                  const __grid_constant__ CUtensorMap tmO0 /* output (FWD1: H) */,
                  const __grid_constant__ CUtensorMap tmO1 /* FWD1: saved A1 */,
-                 const __grid_constant__ CUtensorMap tmA0h /* half tiles: 64-row A boxes */,
+                 const __grid_constant__ CUtensorMap tmA0h /* half tiles: 64-row A boxes
+                                                              (DW: A as 3-D chunks) */,
                  const __grid_constant__ CUtensorMap tmA1h,
-                 const __grid_constant__ CUtensorMap tmBh /* FWD1 half tiles: 64-row B boxes */,
+                 const __grid_constant__ CUtensorMap tmBh /* FWD1 half tiles: 64-row B boxes
+                                                             (DX / DW: B as 3-D chunks) */,
                  const __grid_constant__ EpMaps epm, const GemmArgs args) {
   constexpr bool A_MN = (MODE == MODE_DW2 || MODE == MODE_DW1);
   constexpr bool B_MN = (MODE != MODE_FWD1 && MODE != MODE_FWD2);
@@ -341,7 +358,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int npairs = gridDim.x >> 1;
   volatile int* abort_flag = &ctl->abort_flag;
 
   if (threadIdx.x == 0) {
@@ -354,6 +371,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ctl->tempty[a], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
     }
     mbar_init(&ctl->drain, 1);
+    for (int s = 0; s < SCHED_SLOTS; ++s) {
+      mbar_init(&ctl->sfull[s], 1);
+      mbar_init(&ctl->sempty[s], SCHED_READERS);
+      ctl->sched[s] = -1;
+    }
     ctl->abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
@@ -387,6 +409,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const int total_tiles =
       IS_DW ? args.G * args.MT * args.NT : __ldg(args.mtile_prefix + args.G) * args.NT;
 
+  // Tiles are handed out at run time: the leader's producer draws each next tile
+  // from the launch's counter (a ticket) and publishes it in the ring; -1 ends the
+  // pair's work.  All pairs therefore work on one window of consecutive tiles, in
+  // the order decode_tile gives, however long their tiles take, so the operands of
+  // the tiles in flight are shared in L2.  Every pair draws exactly one ticket at
+  // or past total_tiles, so the pair that draws total_tiles + npairs - 1 is the
+  // last to draw and puts the counter back to 0 for the next launch.
+  // No ring operation is a release fence at cluster scope (one would wait for the
+  // thread's copies or MMAs in flight): the peer's entry is written by st.async,
+  // whose bytes complete the peer's sfull phase, and a reader hands an entry back
+  // with an arrive predicated on the value it read.
+  auto ring_put = [&](int seq, int tile) -> bool {
+    const int s = seq % SCHED_SLOTS;
+    const uint32_t par = (uint32_t)(seq / SCHED_SLOTS) & 1u;
+    if (!mbar_wait(&ctl->sempty[s], par ^ 1u, abort_flag, args.status, MOE_ERR_DEVICE_TIMEOUT,
+                   args.budget_ns))
+      return false;
+    ctl->sched[s] = tile;
+    mbar_arrive(&ctl->sfull[s]);
+    const uint32_t peer_full = map_to_rank(&ctl->sfull[s], 1);
+    mbar_arrive_expect_tx_remote(peer_full, 4u);
+    st_async_u32(map_to_rank(&ctl->sched[s], 1), (uint32_t)tile, peer_full);
+    return true;
+  };
+  auto ring_get = [&](int seq, int& tile) -> bool {
+    const int s = seq % SCHED_SLOTS;
+    const uint32_t par = (uint32_t)(seq / SCHED_SLOTS) & 1u;
+    if (!mbar_wait(&ctl->sfull[s], par, abort_flag, args.status, MOE_ERR_DEVICE_TIMEOUT,
+                   args.budget_ns))
+      return false;
+    tile = *reinterpret_cast<volatile int*>(&ctl->sched[s]);
+    mbar_arrive_remote_after(map_to_rank(&ctl->sempty[s], 0), tile);
+    return true;
+  };
+  auto ticket_done = [&](int ticket) {
+    if (ticket == total_tiles + npairs - 1) atomicExch(args.tile_ctr, 0);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     // Lane 0 waits for free stages, arms the leader's full barrier and issues the
@@ -401,9 +461,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       bool rows_in = args.ep.wait_ctr == 0;  // the routed rows of other ranks have arrived
       int waited_g = -1;  // per-group waits: the last group whose rows this CTA waited for
-      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+      // The leader feeds the ring one tile ahead: it draws the next tile's ticket when
+      // a tile starts and publishes it a few K blocks in (the draw has returned by
+      // then), so the peer's producer never waits for a tile at a tile boundary.
+      int seq = 0;        // ring position of the current tile
+      int cur = -1;       // leader: the tile at ring position seq (-1: no more)
+      int nxt = -1;       // leader: the next tile's ticket, drawn but not yet published
+      bool last = false;  // leader: this pair has drawn its ticket past the last tile
+      auto publish = [&](int pos, int tk) -> bool {
+        cur = tk;
+        if (tk >= total_tiles) {
+          ticket_done(tk);
+          last = true;
+          cur = -1;
+        }
+        return ring_put(pos, cur);
+      };
+      if (leader && lane == 0 && !publish(0, atomicAdd(args.tile_ctr, 1))) abort_pair();
+      while (ok) {
+        int tile = -1, got = 1;
+        if (lane == 0) {
+          if (leader) {
+            tile = cur;
+            if (tile >= 0) nxt = atomicAdd(args.tile_ctr, 1);
+          } else {
+            got = ring_get(seq, tile);
+          }
+        }
+        if constexpr (WIDE) {
+          got = __shfl_sync(0xffffffffu, got, 0);
+          tile = __shfl_sync(0xffffffffu, tile, 0);
+        }
+        if (!got) {
+          if (lane == 0) abort_pair();
+          break;
+        }
+        if (tile < 0) break;
+        bool pub_done = !leader;
+        auto pub = [&]() {  // leader: the next tile goes to ring position seq + 1
+          if (!pub_done) {
+            pub_done = true;
+            if (lane == 0) {
+              const int tk = nxt;
+              nxt = -1;
+              if (!publish(seq + 1, tk)) abort_pair();
+            }
+          }
+        };
         const TileInfo t = decode_tile<MODE>(tile, args);
-        if (!tile_ok<MODE>(args, t)) continue;
+        if (!tile_ok<MODE>(args, t)) {
+          pub();
+          ++seq;
+          continue;
+        }
         const GroupRec gr = load_group(args, t.g);
         const int roff = (int)rank * (t.half ? BM / 2 : BM);  // this CTA's rows of A
         const bool shared = t.g >= args.E;
@@ -492,30 +602,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               tma_load_2d_pair(a_dst, t.half ? &tmA0h : &tmA0, fb, k0, gr.out_row + t.m0 + roff);
             }
             const int brow = t.g * args.b_group_rows + k0;
-            for (int c = 0; c < bchunks; ++c)
-              tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + boff + c * 64, brow);
+            if (bchunks == 2 && (args.mn3 & 2))
+              tma_load_3d_pair(b_dst, &tmBh, fb, 0, brow, (t.n0 + boff) >> 6);
+            else
+              for (int c = 0; c < bchunks; ++c)
+                tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + boff + c * 64, brow);
           } else {  // DW2 / DW1: K runs over the group's rows
             const CUtensorMap* ma;
             const CUtensorMap* mb;
+            const CUtensorMap* ma3;  // the same tensors as 3-D chunks
+            const CUtensorMap* mb3;
             int arow, brow;
             if constexpr (MODE == MODE_DW2) {
               ma = shared ? &tmA1 : &tmA0;
+              ma3 = shared ? &tmA1h : &tmA0h;
               arow = shared ? 0 : gr.a_row;
               mb = &tmB0;
+              mb3 = &tmBh;
               brow = gr.out_row;
             } else {
               ma = &tmA0;
+              ma3 = &tmA0h;
               arow = gr.out_row;
               mb = shared ? &tmB1 : &tmB0;
+              mb3 = shared ? &tmC : &tmBh;
               brow = shared ? 0 : gr.a_row;
             }
             if (lane == 0) {
+              if (args.mn3 & 1) {
+                tma_load_3d_pair(a_dst, ma3, fb, 0, arow + k0, (t.m0 + roff) >> 6);
+              } else {
 #pragma unroll
-              for (int c = 0; c < 2; ++c)
-                tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
-              if (!gat)
-                for (int c = 0; c < bchunks; ++c)
-                  tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + boff + c * 64, brow + k0);
+                for (int c = 0; c < 2; ++c)
+                  tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
+              }
+              if (!gat) {
+                if (bchunks == 2 && (args.mn3 & 2))
+                  tma_load_3d_pair(b_dst, mb3, fb, 0, brow + k0, (t.n0 + boff) >> 6);
+                else
+                  for (int c = 0; c < bchunks; ++c)
+                    tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + boff + c * 64, brow + k0);
+              }
             }
             if constexpr (MODE == MODE_DW1) {
               if (gat) {
@@ -535,7 +662,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             stage = 0;
             phase ^= 1;
           }
+          if (kb == min(t.nkb - 1, 3)) pub();
         }
+        pub();  // a tile without K blocks (a DW group with no rows), or an early stop
+        ++seq;
+      }
+      // A pair that stopped early still draws up to its ticket past the last tile,
+      // so the launch's last ticket is drawn and the counter goes back to 0.
+      if (leader && lane == 0 && !last) {
+        int tk = nxt >= 0 ? nxt : atomicAdd(args.tile_ctr, 1);
+        while (tk < total_tiles) tk = atomicAdd(args.tile_ctr, 1);
+        ticket_done(tk);
       }
       // The leader's full barriers count both CTAs' copies: once they have
       // completed, every copy either CTA started has landed.
@@ -559,7 +696,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int it = 0;  // tiles processed (the debug build skips invalid ones)
       bool ok = true;
-      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+      for (int seq = 0; ok; ++seq) {
+        int tile = -1;
+        if (!ring_get(seq, tile)) {
+          abort_pair();
+          break;
+        }
+        if (tile < 0) break;
         const TileInfo t = decode_tile<MODE>(tile, args);
         if (!tile_ok<MODE>(args, t)) continue;
         const int acc = it & 1;
@@ -626,7 +769,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive_remote(tempty_leader[acc]);
     };
     int it = 0;  // tiles processed
-    for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
+    for (int seq = 0;; ++seq, ++it) {
+      int tile = -1, got = 1;
+      if (lane == 0) got = ring_get(seq, tile);
+      got = __shfl_sync(0xffffffffu, got, 0);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (!got) {
+        abort_pair();
+        break;
+      }
+      if (tile < 0) break;
       const TileInfo t = decode_tile<MODE>(tile, args);
       if (!tile_ok<MODE>(args, t)) {
         --it;
@@ -920,7 +1072,7 @@ int launch_mode(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap&
     cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     num_sms &= ~1;  // whole CTA pairs, one CTA per SM
     // A pair needs two co-scheduled SMs: launch only as many pairs as can be
-    // resident at once, so the static tile split has no late-starting pairs.
+    // resident at once (one persistent pair per two SMs; tiles are drawn at run time).
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms);
     cfg.blockDim = dim3(NUM_THREADS);
@@ -980,6 +1132,25 @@ bool make_map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
   return make_map_2d(m, base, rows, cols, 2, box_rows);
 }
 
+// A row-major bf16 matrix [rows, cols] seen as 64-column chunks [cols / 64][rows][64]
+// (the chunk index outermost, 128 bytes apart): one box = 64 rows of two adjacent
+// chunks, landing in shared memory as chunk 0's 64 x 128-byte rows, then chunk 1's
+// -- the layout of two 64-row 2-D boxes 8 KB apart.  False when cols is not a
+// multiple of 64 or the driver does not take the map; the caller then keeps the
+// 2-D boxes.
+static bool make_map_mn3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc || base == nullptr || rows <= 0 || cols % 64 != 0 || cols < 128) return false;
+  cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), 128u};
+  cuuint32_t box[3] = {64u, 64u, 2u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 uint64_t wait_budget_ns() {
   static uint64_t v = [] {
     const char* s = getenv("MOE_WAIT_BUDGET_NS");
@@ -1004,6 +1175,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   a.groups = reinterpret_cast<const GroupRec*>(wsb + L.groups);
   a.mtile_prefix = reinterpret_cast<const int*>(wsb + L.mtile_prefix);
   a.dw_order = reinterpret_cast<const int*>(wsb + L.dw_order);
+  a.tile_ctr = reinterpret_cast<int*>(const_cast<void*>(ws)) + kTileCtrWord + (int)mode;
   a.G = G;
   a.E = dm.E;
   a.I = I;
@@ -1044,7 +1216,9 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
   }
 
   CUtensorMap m0{}, m1{}, n0{}, n1{}, o0{}, o1{};
-  CUtensorMap mh0{}, mh1{}, nh{};  // half tiles: 64-row boxes of A (and of B in FWD1)
+  CUtensorMap mh0{}, mh1{}, nh{};  // half tiles: 64-row boxes of A (and of B in FWD1);
+                                   // DX / DW: 3-D chunk maps of A (mh) and B (nh)
+  CUtensorMap cw{};                // DW1: 3-D chunk map of the shared groups' x
   bool ok = true;
   // a dummy map stands in for unused slots (never read by the kernel)
   auto same = [](CUtensorMap& dst, const CUtensorMap& src) { dst = src; };
@@ -1127,7 +1301,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.idesc_h_narrow = idesc_bf16_f32(BM, 128, false, true);
       ok &= make_map_bf16(&mh0, ops.a0, Rr, d, BM / 2);
       if (dm.S > 0 && T > 0) ok &= make_map_bf16(&mh1, ops.a1, T, d, BM / 2); else same(mh1, mh0);
-      same(nh, n0);
+      if (make_map_mn3(&nh, ops.b0, (int64_t)G * d, I)) a.mn3 = 2; else same(nh, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, 2 * I, 2, 32)) return MOE_ERR_CUDA;
@@ -1150,7 +1324,7 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       a.idesc_h_narrow = idesc_bf16_f32(BM, 128, false, true);
       ok &= make_map_bf16(&mh0, ops.a0, Rt, 2 * I, BM / 2);
       same(mh1, mh0);
-      same(nh, n0);
+      if (make_map_mn3(&nh, ops.b0, (int64_t)G * 2 * I, d)) a.mn3 = 2; else same(nh, n0);
       if (!ok) return MOE_ERR_CUDA;
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, Rt, d, 2, 32)) return MOE_ERR_CUDA;
@@ -1168,9 +1342,15 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       ok &= make_map_bf16(&n0, ops.b0, Rt, I, 64);
       same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
+      if (make_map_mn3(&mh0, ops.a0, Rr, d) &&
+          (dm.S > 0 && T > 0 ? make_map_mn3(&mh1, ops.a1, T, d) : (same(mh1, mh0), true)))
+        a.mn3 |= 1;
+      else
+        same(mh0, m0), same(mh1, m0);
+      if (make_map_mn3(&nh, ops.b0, Rt, I)) a.mn3 |= 2; else same(nh, n0);
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * d, I, 4, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, epm, a, st);
+      return launch_mode<MODE_DW2>(m0, m1, n0, n1, n0, o0, o0, mh0, mh1, nh, epm, a, st);
     }
     case MODE_DW1: {  // dW1_g [2I, d] = dA_g^T X_g
       a.m_out = 2 * I;
@@ -1191,9 +1371,19 @@ int launch_grouped_gemm(GemmMode mode, const moe_dims& dm, const void* ws,
       }
       if (dm.S > 0 && T > 0) ok &= make_map_bf16(&n1, ops.b1, T, d, 64); else same(n1, n0);
       if (!ok) return MOE_ERR_CUDA;
+      if (make_map_mn3(&mh0, ops.a0, Rt, 2 * I)) a.mn3 |= 1; else same(mh0, m0);
+      same(mh1, mh0);
+      {
+        // B: the routed rows (unless gathered) and the shared groups' x rows
+        const bool rb = ops.gather_ids != nullptr || make_map_mn3(&nh, ops.b0, Rr, d);
+        const bool sb = !(dm.S > 0 && T > 0) || make_map_mn3(&cw, ops.b1, T, d);
+        if (ops.gather_ids != nullptr) same(nh, n0);
+        if (!(dm.S > 0 && T > 0)) same(cw, n0);
+        if (rb && sb) a.mn3 |= 2; else same(nh, n0), same(cw, n0);
+      }
       a.staged = 1;
       if (!make_map_2d(&o0, ops.out, (int64_t)G * 2 * I, d, 4, 32)) return MOE_ERR_CUDA;
-      return launch_mode<MODE_DW1>(m0, m1, n0, n1, n0, o0, o0, m0, m0, m0, epm, a, st);
+      return launch_mode<MODE_DW1>(m0, m1, n0, n1, cw, o0, o0, mh0, mh1, nh, epm, a, st);
     }
   }
   return MOE_ERR_INVALID_ARG;

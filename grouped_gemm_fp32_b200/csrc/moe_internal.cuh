@@ -41,7 +41,13 @@ struct GroupRec {
 
 constexpr int kChunk = 1024;      // routed assignments per histogram chunk
 constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] tiles total,
-                                  // [3] routing valid, [4] bad expert id seen
+                                  // [3] routing valid, [4] bad expert id seen,
+                                  // [5 + mode] tile counter of each grouped-GEMM mode
+constexpr int kTileCtrWord = 5;
+// what each routing call clears: header words 3 (routing valid) to 10 (the last
+// tile counter); a counter left past 0 by a launch that was cut short starts the
+// next step at 0 again
+constexpr size_t kHeaderClearBytes = (kTileCtrWord + 6 - 3) * sizeof(int32_t);
 
 // Layer workspace: the routing tables first (`bytes` of them), then the
 // gate's split weights, then the router backward's scratch.

@@ -289,7 +289,7 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
   const int64_t Rr = rows_routed(dm);
 
   if (!cuda_ok(cudaMemsetAsync(sorted_ids, 0xFF, sizeof(int32_t) * Rr, st)) ||
-      !cuda_ok(cudaMemsetAsync(wsb + 3 * sizeof(int), 0, 2 * sizeof(int), st)))
+      !cuda_ok(cudaMemsetAsync(wsb + 3 * sizeof(int), 0, kHeaderClearBytes, st)))
     return MOE_ERR_CUDA;
   if (n > 0) {
     hist_kernel<<<L.nchunks, 256, 0, st>>>(idx, n, dm.E, hist, status);
@@ -328,7 +328,7 @@ int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offset
   int32_t* hist = reinterpret_cast<int32_t*>(wsb + L.chunk_hist);
   if (!cuda_ok(cudaMemcpyAsync(hist, counts, sizeof(int32_t) * dm.E, cudaMemcpyDeviceToDevice,
                                st)) ||
-      !cuda_ok(cudaMemsetAsync(wsb + 3 * sizeof(int), 0, 2 * sizeof(int), st)))
+      !cuda_ok(cudaMemsetAsync(wsb + 3 * sizeof(int), 0, kHeaderClearBytes, st)))
     return MOE_ERR_CUDA;
   return launch_groups(dm, hist, 1, nullptr, offsets, ws, st);
 }

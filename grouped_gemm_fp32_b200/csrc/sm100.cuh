@@ -111,6 +111,43 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Arrive with no release fence on a barrier of any CTA of the cluster, once
+// `used` -- a value this thread loaded -- is in a register: the arrive is
+// predicated on it, so it cannot be performed before that load has completed.
+// It tells a writer that the loaded entry may be overwritten, and orders
+// nothing else (no wait for this thread's copies, MMAs or stores in flight).
+__device__ __forceinline__ void mbar_arrive_remote_after(uint32_t cluster_addr, int used) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.s32 p, %1, 2147483647;\n\t"
+      "@p mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n\t}" ::"r"(cluster_addr),
+      "r"(used)
+      : "memory");
+}
+
+// Arrive on a barrier of another CTA of the cluster and raise the bytes its
+// phase waits for (no release fence: the bytes come from st_async_u32 below).
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_addr,
+                                                             uint32_t bytes) {
+  asm volatile(
+      "mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+          cluster_addr),
+      "r"(bytes)
+      : "memory");
+}
+
+// 32-bit store into another CTA's shared memory that counts 4 transaction bytes on
+// the barrier `cluster_bar` of that CTA once the value is there: a thread of that
+// CTA that sees the barrier's phase complete sees the value.
+__device__ __forceinline__ void st_async_u32(uint32_t cluster_addr, uint32_t v,
+                                             uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+          cluster_addr),
+      "r"(v), "r"(cluster_bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
@@ -140,6 +177,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
+// The same for a 3-D map (coordinates x, y, z, innermost first).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y,
+                                                 int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 

@@ -87,9 +87,14 @@ int64_t moe_rows_total(const moe_dims* dims);
  * serves a whole layer.  It starts with the routing tables (the status word,
  * the group table, tile prefixes, per-chunk histograms): moe_permute_align (or
  * grouped_gemm_set_groups) writes them, the GEMM and combine-backward calls
- * read them.  After them, 1024-byte aligned, moe_gate_topk keeps the gate
- * weights split into three bf16 planes, 3 * E_pad * d * 2 bytes with E_pad = E
- * rounded up to a multiple of 32. */
+ * read them.  The routing header also holds one tile counter per grouped-GEMM
+ * launch kind (forward GEMM1 and GEMM2, the two data-gradient and the two
+ * weight-gradient GEMMs): the routing calls clear them, and every launch draws
+ * its tiles from its counter and leaves it at 0, also when its waits ran out.
+ * So two launches of the same kind on one workspace must not overlap on the GPU
+ * (launches of different kinds may).  After the routing tables, 1024-byte
+ * aligned, moe_gate_topk keeps the gate weights split into three bf16 planes,
+ * 3 * E_pad * d * 2 bytes with E_pad = E rounded up to a multiple of 32. */
 size_t moe_workspace_size(const moe_dims* dims);
 
 /* Gate and aux-loss-free top-k routing.

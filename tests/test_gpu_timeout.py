@@ -1,8 +1,9 @@
 """Failure detection without a GPU fault: every wait inside the grouped GEMM and
 the gate is bounded.  With a wait budget of 1 ns the kernel's roles give up, record
 MOE_ERR_DEVICE_TIMEOUT in the workspace status word, drain the copies and MMAs
-they already started and return; the host reads the status and the CUDA
-context stays usable.  Runs in a child process because the budget
+they already started and return (each pair still draws up to its ticket past the last
+tile, so the launch's tile counter goes back to 0); the host reads the status and the
+CUDA context stays usable.  Runs in a child process because the budget
 (MOE_WAIT_BUDGET_NS) is read once per process."""
 import os
 import subprocess
@@ -35,6 +36,8 @@ moe.grouped_gemm_fwd(dm, ws, x, None, w1, w2, h, None, y)
 torch.cuda.synchronize()
 st = moe.moe_get_device_status(ws)
 print("gemm status", st)
+# the launch's tile counter is back at 0 although every role gave up early
+print("tile counters", ws[20:44].view(torch.int32).tolist())
 # the context still works: the status was cleared and a plain op runs
 assert moe.moe_get_device_status(ws) == 0
 # the gate's waits are bounded the same way
@@ -59,6 +62,7 @@ def test_bounded_waits_report_timeout_and_keep_context():
                        capture_output=True, text=True, timeout=300)
     assert p.returncode == 0, p.stdout + p.stderr
     assert "gemm status -4" in p.stdout, p.stdout
+    assert "tile counters [0, 0, 0, 0, 0, 0]" in p.stdout, p.stdout
     assert "gate status -4" in p.stdout, p.stdout
     assert "context ok True" in p.stdout, p.stdout
 
