@@ -12,13 +12,15 @@
 // a counter in the workspace, with the paired tcgen05.mma (cta_group::2):
 // each CTA stages its own 128 rows of A and half of B (N/2 columns), so one
 // SM's shared memory feeds half the B traffic of a 1-CTA 128 x 256 tile.
-//   warp 0        TMA producer of this CTA's halves (6-stage ring, 32 KB a stage);
-//                 completions are counted on the leader CTA's barriers
+//   warp 0        TMA producer of this CTA's rows of A (6-stage ring, 32 KB a stage
+//                 with B); in the leader CTA also the tile hand-out and the arming of
+//                 each stage; completions are counted on the leader CTA's barriers
 //   warp 1        tensor-memory owner; in the leader CTA the single-thread
 //                 tcgen05.mma issuer for the pair
 //   warps 2..9    epilogue of this CTA's 128 accumulator rows (two warps per
 //                 32-lane quarter, each on half the columns): tcgen05.ld, fused
 //                 SwiGLU / SwiGLU-backward, bf16 or f32 stores
+//   warp 10       TMA producer of this CTA's half of B
 // with two 256-column FP32 accumulators in tensor memory per CTA so the
 // epilogue of one tile overlaps the MMAs of the next.  Segments are padded to
 // 128-row blocks, so a group's last m-tile may hold only 128 rows: it runs as a
@@ -58,15 +60,17 @@ constexpr int A_BYTES = BM * BK * 2;    // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = 128 * BK * 2;   // 16 KB: this CTA's half of B (N/2 <= 128)
 constexpr int EPI_WARPS = 8;            // two per tensor-memory lane quarter
 constexpr int SLOT_BYTES = 32 * 128;    // an epilogue warp's staging slot: 32 rows x 128 B
-constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int B_WARP = 2 + EPI_WARPS;        // the producer of B (after the epilogue warps)
+constexpr int NUM_THREADS = 96 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;     // two 256-column FP32 accumulators
 constexpr int MAX_GROUPS = 264;  // E <= 256 routed + S <= 8 shared
 constexpr int M_BAND = 8;        // m-tiles per band of the FWD / DX tile order
 // Tile indices reach the roles of a pair through a ring of SCHED_SLOTS entries in
 // each CTA's shared memory.  Each entry is read once by the MMA thread, by the
-// peer CTA's producer and by every epilogue warp of both CTAs.
+// peer CTA's A producer, by both CTAs' B producers and by every epilogue warp of
+// both CTAs.
 constexpr int SCHED_SLOTS = 8;
-constexpr int SCHED_READERS = 2 + 2 * EPI_WARPS;
+constexpr int SCHED_READERS = 4 + 2 * EPI_WARPS;
 
 struct GemmArgs {
   int* status;
@@ -447,27 +451,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (ticket == total_tiles + npairs - 1) atomicExch(args.tile_ctr, 0);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer --
-    // Lane 0 waits for free stages, arms the leader's full barrier and issues the
-    // tile copies.  With gathered x rows (FWD1's routed A, DW1's routed B) all 32
-    // lanes issue four-row gathers of the same stage as well.
-    constexpr bool CAN_GATHER = (MODE == MODE_FWD1 || MODE == MODE_DW1);
-    // one loop, compiled twice: WIDE (all lanes, gathers) and lane 0 alone
-    auto produce = [&](auto wide_tag) {
+  if (warp == 0 || warp == B_WARP) {
+    // ----------------------------------------------------------- producers --
+    // Two producer warps per CTA, each waiting for free stages on its own: warp 0
+    // copies this CTA's A and hands out the tiles (the leader's warp 0 draws them and
+    // arms the leader's full barrier with both operands' bytes of both CTAs; the
+    // other operand's copies may land before it arms, the barrier's transaction count
+    // allows that), warp B_WARP copies this CTA's half of B.  Lane 0 issues the
+    // copies; with gathered x rows (FWD1's routed A, DW1's routed B) all 32 lanes of
+    // that operand's warp issue four-row gathers.
+    constexpr bool GATHER_A = MODE == MODE_FWD1;
+    constexpr bool GATHER_B = MODE == MODE_DW1;
+    // one loop, compiled per operand (PART 0: A and the tiles, 1: B) and per width
+    // (WIDE: all lanes, gathers; otherwise lane 0 alone)
+    auto produce = [&](auto wide_tag, auto part_tag) {
       constexpr bool WIDE = decltype(wide_tag)::value;
+      constexpr int PART = decltype(part_tag)::value;
+      const bool writer = PART == 0 && leader;  // draws and publishes the tiles
       int stage = 0;
       uint32_t phase = 0, issued = 0, lastpar = 0;
       bool ok = true;
-      bool rows_in = args.ep.wait_ctr == 0;  // the routed rows of other ranks have arrived
+      bool rows_in = PART == 1 || args.ep.wait_ctr == 0;  // other ranks' A rows have arrived
       int waited_g = -1;  // per-group waits: the last group whose rows this CTA waited for
-      // The leader feeds the ring one tile ahead: it draws the next tile's ticket when
+      // The writer feeds the ring one tile ahead: it draws the next tile's ticket when
       // a tile starts and publishes it a few K blocks in (the draw has returned by
-      // then), so the peer's producer never waits for a tile at a tile boundary.
+      // then), so no other producer waits for a tile at a tile boundary.
       int seq = 0;        // ring position of the current tile
-      int cur = -1;       // leader: the tile at ring position seq (-1: no more)
-      int nxt = -1;       // leader: the next tile's ticket, drawn but not yet published
-      bool last = false;  // leader: this pair has drawn its ticket past the last tile
+      int cur = -1;       // writer: the tile at ring position seq (-1: no more)
+      int nxt = -1;       // writer: the next tile's ticket, drawn but not yet published
+      bool last = false;  // writer: this pair has drawn its ticket past the last tile
       auto publish = [&](int pos, int tk) -> bool {
         cur = tk;
         if (tk >= total_tiles) {
@@ -477,11 +489,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         return ring_put(pos, cur);
       };
-      if (leader && lane == 0 && !publish(0, atomicAdd(args.tile_ctr, 1))) abort_pair();
+      if (writer && lane == 0 && !publish(0, atomicAdd(args.tile_ctr, 1))) abort_pair();
       while (ok) {
         int tile = -1, got = 1;
         if (lane == 0) {
-          if (leader) {
+          if (writer) {
             tile = cur;
             if (tile >= 0) nxt = atomicAdd(args.tile_ctr, 1);
           } else {
@@ -497,8 +509,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         if (tile < 0) break;
-        bool pub_done = !leader;
-        auto pub = [&]() {  // leader: the next tile goes to ring position seq + 1
+        bool pub_done = !writer;
+        auto pub = [&]() {  // writer: the next tile goes to ring position seq + 1
           if (!pub_done) {
             pub_done = true;
             if (lane == 0) {
@@ -519,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const bool shared = t.g >= args.E;
         if (!shared && !rows_in && t.g != waited_g) {
           // expert parallelism: every source's rows of this group (per-group counters),
-          // or of all groups, must have landed before the tile's copies (bounded wait)
+          // or of all groups, must have landed before the tile's A copies (bounded wait)
           int got = 1;
           if (lane == 0) {
             got = ep_wait_counter(args.ep.ep_ws, args.ep.wait_ctr + (args.ep.per_group ? t.g : 0),
@@ -564,23 +576,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          if (leader && lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], pair_bytes);
+          if (writer && lane == 0) mbar_arrive_expect_tx(&ctl->full[stage], pair_bytes);
           const uint32_t fb = map_to_rank(&ctl->full[stage], 0);
-          uint8_t* a_dst = sA + stage * A_BYTES;
-          uint8_t* b_dst = sB + stage * B_BYTES;
+          [[maybe_unused]] uint8_t* a_dst = sA + stage * A_BYTES;
+          [[maybe_unused]] uint8_t* b_dst = sB + stage * B_BYTES;
           const int k0 = kb * BK;
-          if constexpr (MODE == MODE_FWD1) {
-            // A: rows m0 + roff; B: the leader stages the gate rows, the peer the up
-            // rows -- in a half tile each CTA stages 64 gate rows and the matching 64
-            // up rows, so a row's gate and up sums land in the same tensor-memory lane
-            if (gat && (!t.half || lane < 16))
-              tma_gather4_pair(a_dst + lane * 512, &tmA0, fb, k0, rows4.x, rows4.y, rows4.z,
-                               rows4.w);
-            if (lane == 0) {
-              if (!gat)
+          if constexpr (PART == 0) {
+            // ---- A: this CTA's rows of the tile (DW: its 128 columns of A^T)
+            if constexpr (MODE == MODE_FWD1) {
+              if (gat && (!t.half || lane < 16))
+                tma_gather4_pair(a_dst + lane * 512, &tmA0, fb, k0, rows4.x, rows4.y, rows4.z,
+                                 rows4.w);
+              if (lane == 0 && !gat)
                 tma_load_2d_pair(a_dst,
                                  t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0),
                                  fb, k0, (shared ? 0 : gr.a_row) + t.m0 + roff);
+            } else if constexpr (MODE == MODE_FWD2 || MODE == MODE_DX1) {
+              tma_load_2d_pair(a_dst, t.half ? &tmA0h : &tmA0, fb, k0, gr.out_row + t.m0 + roff);
+            } else if constexpr (MODE == MODE_DX2) {
+              tma_load_2d_pair(a_dst,
+                               t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0),
+                               fb, k0, (shared ? 0 : gr.a_row) + t.m0 + roff);
+            } else {  // DW2 / DW1: K runs over the group's rows
+              const int arow = (MODE == MODE_DW2) ? (shared ? 0 : gr.a_row) : gr.out_row;
+              if (args.mn3 & 1) {
+                const CUtensorMap* ma3 = (MODE == MODE_DW2 && shared) ? &tmA1h : &tmA0h;
+                tma_load_3d_pair(a_dst, ma3, fb, 0, arow + k0, (t.m0 + roff) >> 6);
+              } else {
+                const CUtensorMap* ma = (MODE == MODE_DW2 && shared) ? &tmA1 : &tmA0;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                  tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
+              }
+            }
+          } else {
+            // ---- B: this CTA's half of the tile's columns
+            if constexpr (MODE == MODE_FWD1) {
+              // the leader stages the gate rows, the peer the up rows -- in a half tile
+              // each CTA stages 64 gate rows and the matching 64 up rows, so a row's
+              // gate and up sums land in the same tensor-memory lane
               const int brow = t.g * args.b_group_rows + t.n0;
               if (t.half) {
                 tma_load_2d_pair(b_dst, &tmBh, fb, k0, brow + (int)rank * 64);
@@ -588,71 +622,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               } else {
                 tma_load_2d_pair(b_dst, &tmB0, fb, k0, brow + (leader ? 0 : args.I));
               }
-            }
-          } else if constexpr (MODE == MODE_FWD2) {
-            tma_load_2d_pair(a_dst, t.half ? &tmA0h : &tmA0, fb, k0, gr.out_row + t.m0 + roff);
-            tma_load_2d_pair(b_dst, &tmB0, fb, k0,
-                             t.g * args.b_group_rows + t.n0 + (int)rank * 128);
-          } else if constexpr (MODE == MODE_DX2 || MODE == MODE_DX1) {
-            if constexpr (MODE == MODE_DX2) {
-              tma_load_2d_pair(a_dst,
-                               t.half ? (shared ? &tmA1h : &tmA0h) : (shared ? &tmA1 : &tmA0),
-                               fb, k0, (shared ? 0 : gr.a_row) + t.m0 + roff);
-            } else {
-              tma_load_2d_pair(a_dst, t.half ? &tmA0h : &tmA0, fb, k0, gr.out_row + t.m0 + roff);
-            }
-            const int brow = t.g * args.b_group_rows + k0;
-            if (bchunks == 2 && (args.mn3 & 2))
-              tma_load_3d_pair(b_dst, &tmBh, fb, 0, brow, (t.n0 + boff) >> 6);
-            else
-              for (int c = 0; c < bchunks; ++c)
-                tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + boff + c * 64, brow);
-          } else {  // DW2 / DW1: K runs over the group's rows
-            const CUtensorMap* ma;
-            const CUtensorMap* mb;
-            const CUtensorMap* ma3;  // the same tensors as 3-D chunks
-            const CUtensorMap* mb3;
-            int arow, brow;
-            if constexpr (MODE == MODE_DW2) {
-              ma = shared ? &tmA1 : &tmA0;
-              ma3 = shared ? &tmA1h : &tmA0h;
-              arow = shared ? 0 : gr.a_row;
-              mb = &tmB0;
-              mb3 = &tmBh;
-              brow = gr.out_row;
-            } else {
-              ma = &tmA0;
-              ma3 = &tmA0h;
-              arow = gr.out_row;
-              mb = shared ? &tmB1 : &tmB0;
-              mb3 = shared ? &tmC : &tmBh;
-              brow = shared ? 0 : gr.a_row;
-            }
-            if (lane == 0) {
-              if (args.mn3 & 1) {
-                tma_load_3d_pair(a_dst, ma3, fb, 0, arow + k0, (t.m0 + roff) >> 6);
+            } else if constexpr (MODE == MODE_FWD2) {
+              tma_load_2d_pair(b_dst, &tmB0, fb, k0,
+                               t.g * args.b_group_rows + t.n0 + (int)rank * 128);
+            } else if constexpr (MODE == MODE_DX2 || MODE == MODE_DX1) {
+              const int brow = t.g * args.b_group_rows + k0;
+              if (bchunks == 2 && (args.mn3 & 2))
+                tma_load_3d_pair(b_dst, &tmBh, fb, 0, brow, (t.n0 + boff) >> 6);
+              else
+                for (int c = 0; c < bchunks; ++c)
+                  tma_load_2d_pair(b_dst + c * 8192, &tmB0, fb, t.n0 + boff + c * 64, brow);
+            } else {  // DW2 / DW1
+              const CUtensorMap* mb;
+              const CUtensorMap* mb3;  // the same tensor as 3-D chunks
+              int brow;
+              if constexpr (MODE == MODE_DW2) {
+                mb = &tmB0;
+                mb3 = &tmBh;
+                brow = gr.out_row;
               } else {
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                  tma_load_2d_pair(a_dst + c * 8192, ma, fb, t.m0 + roff + c * 64, arow + k0);
+                mb = shared ? &tmB1 : &tmB0;
+                mb3 = shared ? &tmC : &tmBh;
+                brow = shared ? 0 : gr.a_row;
               }
-              if (!gat) {
+              if (lane == 0 && !gat) {
                 if (bchunks == 2 && (args.mn3 & 2))
                   tma_load_3d_pair(b_dst, mb3, fb, 0, brow + k0, (t.n0 + boff) >> 6);
                 else
                   for (int c = 0; c < bchunks; ++c)
                     tma_load_2d_pair(b_dst + c * 8192, mb, fb, t.n0 + boff + c * 64, brow + k0);
               }
-            }
-            if constexpr (MODE == MODE_DW1) {
-              if (gat) {
-                // lanes 0..15: 64-column chunk 0, lanes 16..31: chunk 1; lane i % 16
-                // brings K rows 4 i .. 4 i + 3 of this block
-                const int c = lane >> 4;
-                if (c < bchunks)
-                  tma_gather4_pair(b_dst + c * 8192 + (lane & 15) * 512, mb, fb,
-                                   t.n0 + boff + c * 64, rows4.x, rows4.y, rows4.z, rows4.w);
-                if (kb + 1 < t.nkb) rows4 = gather_rows4(args, gr, k0 + BK + 4 * (lane & 15), first);
+              if constexpr (MODE == MODE_DW1) {
+                if (gat) {
+                  // lanes 0..15: 64-column chunk 0, lanes 16..31: chunk 1; lane i % 16
+                  // brings K rows 4 i .. 4 i + 3 of this block
+                  const int c = lane >> 4;
+                  if (c < bchunks)
+                    tma_gather4_pair(b_dst + c * 8192 + (lane & 15) * 512, mb, fb,
+                                     t.n0 + boff + c * 64, rows4.x, rows4.y, rows4.z, rows4.w);
+                  if (kb + 1 < t.nkb)
+                    rows4 = gather_rows4(args, gr, k0 + BK + 4 * (lane & 15), first);
+                }
               }
             }
           }
@@ -669,14 +679,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
       // A pair that stopped early still draws up to its ticket past the last tile,
       // so the launch's last ticket is drawn and the counter goes back to 0.
-      if (leader && lane == 0 && !last) {
+      if (writer && lane == 0 && !last) {
         int tk = nxt >= 0 ? nxt : atomicAdd(args.tile_ctr, 1);
         while (tk < total_tiles) tk = atomicAdd(args.tile_ctr, 1);
         ticket_done(tk);
       }
-      // The leader's full barriers count both CTAs' copies: once they have
-      // completed, every copy either CTA started has landed.
-      if (leader && lane == 0)
+      // The leader's full barriers count both operands' copies of both CTAs: once the
+      // phases it armed have completed, every copy of those stages has landed.
+      if (writer && lane == 0)
         for (int s = 0; s < STAGES; ++s)
           if (issued & (1u << s)) {
             volatile int never = 0;
@@ -684,10 +694,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                       MOE_ERR_DEVICE_TIMEOUT, drain_budget);
           }
     };
-    if (CAN_GATHER && args.gather_ids != nullptr) {
-      if constexpr (CAN_GATHER) produce(std::true_type{});
-    } else if (lane == 0) {
-      produce(std::false_type{});
+    using A_PART = std::integral_constant<int, 0>;
+    using B_PART = std::integral_constant<int, 1>;
+    if (warp == 0) {
+      if (GATHER_A && args.gather_ids != nullptr) {
+        if constexpr (GATHER_A) produce(std::true_type{}, A_PART{});
+      } else if (lane == 0) {
+        produce(std::false_type{}, A_PART{});
+      }
+    } else {
+      if (GATHER_B && args.gather_ids != nullptr) {
+        if constexpr (GATHER_B) produce(std::true_type{}, B_PART{});
+      } else if (lane == 0) {
+        produce(std::false_type{}, B_PART{});
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer (leader) --
