@@ -636,13 +636,13 @@ def run_ours(args):
     case.check_status(stream, "after timing")
 
     # kernels per step: gate 2 (weight split, gate), permute 3 (histogram, groups,
-    # scatter; + row copy and pad zeroing without gathering), forward GEMMs 2, combine 1;
-    # train adds the balance loss 2 (chunk sums, finish), combine backward 2, backward
-    # GEMMs 4, un-permute 1, router backward 5 (weight split, dlogits, dX GEMM, dWg GEMM,
-    # split-K sum), bias step 1
-    permute_launches = 3 if args.gather else 5
+    # scatter; + the row copy, which also zeroes the pad rows, without gathering), forward
+    # GEMMs 2, combine 1; train adds the balance loss 2 (chunk sums, finish), combine
+    # backward 1 (dY pad rows zeroed by the same launch), backward GEMMs 4, un-permute 1,
+    # router backward 5 (weight split, dlogits, dX GEMM, dWg GEMM, split-K sum), bias step 1
+    permute_launches = 3 if args.gather else 4
     launches_per_step = (2 if gate_only else 2 if gemm_only else
-                         2 + permute_launches + 2 + 1 + ((2 + 2 + 4 + 1 + 5 + 1) if train else 0))
+                         2 + permute_launches + 2 + 1 + ((2 + 1 + 4 + 1 + 5 + 1) if train else 0))
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,

@@ -111,12 +111,30 @@ __global__ void combine_kernel_any(const uint4* __restrict__ y, const uint4* __r
   }
 }
 
+// The pads of a local dY: with `pads` set, the launch's last E * kPadSplit CTAs
+// zero the segments' pad rows (the dW GEMMs read them as K rows) while the others
+// scatter.  Not used under expert parallelism, where the owners zero theirs.
+struct DyPads {
+  const GroupRec* groups;  // null: no pad CTAs
+  int E;
+  int* status;
+};
+
 // dy[row_of[t, j]] = w[t, j] dout[t] (bf16);  dw[t, j] = <dout[t], y[row_of[t, j]]>
 __global__ void combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                                    const int32_t* __restrict__ row_of, const float* __restrict__ w,
                                    int64_t T, int row_vec, int k, int64_t Rr,
                                    uint4* __restrict__ dy,
-                                   float* __restrict__ dw, EpDy ep) {
+                                   float* __restrict__ dw, EpDy ep, DyPads pads) {
+  if (pads.groups != nullptr) {
+    const unsigned tok_blocks = gridDim.x - (unsigned)pads.E * kPadSplit;
+    if (blockIdx.x >= tok_blocks) {
+      const int pb = (int)(blockIdx.x - tok_blocks);
+      zero_group_pad_rows(pads.groups, pb / kPadSplit, pb % kPadSplit, row_vec, dy, Rr,
+                          pads.status);
+      return;
+    }
+  }
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   for (int j = 0; t < T && j < k; ++j) {
@@ -155,8 +173,18 @@ template <int VPL>
 __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                                        const int32_t* __restrict__ row_of,
                                        const float* __restrict__ w, int64_t T, int k, int64_t Rr,
-                                       uint4* __restrict__ dy, float* __restrict__ dw, EpDy ep) {
+                                       uint4* __restrict__ dy, float* __restrict__ dw, EpDy ep,
+                                       DyPads pads) {
   constexpr int row_vec = 32 * VPL;
+  if (pads.groups != nullptr) {
+    const unsigned tok_blocks = gridDim.x - (unsigned)pads.E * kPadSplit;
+    if (blockIdx.x >= tok_blocks) {
+      const int pb = (int)(blockIdx.x - tok_blocks);
+      zero_group_pad_rows(pads.groups, pb / kPadSplit, pb % kPadSplit, row_vec, dy, Rr,
+                          pads.status);
+      return;
+    }
+  }
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   uint4 g[VPL];
@@ -199,8 +227,6 @@ __global__ void combine_bwd_reg_kernel(const uint4* __restrict__ dout, const uin
 
 }  // namespace
 
-int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream);
-
 int launch_combine(const moe_dims& dm, const void* y, const void* y_shared,
                    const int32_t* row_of, const float* w, void* out, bool f32_out, void* stream) {
   if (dm.T == 0) return MOE_OK;
@@ -232,35 +258,40 @@ int launch_combine(const moe_dims& dm, const void* y, const void* y_shared,
 
 static int combine_bwd_kernels(const moe_dims& dm, const void* dout, const void* y,
                                const int32_t* row_of, const float* w, void* dy, float* dw,
-                               const EpDy& ep, cudaStream_t st) {
+                               const EpDy& ep, const DyPads& pads, cudaStream_t st) {
   const int warps = 8;
+  const unsigned pad_blocks = pads.groups != nullptr ? (unsigned)dm.E * kPadSplit : 0u;
   // one CTA at least: under expert parallelism the last CTA signals the owners
-  const unsigned blocks = (unsigned)(dm.T > 0 ? (dm.T + warps - 1) / warps : 1);
+  const unsigned blocks = (unsigned)(dm.T > 0 ? (dm.T + warps - 1) / warps : 1) + pad_blocks;
   const int64_t Rr = rows_routed(dm);
   const uint4* dv = reinterpret_cast<const uint4*>(dout);
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* dyv = reinterpret_cast<uint4*>(dy);
   const int row_vec = dm.d / 8;
   // the register-resident form uses ~170 registers a thread: 4-warp CTAs, three per SM
-  const unsigned blocks4 = (unsigned)(dm.T > 0 ? (dm.T + 3) / 4 : 1);
+  const unsigned blocks4 = (unsigned)(dm.T > 0 ? (dm.T + 3) / 4 : 1) + pad_blocks;
   if (row_vec == 512)
     combine_bwd_reg_kernel<16><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, Rr, dyv,
-                                                        dw, ep);
+                                                        dw, ep, pads);
   else if (row_vec == 256)
     combine_bwd_reg_kernel<8><<<blocks4, 128, 0, st>>>(dv, yv, row_of, w, dm.T, dm.k, Rr, dyv,
-                                                       dw, ep);
+                                                       dw, ep, pads);
   else
     combine_bwd_kernel<<<blocks, warps * 32, 0, st>>>(dv, yv, row_of, w, dm.T, row_vec, dm.k, Rr,
-                                                      dyv, dw, ep);
+                                                      dyv, dw, ep, pads);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_combine_bwd(const moe_dims& dm, const void* ws, const void* dout, const void* y,
                        const int32_t* row_of, const float* w, void* dy, float* dw, void* stream) {
-  int rc = launch_zero_pad_rows(dm, ws, dy, dm.d, stream);
-  if (rc != MOE_OK || dm.T == 0) return rc;
+  if (dm.T == 0) return MOE_OK;  // no routed rows, so no pad rows either
   EpDy none{};
-  return combine_bwd_kernels(dm, dout, y, row_of, w, dy, dw, none,
+  DyPads pads{};
+  const uint8_t* wsb = reinterpret_cast<const uint8_t*>(ws);
+  pads.groups = reinterpret_cast<const GroupRec*>(wsb + ws_layout(dm).groups);
+  pads.E = dm.E;
+  pads.status = reinterpret_cast<int*>(const_cast<void*>(ws));
+  return combine_bwd_kernels(dm, dout, y, row_of, w, dy, dw, none, pads,
                              reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -281,7 +312,7 @@ int launch_combine_bwd_ep(const moe_dims& dm, const moe_ep_peers& pe, const void
   ep.done = reinterpret_cast<int*>(epb) + EP_DONE_DY;
   ep.El = dm.E / pe.world;
   ep.W = pe.world;
-  return combine_bwd_kernels(dm, dout, y, row_of, w, nullptr, dw, ep,
+  return combine_bwd_kernels(dm, dout, y, row_of, w, nullptr, dw, ep, DyPads{},
                              reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -39,6 +39,30 @@ struct GroupRec {
   int32_t a_row, out_row, rows, rows_pad;
 };
 
+constexpr int kPadSplit = 8;  // CTAs per routed group zeroing its pad rows
+
+#ifdef __CUDACC__
+// Zero the pad rows [out_row + rows, out_row + rows_pad) of routed group e of a
+// bf16 matrix [Rr, row_vec * 8]; this CTA is part `part` of kPadSplit CTAs on the
+// group.  The debug build reports a record outside the routed rows instead of
+// following it.
+__device__ __forceinline__ void zero_group_pad_rows(const GroupRec* __restrict__ groups, int e,
+                                                    int part, int row_vec, uint4* __restrict__ m,
+                                                    int64_t Rr, int* status) {
+  const GroupRec g = groups[e];
+  const int64_t r0 = (int64_t)g.out_row + g.rows, r1 = (int64_t)g.out_row + g.rows_pad;
+  if (MOE_DEBUG && (g.out_row < 0 || g.rows < 0 || r0 > r1 || r1 > Rr)) {
+    if (threadIdx.x == 0) atomicCAS(status, 0, MOE_ERR_BAD_ROUTING);
+    return;
+  }
+  const int64_t n = (r1 - r0) * row_vec;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (int64_t i = (int64_t)part * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)kPadSplit * blockDim.x)
+    m[r0 * row_vec + i] = z;
+}
+#endif
+
 constexpr int kChunk = 1024;      // routed assignments per histogram chunk
 constexpr int kHeaderWords = 16;  // [0] status, [1] padded routed total, [2] tiles total,
                                   // [3] routing valid, [4] bad expert id seen,

@@ -27,8 +27,6 @@
 namespace moe {
 namespace {
 
-constexpr int kPadSplit = 8;  // CTAs per group zeroing its pad rows
-
 constexpr int kScatterThreads = 256;
 
 __global__ void hist_kernel(const int32_t* __restrict__ idx, int64_t n, int E,
@@ -200,11 +198,20 @@ __global__ void __launch_bounds__(kScatterThreads)
   }
 }
 
-// One warp per token: x[t] is read once and written to its k routed rows.
+// One warp per token: x[t] is read once and written to its k routed rows.  The
+// last E * kPadSplit CTAs zero the segments' pad rows meanwhile (no launch of
+// their own).
 __global__ void copy_rows_kernel(const uint4* __restrict__ x, int64_t T, int row_vec, int k,
                                  const int32_t* __restrict__ row_of, uint4* __restrict__ x_perm,
-                                 const int* header) {
+                                 int* header, const GroupRec* __restrict__ groups, int E,
+                                 int64_t Rr) {
   if (header[3] != 1) return;
+  const unsigned tok_blocks = gridDim.x - (unsigned)E * kPadSplit;
+  if (blockIdx.x >= tok_blocks) {
+    const int pb = (int)(blockIdx.x - tok_blocks);
+    zero_group_pad_rows(groups, pb / kPadSplit, pb % kPadSplit, row_vec, x_perm, Rr, header);
+    return;
+  }
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -232,8 +239,15 @@ __global__ void copy_rows_kernel(const uint4* __restrict__ x, int64_t T, int row
 // Generic version for k > 16 (rows read from row_of on the fly).
 __global__ void copy_rows_kernel_bigk(const uint4* __restrict__ x, int64_t T, int row_vec, int k,
                                       const int32_t* __restrict__ row_of,
-                                      uint4* __restrict__ x_perm, const int* header) {
+                                      uint4* __restrict__ x_perm, int* header,
+                                      const GroupRec* __restrict__ groups, int E, int64_t Rr) {
   if (header[3] != 1) return;
+  const unsigned tok_blocks = gridDim.x - (unsigned)E * kPadSplit;
+  if (blockIdx.x >= tok_blocks) {
+    const int pb = (int)(blockIdx.x - tok_blocks);
+    zero_group_pad_rows(groups, pb / kPadSplit, pb % kPadSplit, row_vec, x_perm, Rr, header);
+    return;
+  }
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -242,25 +256,6 @@ __global__ void copy_rows_kernel_bigk(const uint4* __restrict__ x, int64_t T, in
     const uint4 v = src[c];
     for (int j = 0; j < k; ++j) x_perm[(int64_t)row_of[t * k + j] * row_vec + c] = v;
   }
-}
-
-// Zero the pad rows [off_e + c_e, off_e + roundup(c_e, P)) of every routed
-// segment (of a bf16 [Rr, row_vec * 8] matrix).  grid.x = E.
-__global__ void zero_pad_rows_kernel(const GroupRec* __restrict__ groups, int row_vec,
-                                     uint4* __restrict__ m, int64_t Rr, int* status) {
-  const GroupRec g = groups[blockIdx.x];
-  const int64_t r0 = (int64_t)g.out_row + g.rows, r1 = (int64_t)g.out_row + g.rows_pad;
-  if (MOE_DEBUG && (g.out_row < 0 || g.rows < 0 || r0 > r1 || r1 > Rr)) {
-    // debug build: a group record outside the routed rows is reported, not followed
-    if (threadIdx.x == 0) atomicCAS(status, 0, MOE_ERR_BAD_ROUTING);
-    return;
-  }
-  const int64_t n = (r1 - r0) * row_vec;
-  const uint4 z = make_uint4(0, 0, 0, 0);
-  // blockIdx.y splits one group's pad rows across several CTAs
-  for (int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.y * blockDim.x)
-    m[r0 * row_vec + i] = z;
 }
 
 }  // namespace
@@ -305,18 +300,19 @@ int launch_permute(const moe_dims& dm, const int32_t* idx, const void* x, int32_
     return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
   const int row_vec = dm.d / 8;
   const int warps = 8;
-  const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps);
+  // one warp per token, then E * kPadSplit CTAs for the pad rows
+  const unsigned blocks = (unsigned)((dm.T + warps - 1) / warps + (int64_t)dm.E * kPadSplit);
+  const GroupRec* groups = reinterpret_cast<const GroupRec*>(wsb + L.groups);
   if (dm.k <= 16)
     copy_rows_kernel<<<blocks, warps * 32, 0, st>>>(reinterpret_cast<const uint4*>(x), dm.T,
                                                     row_vec, dm.k, row_of,
-                                                    reinterpret_cast<uint4*>(x_perm), status);
+                                                    reinterpret_cast<uint4*>(x_perm), status,
+                                                    groups, dm.E, Rr);
   else
     copy_rows_kernel_bigk<<<blocks, warps * 32, 0, st>>>(reinterpret_cast<const uint4*>(x), dm.T,
                                                          row_vec, dm.k, row_of,
-                                                         reinterpret_cast<uint4*>(x_perm), status);
-  zero_pad_rows_kernel<<<dim3(dm.E, kPadSplit), 256, 0, st>>>(
-      reinterpret_cast<const GroupRec*>(wsb + L.groups), row_vec, reinterpret_cast<uint4*>(x_perm),
-      Rr, status);
+                                                         reinterpret_cast<uint4*>(x_perm), status,
+                                                         groups, dm.E, Rr);
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -334,13 +330,5 @@ int launch_set_groups(const moe_dims& dm, const int32_t* counts, int32_t* offset
 }
 
 // Zero the pad rows of a routed-space bf16 matrix with `cols` columns.
-int launch_zero_pad_rows(const moe_dims& dm, const void* ws, void* m, int cols, void* stream) {
-  const WsLayout L = ws_layout(dm);
-  const uint8_t* wsb = reinterpret_cast<const uint8_t*>(ws);
-  zero_pad_rows_kernel<<<dim3(dm.E, kPadSplit), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const GroupRec*>(wsb + L.groups), cols / 8, reinterpret_cast<uint4*>(m),
-      rows_routed(dm), reinterpret_cast<int*>(const_cast<uint8_t*>(wsb)));
-  return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
-}
 
 }  // namespace moe
