@@ -18,9 +18,10 @@
 //     the layer workload, one accumulator over all of d = 4096 drifts ~10x
 //     further from the exact logits than an FP32 FMA loop.  So each 64-wide K
 //     block accumulates from zero in tensor memory (12 MMAs over small partial
-//     sums), and the block results are added in FP32 registers with
-//     round-to-nearest; the truncations of different blocks then have random
-//     signs and the logits match an FP32 FMA loop's accuracy.
+//     sums; with E_pad <= 128 the hi products in one set of columns and the mid
+//     and lo products in another), and the block results are added in FP32
+//     registers with round-to-nearest; the truncations of different blocks then
+//     have random signs and the logits match an FP32 FMA loop's accuracy.
 //
 // split_wg_kernel writes the three planes [3][E_pad][d] (bf16, rows E..E_pad-1
 // zero) into the layer workspace.  gate_tc_kernel, one CTA per 128 tokens:
@@ -28,7 +29,12 @@
 //                    and the three E_pad x 64 tiles of the planes, 128-byte swizzle
 //   warp 1           tensor-memory owner; lane 0 issues, per K block, 12 MMAs
 //                    (four 16-wide K steps x hi, mid, lo; M = 128, N = E_pad) into
-//                    one of two E_pad-column accumulators, alternating
+//                    one of two E_pad-column accumulators, alternating.  With
+//                    E_pad <= 128 the hi and mid tiles, consecutive in shared memory,
+//                    form one N = 2 E_pad operand: 8 MMAs, x.hi in the accumulator's
+//                    first E_pad columns and x.mid + x.lo in the next E_pad, which the
+//                    summing warps add (a third fewer MMAs, and X read twice instead
+//                    of three times per K step)
 //   warps 2..9       summing warps (two per tensor-memory lane quarter, one column
 //                    half each): add each finished block accumulator into FP32
 //                    registers, then write the logits to shared memory
@@ -67,7 +73,7 @@ struct GateArgs {
   float* probs;
   int64_t T;
   int d, E, e_pad, k, stages;
-  uint32_t stage_bytes, tmem_cols, idesc;
+  uint32_t stage_bytes, tmem_cols, idesc, idesc2;
   uint64_t budget_ns;
 };
 
@@ -210,7 +216,9 @@ __global__ void split_wg_kernel(const float* __restrict__ wg, int E, int e_pad, 
 // half of the K blocks and CTA 1 the second; each then adds the two partial
 // logits (low half + high half, the same FP32 sum in both) for 64 of the tokens
 // and routes them.  Used when one CTA per tile would leave most SMs idle.
-template <bool SPLIT>
+// PAIRED (E_pad <= 128): the hi and mid planes go through one N = 2 E_pad MMA, and each
+// summing thread keeps two 32-column groups of its row (four otherwise).
+template <bool SPLIT, bool PAIRED>
 __global__ void __launch_bounds__(GT_THREADS, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                    const GateArgs a) {
@@ -225,6 +233,8 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   const int kb0 = (SPLIT && crank) ? nkb_all / 2 : 0;  // this CTA's K blocks [kb0, kb0 + nkb)
   const int nkb = SPLIT ? (crank ? nkb_all - nkb_all / 2 : nkb_all / 2) : nkb_all;
   const uint32_t plane_bytes = (uint32_t)a.e_pad * GT_BK * 2;
+  const int acc_cols = PAIRED ? 2 * a.e_pad : a.e_pad;  // columns of one block accumulator
+  constexpr int NI = PAIRED ? 2 : 4;                     // column groups a summing thread keeps
   volatile int* abort_flag = &ctl->abort_flag;
 
   if (threadIdx.x == 0) {
@@ -256,7 +266,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 
   // Logits of this thread's row, in registers: 32-column groups g = 2 i + h of the
   // accumulator (h = this warp's column half), summed over the K blocks.
-  float sum[4][32];
+  float sum[NI][32];
   const int ngroups = a.e_pad / 32;
   const int q = warp & 3;             // tensor-memory lane quarter of a summing warp
   const int h = (warp - 2) >> 2;      // its column half
@@ -312,16 +322,26 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
                        a.budget_ns))
           break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * a.e_pad);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * acc_cols);
         const uint32_t a_base = smem_u32(smem + (size_t)stage * a.stage_bytes);
         const uint32_t b_base = a_base + GT_A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < GT_BK / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+          if constexpr (PAIRED) {
+            // the hi and mid planes are consecutive E_pad-row tiles: one N = 2 E_pad MMA
+            // puts x.hi in columns [0, E_pad) and x.mid in [E_pad, 2 E_pad); x.lo is added
+            // to the mid columns
+            const uint64_t b01 = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+            const uint64_t b2 = smem_desc_sw128(b_base + 2 * plane_bytes + kk * 32, 16, 1024);
+            umma_f16(d_tmem, ad, b01, a.idesc2, kk != 0 ? 1u : 0u);
+            umma_f16(d_tmem + (uint32_t)a.e_pad, ad, b2, a.idesc, 1u);
+          } else {
 #pragma unroll
-          for (int j = 0; j < 3; ++j) {
-            const uint64_t bd = smem_desc_sw128(b_base + j * plane_bytes + kk * 32, 16, 1024);
-            umma_f16(d_tmem, ad, bd, a.idesc, (kk | j) != 0 ? 1u : 0u);
+            for (int j = 0; j < 3; ++j) {
+              const uint64_t bd = smem_desc_sw128(b_base + j * plane_bytes + kk * 32, 16, 1024);
+              umma_f16(d_tmem, ad, bd, a.idesc, (kk | j) != 0 ? 1u : 0u);
+            }
           }
         }
         umma_commit(&ctl->empty[stage]);
@@ -339,7 +359,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   } else {
     // ----------------------------------------------------- summing warps --
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < NI; ++i)
 #pragma unroll
       for (int j = 0; j < 32; ++j) sum[i][j] = 0.0f;
     for (int kb = 0; kb < nkb; ++kb) {
@@ -350,15 +370,20 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
         break;
       __syncwarp();  // tcgen05.ld is warp-collective
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (uint32_t)(acc * a.e_pad) + ((uint32_t)(q * 32) << 16);
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * acc_cols) + ((uint32_t)(q * 32) << 16);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < NI; ++i) {
         const int g = 2 * i + h;
         if (g < ngroups) {
           uint32_t r[32];
           tmem_ld32_sync(taddr + (uint32_t)(g * 32), r);
 #pragma unroll
           for (int j = 0; j < 32; ++j) sum[i][j] += __uint_as_float(r[j]);
+          if constexpr (PAIRED) {  // the block's mid + lo sums of the same experts
+            tmem_ld32_sync(taddr + (uint32_t)(a.e_pad + g * 32), r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sum[i][j] += __uint_as_float(r[j]);
+          }
         }
       }
       tc_fence_before();
@@ -377,7 +402,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   const int LS = a.E + 1;
   if (warp >= 2 && !aborted) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < NI; ++i) {
       const int g = 2 * i + h;
       if (g < ngroups)
 #pragma unroll
@@ -458,10 +483,12 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
   // the logits tile [128][E + 1] f32 reuses the stage buffers
   if ((size_t)GT_BM * (dm.E + 1) * sizeof(float) > (size_t)stages * a.stage_bytes)
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  uint32_t cols = 32;  // two accumulators of e_pad columns
-  while (cols < (uint32_t)(2 * e_pad)) cols <<= 1;
+  const bool paired = e_pad <= 128;
+  uint32_t cols = 32;  // two accumulators of e_pad (paired: 2 e_pad) columns
+  while (cols < (uint32_t)((paired ? 4 : 2) * e_pad)) cols <<= 1;
   a.tmem_cols = cols;
   a.idesc = idesc_bf16_f32(GT_BM, e_pad, false, false);
+  a.idesc2 = idesc_bf16_f32(GT_BM, 2 * e_pad, false, false);
   a.budget_ns = wait_budget_ns();
 
   CUtensorMap mx{}, mw{};
@@ -472,9 +499,13 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
   static bool attr_set = false;
   static int num_sms = 0;
   if (!attr_set) {
-    if (!cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<false>,
+    if (!cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<false, false>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GT_MAX_SMEM)) ||
-        !cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<true>,
+        !cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<true, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GT_MAX_SMEM)) ||
+        !cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<false, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, GT_MAX_SMEM)) ||
+        !cuda_ok(cudaFuncSetAttribute(gate_tc_kernel<true, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, GT_MAX_SMEM)))
       return MOE_ERR_CUDA;
     int dev = 0;
@@ -497,9 +528,14 @@ int launch_gate_topk(const moe_dims& dm, const void* x, const float* wg, const f
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (!cuda_ok(cudaLaunchKernelEx(&cfg, gate_tc_kernel<true>, mx, mw, a))) return MOE_ERR_CUDA;
+    if (!cuda_ok(cudaLaunchKernelEx(&cfg, paired ? gate_tc_kernel<true, true>
+                                                 : gate_tc_kernel<true, false>,
+                                    mx, mw, a)))
+      return MOE_ERR_CUDA;
+  } else if (paired) {
+    gate_tc_kernel<false, true><<<(unsigned)tiles, GT_THREADS, smem, st>>>(mx, mw, a);
   } else {
-    gate_tc_kernel<false><<<(unsigned)tiles, GT_THREADS, smem, st>>>(mx, mw, a);
+    gate_tc_kernel<false, false><<<(unsigned)tiles, GT_THREADS, smem, st>>>(mx, mw, a);
   }
   return cuda_ok(cudaGetLastError()) ? MOE_OK : MOE_ERR_CUDA;
 }
