@@ -38,9 +38,10 @@
 //   warps 2..9       summing warps (two per tensor-memory lane quarter, one column
 //                    half each): add each finished block accumulator into FP32
 //                    registers, then write the logits to shared memory
-//   all warps        routing, one warp per token: softmax (max-subtracted, expf),
-//                    s = p + bias, k rounds of a warp-shuffle arg-max (equal s ->
-//                    lower index), the renormalised weights
+//   all warps        routing, eight lanes per token (four tokens per warp at a
+//                    time): softmax (max-subtracted, expf), s = p + bias, k rounds of
+//                    a shuffle arg-max within the token's lanes (equal s -> lower
+//                    index), the renormalised weights
 // With fewer 128-token tiles than half the SMs (T <= 9472 on 148 SMs) each tile
 // runs on a cluster pair instead: CTA 0 takes the first half of the K blocks,
 // CTA 1 the second, and after an exchange of partial logits through distributed
@@ -88,67 +89,71 @@ struct GateCtl {
 };
 
 // Routing of the TM tokens whose logits sit in shared memory, row r at L + r * LS:
-// one warp per token.
+// eight lanes per token, four tokens per warp at a time (lane l of a token's group
+// holds experts l, l + 8, ..., EPL of them).  Softmax with the max subtracted, s = p
+// + bias, then k rounds of an arg-max over the group (equal s -> lower index; a NaN
+// score ranks as -inf), the chosen affinities renormalised.  A group reduction is
+// three shuffle steps, and a warp has 3-4 rounds of four tokens in a 128-token tile
+// instead of 13 tokens one after another.
+template <int EPL>
 __device__ __forceinline__ void route_tile(const float* L, int LS, int64_t t0, int TM, int64_t T,
                                            int E, int k, const float* __restrict__ bias,
                                            int32_t* __restrict__ topk_idx,
                                            float* __restrict__ topk_w, float* __restrict__ probs) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int per = (E + 31) / 32;  // experts per lane (<= 8)
-  for (int r = warp; r < TM; r += nwarps) {
+  const int gl = lane & 7;  // this lane's place in its token's group
+  for (int rb = 4 * warp; rb < TM; rb += 4 * nwarps) {
+    const int r = rb + (lane >> 3);
     const int64_t t = t0 + r;
-    if (t >= T) break;
-    float p[8], s[8];
+    const bool active = r < TM && t < T;  // idle groups still join the shuffles
+    float p[EPL], s[EPL];
     float m = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = lane + 32 * q;
-      p[q] = (q < per && e < E) ? L[r * LS + e] : -INFINITY;
+    for (int q = 0; q < EPL; ++q) {
+      const int e = gl + 8 * q;
+      p[q] = (active && e < E) ? L[r * LS + e] : -INFINITY;
       m = fmaxf(m, p[q]);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float z = 0.0f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = lane + 32 * q;
-      p[q] = (q < per && e < E) ? expf(p[q] - m) : 0.0f;
+    for (int q = 0; q < EPL; ++q) {
+      const int e = gl + 8 * q;
+      p[q] = (active && e < E) ? expf(p[q] - m) : 0.0f;
       z += p[q];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    for (int o = 4; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
     const float inv = 1.0f / z;
+    uint32_t alive = 0;  // experts this lane may still pick (a bit per q)
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = lane + 32 * q;
-      const bool valid = q < per && e < E;
+    for (int q = 0; q < EPL; ++q) {
+      const int e = gl + 8 * q;
+      const bool valid = active && e < E;
       p[q] = valid ? p[q] * inv : 0.0f;
       s[q] = valid ? p[q] + (bias ? bias[e] : 0.0f) : -INFINITY;
       if (s[q] != s[q]) s[q] = -INFINITY;  // a NaN score ranks last (ties by index)
       if (valid && probs) probs[t * E + e] = p[q];
+      if (valid) alive |= 1u << q;
     }
     float psel = 0.0f;
-    // experts this lane may still pick (a bit per q); a pick clears its bit
-    uint32_t alive = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < per && lane + 32 * q < E) alive |= 1u << q;
     for (int j = 0; j < k; ++j) {
       // lane-local best: larger s, then lower index (q ascending = index ascending).  The
-      // first live expert is taken before any comparison and NaN scores rank as -inf,
-      // so even non-finite inputs yield k distinct, valid experts.
+      // first live expert is taken before any comparison, so even non-finite inputs
+      // yield k distinct, valid experts.
       float bs = -INFINITY, bp = 0.0f;
       int be = 0x7fffffff;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < EPL; ++q) {
         if (((alive >> q) & 1u) && (be == 0x7fffffff || s[q] > bs)) {
           bs = s[q];
-          be = lane + 32 * q;
+          be = gl + 8 * q;
           bp = p[q];
         }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
+      for (int o = 4; o > 0; o >>= 1) {
         const float os = __shfl_xor_sync(0xffffffffu, bs, o);
         const int oe = __shfl_xor_sync(0xffffffffu, be, o);
         const float op = __shfl_xor_sync(0xffffffffu, bp, o);
@@ -159,17 +164,18 @@ __device__ __forceinline__ void route_tile(const float* L, int LS, int64_t t0, i
         }
       }
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (lane + 32 * q == be) alive &= ~(1u << q);  // remove the winner
+      for (int q = 0; q < EPL; ++q)
+        if (gl + 8 * q == be) alive &= ~(1u << q);  // remove the winner
       psel += bp;
-      if (lane == 0) {
+      if (gl == 0 && active) {
         topk_idx[t * k + j] = be;
         topk_w[t * k + j] = bp;
       }
     }
     __syncwarp();
     const float rn = 1.0f / psel;
-    for (int j = lane; j < k; j += 32) topk_w[t * k + j] *= rn;
+    if (active)
+      for (int j = gl; j < k; j += 8) topk_w[t * k + j] *= rn;
     __syncwarp();
   }
 }
@@ -425,9 +431,14 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     }
     __syncthreads();
   }
-  if (!aborted)
-    route_tile(L + r0 * LS, LS, m0 + r0, rows, a.T, a.E, a.k, a.bias, a.topk_idx, a.topk_w,
-               a.probs);
+  if (!aborted) {
+    if (a.E <= 128)
+      route_tile<16>(L + r0 * LS, LS, m0 + r0, rows, a.T, a.E, a.k, a.bias, a.topk_idx,
+                     a.topk_w, a.probs);
+    else
+      route_tile<32>(L + r0 * LS, LS, m0 + r0, rows, a.T, a.E, a.k, a.bias, a.topk_idx,
+                     a.topk_w, a.probs);
+  }
   if constexpr (SPLIT) cluster_sync();  // the peer has read this CTA's partials
   if (warp == 1) {
     tc_fence_after();
